@@ -1,0 +1,51 @@
+"""The oracle pins must catch plausible mistakes.
+
+Each case plants one slip in a private copy of the oracle's source (on the CPU,
+never in the CUDA path), swaps the copy in, and checks that at least one pin in
+``test_oracle_pins`` fails.
+"""
+import inspect
+import types
+
+import pytest
+
+import oracle
+import oracle.zebra as zebra
+import tests.test_oracle_pins as pins
+
+MUTATIONS = {
+    "bias in log2 units": ("np.log(n[lm].astype(np.float64))", "np.log2(n[lm].astype(np.float64))"),
+    "landmark bias dropped": ("+ np.log(n[lm].astype(np.float64))[None, :]", ""),
+    "landmark value = mean key": ("value_parts.append(Vbar[h, lm])", "value_parts.append(Kbar[h, lm])"),
+    "selected tiles also landmarks": ("mask[sel] = False", "pass"),
+    "ties go to the upper index": ("order = np.lexsort((j, -flat[r]))", "order = np.lexsort((-j, -flat[r]))"),
+    "softmax scale dropped": ("logit_parts = [scale * q @ K[h, cols].T]", "logit_parts = [q @ K[h, cols].T]"),
+    "feature map off by one": ("x + 1.0, np.exp", "x, np.exp"),
+    "fit without intercept": ("D = np.concatenate([X[h], np.ones((R, 1))], axis=1)",
+                              "D = np.concatenate([X[h], np.zeros((R, 1))], axis=1)"),
+    "score transposed": ("np.matmul(Qbar, np.swapaxes(Kbar, -1, -2))",
+                         "np.swapaxes(np.matmul(Qbar, np.swapaxes(Kbar, -1, -2)), -1, -2)"),
+    "ragged tile divided by full size": ("out /= n[None, :, None].astype(np.float64)", "out /= float(tile)"),
+}
+
+
+def _pin_tests():
+    return [f for name, f in inspect.getmembers(pins, inspect.isfunction) if name.startswith("test_")]
+
+
+@pytest.mark.parametrize("name", sorted(MUTATIONS))
+def test_pins_catch_mutation(name, monkeypatch):
+    old, new = MUTATIONS[name]
+    src = inspect.getsource(zebra)
+    assert old in src
+    mod = types.ModuleType("oracle_mutant")
+    exec(compile(src.replace(old, new), "oracle_mutant", "exec"), mod.__dict__)
+    for fn in zebra.__all__:
+        monkeypatch.setattr(oracle, fn, getattr(mod, fn))
+    failures = 0
+    for test in _pin_tests():
+        try:
+            test()
+        except (AssertionError, ValueError, IndexError):
+            failures += 1
+    assert failures > 0, f"no pin catches: {name}"

@@ -1,0 +1,274 @@
+"""Pins for the fp64 oracle: closed forms, invariants, library routines, brute force.
+
+Each test ties one oracle function to something other than itself, chosen so
+that a plausible slip (a dropped term, a wrong sign or index, a transposed
+operand, a wrong log base) fails at least one test.  CPU only.
+"""
+import itertools
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import synth
+
+RNG = np.random.default_rng(12345)
+
+
+def _bf16_grid(shape, std=1.0, rng=RNG):
+    """Random values that are exactly representable in bf16 (as fp64)."""
+    x = torch.from_numpy(rng.standard_normal(shape) * std).to(torch.bfloat16)
+    return x.to(torch.float64).numpy()
+
+
+# ----------------------------------------------------------------- tiles ----
+
+def test_tile_lengths_closed_form():
+    assert oracle.tile_lengths(256, 64).tolist() == [64, 64, 64, 64]
+    n = oracle.tile_lengths(32 * 1374, 128)
+    assert n.shape == (344,) and n[-1] == 43968 - 343 * 128 == 64
+    assert (n[:-1] == 128).all() and n.sum() == 43968
+    assert oracle.tile_lengths(1, 128).tolist() == [1]
+    assert oracle.tile_lengths(1024 * 1374, 128).shape == (10992,)
+
+
+def test_landmark_means_equal_correctly_rounded_sums():
+    X = _bf16_grid((2, 300, 8), std=0.125)
+    got = oracle.landmark_means(X, 64)
+    n = oracle.tile_lengths(300, 64)
+    for h in range(2):
+        for j in range(len(n)):
+            rows = X[h, j * 64: j * 64 + n[j]]
+            for c in range(8):
+                want = math.fsum(rows[:, c].tolist()) / float(n[j])
+                assert got[h, j, c] == want  # bit-exact
+
+
+def test_landmark_means_of_constant_tile():
+    X = np.zeros((1, 200, 4))
+    X[0, :128] = 0.375
+    X[0, 128:] = -1.5
+    got = oracle.landmark_means(X, 128)
+    assert (got[0, 0] == 0.375).all() and (got[0, 1] == -1.5).all()
+
+
+# --------------------------------------------------------------- scoring ----
+
+def test_tile_scores_pick_coordinates():
+    # Qbar rows are basis vectors, so score[i, j] = Kbar[j, i]; a transposed
+    # product or swapped operands gives a different matrix.
+    d = 5
+    Qbar = np.eye(d)[None]
+    Kbar = RNG.standard_normal((1, 7, d))
+    s = oracle.tile_scores(Qbar, Kbar)
+    assert s.shape == (1, d, 7)
+    np.testing.assert_array_equal(s[0], Kbar[0].T)
+
+
+def test_tile_scores_cauchy_schwarz():
+    A = RNG.standard_normal((1, 9, 6))
+    s = oracle.tile_scores(A, A)
+    norms = (A[0] ** 2).sum(-1)
+    np.testing.assert_allclose(np.diag(s[0]), norms, rtol=1e-14)
+    assert (np.abs(s[0]) <= np.sqrt(norms[:, None] * norms[None, :]) * (1 + 1e-14)).all()
+
+
+def test_select_top_k_equals_best_subset_by_brute_force():
+    for trial in range(20):
+        T, k = 7, 3
+        s = RNG.standard_normal(T)
+        best = max(itertools.combinations(range(T), k), key=lambda c: sum(s[list(c)]))
+        got = oracle.select_tiles(s[None], k)[0]
+        assert got.tolist() == sorted(best)
+
+
+def test_select_tie_break_lower_index_and_ascending():
+    row = np.array([[1.0, 3.0, 3.0, 2.0, 3.0]])
+    assert oracle.select_tiles(row, 2)[0].tolist() == [1, 2]
+    assert oracle.select_tiles(row, 3)[0].tolist() == [1, 2, 4]
+    assert oracle.select_tiles(row, 4)[0].tolist() == [1, 2, 3, 4]
+    assert oracle.select_tiles(row, 0)[0].tolist() == []
+    assert oracle.select_tiles(row, 5)[0].tolist() == [0, 1, 2, 3, 4]
+    neg = np.array([[-0.0, 0.0, -1e-300, 1e-300]])
+    assert oracle.select_tiles(neg, 1)[0].tolist() == [3]
+    assert oracle.select_tiles(neg, 3)[0].tolist() == [0, 1, 3]
+
+
+def test_select_keeps_planted_tiles_tiny():
+    w = synth.WORKLOADS["tiny"]
+    Q, K, V = synth.make_qkv(w)
+    Qbar = oracle.landmark_means(synth.to_f64(Q), w.tile)
+    Kbar = oracle.landmark_means(synth.to_f64(K), w.tile)
+    idx = oracle.select_tiles(oracle.tile_scores(Qbar, Kbar), w.k)
+    hh, ii, jj = synth.planted_pairs(w, synth.default_seed(w))
+    for h, i, j in zip(hh, ii, jj):
+        assert j in idx[h, i]
+
+
+# ------------------------------------------------------ softmax attention ----
+
+def _qkv(H, N, d, std=0.5, rng=RNG):
+    return (rng.standard_normal((H, N, d)) * std, rng.standard_normal((H, N, d)) * std,
+            rng.standard_normal((H, N, d)))
+
+
+def test_dense_attention_matches_library_sdpa():
+    Q, K, V = _qkv(2, 37, 8)
+    s = 1 / math.sqrt(8)
+    got = oracle.dense_attention(Q, K, V, s)
+    want = torch.nn.functional.scaled_dot_product_attention(
+        torch.from_numpy(Q)[None], torch.from_numpy(K)[None], torch.from_numpy(V)[None])[0]
+    np.testing.assert_allclose(got, want.numpy(), rtol=1e-12, atol=1e-13)
+
+
+def test_keep_all_tiles_equals_dense():
+    H, N, d, t = 2, 150, 8, 32   # ragged last tile (22 rows)
+    Q, K, V = _qkv(H, N, d)
+    T = oracle.tile_lengths(N, t).shape[0]
+    idx = np.broadcast_to(np.arange(T), (H, T, T))
+    got = oracle.sparse_attention(Q, K, V, t, idx, 0.125, use_landmarks=True)
+    np.testing.assert_allclose(got, oracle.dense_attention(Q, K, V, 0.125), rtol=1e-12, atol=1e-14)
+
+
+def test_tile_length_one_makes_landmarks_exact():
+    H, N, d = 1, 40, 4
+    Q, K, V = _qkv(H, N, d)
+    for k in (0, 1, 7, 40):
+        idx = np.stack([np.sort(RNG.choice(N, size=k, replace=False)) for _ in range(N)])[None]
+        got = oracle.sparse_attention(Q, K, V, 1, idx, 0.3, use_landmarks=True)
+        np.testing.assert_allclose(got, oracle.dense_attention(Q, K, V, 0.3), rtol=1e-12, atol=1e-14)
+
+
+def test_tile_constant_keys_make_landmarks_exact_for_any_selection():
+    # Every row of a key tile is the same vector, so a landmark (mean key, mean
+    # value, bias ln n_j) reproduces the tile's n_j exact keys.  Values are not
+    # tile-constant.  The last tile is ragged.
+    H, N, d, t = 2, 200, 8, 32
+    T = oracle.tile_lengths(N, t).shape[0]
+    Q, _, V = _qkv(H, N, d)
+    Kt = RNG.standard_normal((H, T, d))
+    K = np.repeat(Kt, t, axis=1)[:, :N]
+    dense = oracle.dense_attention(Q, K, V, 0.25)
+    for k in (0, 1, 3, T):
+        idx = np.stack([np.stack([np.sort(RNG.choice(T, size=k, replace=False)) for _ in range(T)])
+                        for _ in range(H)])
+        got = oracle.sparse_attention(Q, K, V, t, idx, 0.25, use_landmarks=True)
+        np.testing.assert_allclose(got, dense, rtol=1e-12, atol=1e-14)
+
+
+def test_landmarks_only_equal_expanded_mean_keys():
+    # k = 0: the output equals dense attention over a key set where each tile's
+    # mean key (with its mean value) is repeated n_j times.
+    H, N, d, t = 1, 90, 6, 16
+    Q, K, V = _qkv(H, N, d)
+    n = oracle.tile_lengths(N, t)
+    Kb, Vb = oracle.landmark_means(K, t), oracle.landmark_means(V, t)
+    Kx = np.repeat(Kb, n, axis=1)
+    Vx = np.repeat(Vb, n, axis=1)
+    idx = np.zeros((H, len(n), 0), dtype=np.int64)
+    got = oracle.sparse_attention(Q, K, V, t, idx, 0.4, use_landmarks=True)
+    np.testing.assert_allclose(got, oracle.dense_attention(Q, Kx, Vx, 0.4), rtol=1e-12, atol=1e-14)
+
+
+def test_no_landmarks_single_tile_is_local_softmax():
+    H, N, d, t = 1, 96, 8, 32
+    Q, K, V = _qkv(H, N, d)
+    T = 3
+    idx = np.array([[[2], [0], [1]]])
+    got = oracle.sparse_attention(Q, K, V, t, idx, 0.5, use_landmarks=False)
+    for i, j in enumerate([2, 0, 1]):
+        want = oracle.dense_attention(Q[:, i * t:(i + 1) * t], K[:, j * t:(j + 1) * t],
+                                      V[:, j * t:(j + 1) * t], 0.5)
+        np.testing.assert_allclose(got[:, i * t:(i + 1) * t], want, rtol=1e-12, atol=1e-14)
+
+
+def test_sparse_output_is_convex_combination():
+    H, N, d, t = 2, 130, 8, 32
+    Q, K, V = _qkv(H, N, d, std=2.0)
+    T = 5
+    idx = np.stack([np.stack([np.sort(RNG.choice(T, size=2, replace=False)) for _ in range(T)])
+                    for _ in range(H)])
+    O = oracle.sparse_attention(Q, K, V, t, idx, 0.125)
+    lo, hi = V.min(axis=1, keepdims=True), V.max(axis=1, keepdims=True)
+    assert (O >= lo - 1e-12).all() and (O <= hi + 1e-12).all()
+
+
+def test_query_tile_subset_matches_full():
+    H, N, d, t = 1, 100, 4, 32
+    Q, K, V = _qkv(H, N, d)
+    T = 4
+    idx = np.stack([np.sort(RNG.choice(T, size=2, replace=False)) for _ in range(T)])[None]
+    full = oracle.sparse_attention(Q, K, V, t, idx, 0.2)
+    sub = oracle.sparse_attention(Q, K, V, t, idx, 0.2, query_tiles=[3, 1])
+    np.testing.assert_array_equal(sub[:, :4], full[:, 96:100])
+    assert (sub[:, 4:32] == 0).all()
+    np.testing.assert_array_equal(sub[:, 32:64], full[:, 32:64])
+
+
+# --------------------------------------------------------- linear stage ----
+
+def test_elu_plus_one_closed_form():
+    x = np.array([-2.0, -0.5, 0.0, 0.5, 3.0])
+    want = [math.exp(-2.0), math.exp(-0.5), 1.0, 1.5, 4.0]
+    assert oracle.elu_plus_one(x).tolist() == want
+    assert (oracle.elu_plus_one(np.linspace(-30, 30, 101)) > 0).all()
+
+
+def test_linear_associative_equals_quadratic():
+    Q, K, V = _qkv(2, 50, 8, std=1.0)
+    np.testing.assert_allclose(oracle.linear_attention(Q, K, V),
+                               oracle.linear_attention_quadratic(Q, K, V), rtol=1e-12, atol=1e-13)
+
+
+def test_linear_zero_keys_give_mean_value():
+    Q, _, V = _qkv(1, 30, 4)
+    O = oracle.linear_attention(Q, np.zeros_like(Q), V)
+    np.testing.assert_allclose(O, np.broadcast_to(V.mean(axis=1, keepdims=True), O.shape), rtol=1e-13)
+
+
+def test_linear_state_single_token():
+    Q, K, V = _qkv(1, 1, 4)
+    S, z = oracle.linear_state(K, V)
+    phik = oracle.elu_plus_one(K[0, 0])
+    np.testing.assert_allclose(S[0], np.outer(phik, V[0, 0]), rtol=1e-15)
+    np.testing.assert_allclose(z[0], phik, rtol=1e-15)
+    np.testing.assert_allclose(oracle.linear_attention(Q, K, V)[0, 0], V[0, 0], rtol=1e-14)
+
+
+# ----------------------------------------------------------- affine fit ----
+
+def test_affine_fit_recovers_planted_map():
+    H, R, d = 3, 400, 8
+    X = RNG.standard_normal((H, R, d))
+    A0 = RNG.standard_normal((H, d, d))
+    b0 = RNG.standard_normal((H, d))
+    Y = oracle.affine_apply(X, A0, b0)
+    A, b = oracle.affine_fit(X, Y)
+    np.testing.assert_allclose(A, A0, rtol=0, atol=1e-10)
+    np.testing.assert_allclose(b, b0, rtol=0, atol=1e-10)
+
+
+def test_affine_fit_identity():
+    X = RNG.standard_normal((2, 100, 6))
+    A, b = oracle.affine_fit(X, X)
+    np.testing.assert_allclose(A, np.broadcast_to(np.eye(6), A.shape), atol=1e-12)
+    np.testing.assert_allclose(b, 0, atol=1e-12)
+
+
+def test_affine_fit_residual_orthogonal_to_design():
+    X = RNG.standard_normal((2, 300, 5))
+    Y = RNG.standard_normal((2, 300, 5))
+    A, b = oracle.affine_fit(X, Y)
+    E = Y - oracle.affine_apply(X, A, b)
+    for h in range(2):
+        D = np.concatenate([X[h], np.ones((300, 1))], axis=1)
+        np.testing.assert_allclose(D.T @ E[h], 0, atol=1e-10)
+
+
+def test_calibration_rows():
+    rows = oracle.calibration_rows(200, 64, [3, 0])
+    assert rows.tolist() == list(range(192, 200)) + list(range(0, 64))
+    assert synth.calibration_tiles(2748, 32)[:3].tolist() == [0, 85, 171]
+    assert synth.calibration_tiles(4, None).tolist() == [0, 1, 2, 3]
