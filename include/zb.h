@@ -1,0 +1,219 @@
+/*
+ * zb.h -- C ABI of the Zebra3D hybrid global-attention layer for NVIDIA B200
+ * (sm_100a).  Library: linear_hybrid_attention_b200/libzb.so.
+ *
+ * The layer has two stage types.  A sensitive stage runs tile-sparse softmax
+ * attention: every query tile keeps exact softmax over its top-k key tiles and
+ * each omitted key tile is folded into one mean-key/mean-value landmark.  A
+ * tolerant stage runs linear attention whose output is mapped by a per-head
+ * affine (A, b) fitted in closed form to the dense output.  Sources (by page
+ * title): "Zebra3D: Efficient Hybrid Foundation Models For Scalable 3D
+ * Reconstruction" -- Abstract and Figure 1 (a) caption; "Zebra3D speeds up 3D
+ * reconstruction by up to 7.1x on 1024 frames without training from scratch"
+ * -- section "How Zebra3D works".
+ *
+ * Conventions shared by every call
+ * --------------------------------
+ *  - Tensors are DEVICE pointers, row-major and contiguous.  Q, K, V, O are
+ *    [heads][n_tokens][head_dim]; bf16 values are passed as their uint16_t bit
+ *    patterns.  Every pointer must be 16-byte aligned.
+ *  - The caller owns every buffer.  The library allocates no device memory,
+ *    frees nothing it did not allocate, and keeps no reference after return.
+ *  - Every compute call is asynchronous on `stream` (a cudaStream_t passed as
+ *    void*; NULL = the legacy default stream).  Arguments are validated on the
+ *    host before anything is launched: a bad argument returns an error code and
+ *    launches nothing.  A failed launch returns ZB_ERR_CUDA.  No call aborts or
+ *    exits the process.
+ *  - Device-side problems (a bounded wait that ran out, an index list that is
+ *    out of range or not strictly ascending, a singular fit) are recorded in a
+ *    per-device status word that zb_last_device_status() reports.
+ *  - head_dim must be 64; tile must be 64 or 128.  Batch > 1 is folded into
+ *    heads.
+ *  - Tiles are contiguous runs of `tile` tokens of the flattened
+ *    [views x tokens] order; T = ceil(n_tokens / tile); the last tile holds
+ *    n_tokens - (T-1)*tile tokens.
+ */
+#ifndef ZB_H
+#define ZB_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum zb_status {
+    ZB_OK = 0,
+    ZB_ERR_NULL = 1,        /* a required pointer is NULL                         */
+    ZB_ERR_SHAPE = 2,       /* a size or count is out of range                    */
+    ZB_ERR_ALIGN = 3,       /* a pointer is not 16-byte aligned                   */
+    ZB_ERR_UNSUPPORTED = 4, /* head_dim != 64, tile not 64/128, too many tiles    */
+    ZB_ERR_WORKSPACE = 5,   /* workspace pointer NULL or smaller than required    */
+    ZB_ERR_CUDA = 6,        /* a CUDA runtime call or a kernel launch failed      */
+    ZB_ERR_TIMEOUT = 7,     /* a bounded device-side wait gave up (device status) */
+    ZB_ERR_DEVICE = 8,      /* the current device is not an sm_100 GPU            */
+    ZB_ERR_INDEX = 9,       /* an index list was out of range / not ascending     */
+    ZB_ERR_SINGULAR = 10    /* a least-squares system was not positive definite   */
+} zb_status;
+
+typedef struct zb_shape {
+    int32_t heads;    /* H >= 1                                   */
+    int64_t n_tokens; /* N >= 1, views x tokens_per_view          */
+    int32_t head_dim; /* d, must be 64                            */
+    int32_t tile;     /* t, 64 or 128                             */
+} zb_shape;
+
+/* Version of this ABI (major * 100 + minor). */
+int32_t zb_abi_version(void);
+
+/* Human-readable name of a zb_status value (static string, never NULL). */
+const char* zb_status_string(int32_t status);
+
+/*
+ * Landmarks: the per-tile means of Q, K and V.
+ * Figure 1 (a) caption of "Zebra3D: Efficient Hybrid Foundation Models ...":
+ * an omitted key tile is replaced by its mean key and mean value.  The mean
+ * query of a tile is the pooled query used for tile scoring.
+ *   in : Q, K, V      bf16 [H][N][d]
+ *   out: Qbar, Kbar   fp64 [H][T][d]  means, summed in fp64 (exact for bf16
+ *                     inputs unless a tile's values span > ~38 binades)
+ *        Kbar_bf16, Vbar_bf16  bf16 [H][T][d]  the means rounded to nearest
+ *                     even, in the layout zb_tile_sparse_attn reads
+ *   Q and Qbar may both be NULL (no query pooling).
+ * Errors: ZB_ERR_NULL, ZB_ERR_SHAPE, ZB_ERR_ALIGN, ZB_ERR_UNSUPPORTED, ZB_ERR_CUDA.
+ */
+zb_status zb_landmark_build(const uint16_t* Q, const uint16_t* K, const uint16_t* V,
+                            zb_shape s, double* Qbar, double* Kbar,
+                            uint16_t* Kbar_bf16, uint16_t* Vbar_bf16, void* stream);
+
+/*
+ * Tile selection: for every (head h, query tile i) the k key tiles j with the
+ * largest score Qbar[h,i] . Kbar[h,j] (fp64 dot products), equal scores going
+ * to the lower j; the kept set is written in ascending order.  The pages name
+ * "selected tiles" (Figure 1 (a) caption) without the criterion; this is the
+ * mean-pooled reading.  The budget k is the kept share of the key tiles (the
+ * y in "xL/yS" of the Table 20 caption is the dropped share).
+ *   in : Qbar, Kbar fp64 [H][T][d];  0 <= k <= T
+ *   out: idx int32 [H][T][k]
+ * Needs no workspace.  Errors: ZB_ERR_NULL, ZB_ERR_SHAPE, ZB_ERR_ALIGN,
+ * ZB_ERR_UNSUPPORTED (T > 32768), ZB_ERR_CUDA.
+ */
+zb_status zb_tile_score_topk(const double* Qbar, const double* Kbar, zb_shape s,
+                             int32_t k, int32_t* idx, void* stream);
+
+/*
+ * Tile-sparse softmax attention with landmarks (Figure 1 (a) caption; section
+ * "How Zebra3D works").  For query row r of tile i, softmax runs over
+ *   - every key of each selected tile j in idx[h][i] (logit scale * q.k), and
+ *   - if use_landmarks != 0, one landmark per unselected tile j with logit
+ *     scale * q.Kbar_bf16[h][j] + ln(n_j) and value Vbar_bf16[h][j];
+ * O_r is the softmax-weighted sum of the matching values.  bf16 tensor-core
+ * products, fp32 accumulation and softmax, O rounded to bf16.
+ *   in : Q, K, V bf16 [H][N][d];  Kbar_bf16, Vbar_bf16 bf16 [H][T][d] (may be
+ *        NULL when use_landmarks == 0);  idx int32 [H][T][k], each row strictly
+ *        ascending in [0, T) (checked on the device: ZB_ERR_INDEX);  0 <= k <= T
+ *        (k == 0 needs use_landmarks);  scale > 0 (usually 1/sqrt(d)).
+ *   out: O bf16 [H][N][d];  lse fp32 [H][N] natural-log log-sum-exp of each
+ *        row's logits (may be NULL).
+ * Errors: ZB_ERR_NULL, ZB_ERR_SHAPE, ZB_ERR_ALIGN, ZB_ERR_UNSUPPORTED (T > 32768),
+ * ZB_ERR_CUDA.
+ */
+zb_status zb_tile_sparse_attn(const uint16_t* Q, const uint16_t* K, const uint16_t* V,
+                              const uint16_t* Kbar_bf16, const uint16_t* Vbar_bf16,
+                              const int32_t* idx, int32_t k, int32_t use_landmarks,
+                              float scale, zb_shape s, uint16_t* O, float* lse,
+                              void* stream);
+
+/*
+ * Dense softmax attention softmax(scale * Q K^T) V: the unconverted layer the
+ * pages compare against, and the target Y of the affine fit.  Same kernel as
+ * zb_tile_sparse_attn with every key tile kept and no landmarks; queries and
+ * keys may have different lengths.
+ *   in : Q bf16 [H][n_q][d];  K, V bf16 [H][n_kv][d]
+ *   out: O bf16 [H][n_q][d];  lse fp32 [H][n_q] (may be NULL)
+ * Errors: ZB_ERR_NULL, ZB_ERR_SHAPE, ZB_ERR_ALIGN, ZB_ERR_UNSUPPORTED, ZB_ERR_CUDA.
+ */
+zb_status zb_dense_attn(const uint16_t* Q, int64_t n_q, const uint16_t* K,
+                        const uint16_t* V, int64_t n_kv, int32_t heads,
+                        int32_t head_dim, float scale, uint16_t* O, float* lse,
+                        void* stream);
+
+/*
+ * Linear-attention state (Abstract: linear attention for tolerant stages):
+ *   S[h] = sum_r phi(k_r)^T v_r  (d x d),  z[h] = sum_r phi(k_r)  (d),
+ * phi(x) = elu(x) + 1, non-causal over all N tokens.  phi(k) is rounded to
+ * bf16 for the tensor-core product; sums are fp32 and the per-CTA partials are
+ * added in a fixed order (deterministic).
+ *   in : K, V bf16 [H][N][d];  ws of >= zb_linear_state_workspace_bytes() bytes
+ *   out: S fp32 [H][d][d] (row index = feature of phi(k), column = value dim),
+ *        z fp32 [H][d]
+ * Errors: ZB_ERR_NULL, ZB_ERR_SHAPE, ZB_ERR_ALIGN, ZB_ERR_UNSUPPORTED,
+ * ZB_ERR_WORKSPACE, ZB_ERR_CUDA.
+ */
+size_t zb_linear_state_workspace_bytes(int32_t heads, int64_t n_tokens, int32_t head_dim);
+zb_status zb_linear_state(const uint16_t* K, const uint16_t* V, int32_t heads,
+                          int64_t n_tokens, int32_t head_dim, float* S, float* z,
+                          void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * Linear-attention output with the per-head affine map (section "How Zebra3D
+ * works": the linear parts are corrected by a closed-form affine map):
+ *   O_r = (phi(q_r) S / (phi(q_r) . z)) A + b      (row vectors)
+ * computed as phi(q_r) (S A) / (phi(q_r) . z) + b: S A and z are rounded to
+ * bf16 for the tensor-core product, the division and + b are fp32.
+ *   in : Q bf16 [H][n_q][d];  S fp32 [H][d][d];  z fp32 [H][d];
+ *        A fp32 [H][d][d] or NULL (identity);  b fp32 [H][d] or NULL (zero)
+ *   out: O bf16 [H][n_q][d]
+ * Errors: ZB_ERR_NULL, ZB_ERR_SHAPE, ZB_ERR_ALIGN, ZB_ERR_UNSUPPORTED, ZB_ERR_CUDA.
+ */
+zb_status zb_linear_apply(const uint16_t* Q, int32_t heads, int64_t n_q,
+                          int32_t head_dim, const float* S, const float* z,
+                          const float* A, const float* b, uint16_t* O, void* stream);
+
+/*
+ * Closed-form affine fit (Abstract: closed-form affine fitting makes the
+ * conversion training-free; Table 3 (a) of "Zebra3D: Efficient Hybrid
+ * Foundation Models ..." compares no fit with fitted variants): per head, the
+ * least-squares solution of [X 1] [A; b] = Y over R calibration rows.  Solved
+ * in fp64: row means, centred Gram matrices, Cholesky factorisation.
+ *   in : X bf16 [H][R][d] (unfitted linear output), Y bf16 [H][R][d] (dense
+ *        output on the same rows);  R >= d + 1;  ws of >=
+ *        zb_affine_fit_workspace_bytes() bytes
+ *   out: A fp32 [H][d][d], b fp32 [H][d]
+ * A system that is not positive definite sets ZB_ERR_SINGULAR in the device
+ * status and writes NaN into that head's A and b.
+ * Errors: ZB_ERR_NULL, ZB_ERR_SHAPE, ZB_ERR_ALIGN, ZB_ERR_UNSUPPORTED,
+ * ZB_ERR_WORKSPACE, ZB_ERR_CUDA.
+ */
+size_t zb_affine_fit_workspace_bytes(int32_t heads, int64_t rows, int32_t head_dim);
+zb_status zb_affine_fit(const uint16_t* X, const uint16_t* Y, int32_t heads,
+                        int64_t rows, int32_t head_dim, float* A, float* b,
+                        void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * Copy whole tiles of a [H][N][d] bf16 tensor into a compact buffer (the
+ * calibration rows of the affine fit are whole query tiles).
+ *   in : X bf16 [H][N][d];  tiles int32 [n_tiles] DEVICE array, each in [0, T)
+ *   out: out bf16 [H][n_tiles * tile][d]; tile m of the list lands in rows
+ *        [m*tile, (m+1)*tile); rows past N of a ragged tile are zero.
+ * An index out of range sets ZB_ERR_INDEX in the device status (its rows are
+ * zero).  Errors: ZB_ERR_NULL, ZB_ERR_SHAPE, ZB_ERR_ALIGN, ZB_ERR_UNSUPPORTED,
+ * ZB_ERR_CUDA.
+ */
+zb_status zb_gather_tiles(const uint16_t* X, zb_shape s, const int32_t* tiles,
+                          int32_t n_tiles, uint16_t* out, void* stream);
+
+/*
+ * Synchronise `stream`, then report and clear the current device's status
+ * word: ZB_OK, or the first of ZB_ERR_TIMEOUT / ZB_ERR_INDEX / ZB_ERR_SINGULAR
+ * recorded by a kernel since the last call.  ZB_ERR_CUDA if the stream or the
+ * device reports an error.
+ */
+zb_status zb_last_device_status(void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* ZB_H */

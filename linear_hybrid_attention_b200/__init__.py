@@ -1,0 +1,344 @@
+"""Zebra3D hybrid global-attention layer for NVIDIA B200 (sm_100a).
+
+Thin Python binding of the C ABI in ``include/zb.h`` (``libzb.so``).  The
+functions below carry the C names; they only marshal arguments: check tensors,
+allocate outputs with PyTorch (device memory and the current stream are the
+only things PyTorch provides), call the library, and raise ``ZbError`` on a
+non-zero status.  Every step of the layer runs in the library's CUDA kernels;
+there is no CPU fallback -- without the library or a CUDA device the calls
+raise.
+
+The layer ("Zebra3D: Efficient Hybrid Foundation Models For Scalable 3D
+Reconstruction", Abstract and Figure 1 (a) caption):
+  * tile-sparse stage: landmarks -> tile selection -> tile-sparse softmax
+    attention with mean-key/value landmarks for the omitted tiles;
+  * linear stage: elu+1 linear attention -> closed-form affine map fitted to
+    the dense output on calibration rows.
+"""
+from __future__ import annotations
+
+import math
+from typing import NamedTuple, Optional, Sequence
+
+import torch
+
+from . import _lib
+
+__all__ = [
+    "ZbError", "Landmarks", "zb_abi_version", "zb_landmark_build", "zb_tile_score_topk",
+    "zb_tile_sparse_attn", "zb_dense_attn", "zb_linear_state", "zb_linear_apply",
+    "zb_affine_fit", "zb_gather_tiles", "zb_last_device_status", "HybridLayer",
+    "LAUNCHES_PER_CALL",
+]
+
+HEAD_DIM = 64
+
+# kernels each entry point launches (for counting launches in a timed region)
+LAUNCHES_PER_CALL = {
+    "zb_landmark_build": 1, "zb_tile_score_topk": 1, "zb_tile_sparse_attn": 1, "zb_dense_attn": 1,
+    "zb_linear_state": 2, "zb_linear_apply": 1, "zb_affine_fit": 3, "zb_gather_tiles": 1,
+}
+
+
+class ZbError(RuntimeError):
+    """A libzb call returned a non-zero zb_status."""
+
+    def __init__(self, what: str, status: int):
+        self.status = status
+        name = _lib.STATUS.get(status, str(status))
+        super().__init__(f"{what} failed: {name}")
+
+
+class Landmarks(NamedTuple):
+    Qbar: torch.Tensor       # fp64 [H, T, d]
+    Kbar: torch.Tensor       # fp64 [H, T, d]
+    Kbar_bf16: torch.Tensor  # bf16 [H, T, d]
+    Vbar_bf16: torch.Tensor  # bf16 [H, T, d]
+
+
+def _lib_handle():
+    return _lib.load()
+
+
+def _check(status: int, what: str) -> None:
+    if status != 0:
+        raise ZbError(what, status)
+
+
+def _stream() -> int:
+    return torch.cuda.current_stream().cuda_stream
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    return None if t is None else t.data_ptr()
+
+
+def _need(t: torch.Tensor, dtype: torch.dtype, name: str, ndim: int) -> None:
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor (libzb has no CPU path)")
+    if t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if t.dim() != ndim:
+        raise ValueError(f"{name} must have {ndim} dims, got {tuple(t.shape)}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+
+
+def _out(shape, dtype, device, out: Optional[torch.Tensor], name: str) -> torch.Tensor:
+    if out is None:
+        return torch.empty(shape, dtype=dtype, device=device)
+    _need(out, dtype, name, len(shape))
+    if tuple(out.shape) != tuple(shape):
+        raise ValueError(f"{name} must have shape {tuple(shape)}, got {tuple(out.shape)}")
+    return out
+
+
+def n_tiles(n_tokens: int, tile: int) -> int:
+    return -(-n_tokens // tile)
+
+
+def zb_abi_version() -> int:
+    return int(_lib_handle().zb_abi_version())
+
+
+def zb_landmark_build(Q: Optional[torch.Tensor], K: torch.Tensor, V: torch.Tensor, tile: int,
+                      out: Optional[Landmarks] = None) -> Landmarks:
+    """Per-tile means of Q, K, V (see zb.h).  Q may be None (no Qbar)."""
+    _need(K, torch.bfloat16, "K", 3)
+    _need(V, torch.bfloat16, "V", 3)
+    if Q is not None:
+        _need(Q, torch.bfloat16, "Q", 3)
+    H, N, d = K.shape
+    T = n_tiles(N, tile)
+    o = out or Landmarks(None, None, None, None)
+    Qbar = None if Q is None else _out((H, T, d), torch.float64, K.device, o.Qbar, "Qbar")
+    Kbar = _out((H, T, d), torch.float64, K.device, o.Kbar, "Kbar")
+    Kb = _out((H, T, d), torch.bfloat16, K.device, o.Kbar_bf16, "Kbar_bf16")
+    Vb = _out((H, T, d), torch.bfloat16, K.device, o.Vbar_bf16, "Vbar_bf16")
+    st = _lib_handle().zb_landmark_build(_ptr(Q), _ptr(K), _ptr(V), _lib.ZbShape(H, N, d, tile),
+                                         _ptr(Qbar), _ptr(Kbar), _ptr(Kb), _ptr(Vb), _stream())
+    _check(st, "zb_landmark_build")
+    return Landmarks(Qbar, Kbar, Kb, Vb)
+
+
+def zb_tile_score_topk(Qbar: torch.Tensor, Kbar: torch.Tensor, n_tokens: int, tile: int, k: int,
+                       out: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """Indices [H, T, k] (int32, ascending) of the k best key tiles per query tile."""
+    _need(Qbar, torch.float64, "Qbar", 3)
+    _need(Kbar, torch.float64, "Kbar", 3)
+    H, T, d = Kbar.shape
+    idx = _out((H, T, k), torch.int32, Kbar.device, out, "idx")
+    st = _lib_handle().zb_tile_score_topk(_ptr(Qbar), _ptr(Kbar), _lib.ZbShape(H, n_tokens, d, tile),
+                                          int(k), _ptr(idx), _stream())
+    _check(st, "zb_tile_score_topk")
+    return idx
+
+
+def zb_tile_sparse_attn(Q, K, V, Kbar_bf16, Vbar_bf16, idx, k: int, tile: int,
+                        use_landmarks: bool = True, scale: Optional[float] = None,
+                        out: Optional[torch.Tensor] = None, lse: Optional[torch.Tensor] = None,
+                        want_lse: bool = False):
+    """Tile-sparse softmax attention with landmarks; returns O (and lse if asked)."""
+    for t, n in ((Q, "Q"), (K, "K"), (V, "V")):
+        _need(t, torch.bfloat16, n, 3)
+    H, N, d = Q.shape
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    if idx is not None:
+        _need(idx, torch.int32, "idx", 3)
+    if use_landmarks:
+        if Kbar_bf16 is not None:
+            _need(Kbar_bf16, torch.bfloat16, "Kbar_bf16", 3)
+        if Vbar_bf16 is not None:
+            _need(Vbar_bf16, torch.bfloat16, "Vbar_bf16", 3)
+    O = _out((H, N, d), torch.bfloat16, Q.device, out, "O")
+    if want_lse or lse is not None:
+        lse = _out((H, N), torch.float32, Q.device, lse, "lse")
+    st = _lib_handle().zb_tile_sparse_attn(
+        _ptr(Q), _ptr(K), _ptr(V), _ptr(Kbar_bf16 if use_landmarks else None),
+        _ptr(Vbar_bf16 if use_landmarks else None), _ptr(idx), int(k), 1 if use_landmarks else 0,
+        float(scale), _lib.ZbShape(H, N, d, tile), _ptr(O), _ptr(lse), _stream())
+    _check(st, "zb_tile_sparse_attn")
+    return (O, lse) if lse is not None else O
+
+
+def zb_dense_attn(Q, K, V, scale: Optional[float] = None, out: Optional[torch.Tensor] = None,
+                  lse: Optional[torch.Tensor] = None, want_lse: bool = False):
+    """Dense softmax attention softmax(scale Q K^T) V on the tensor cores."""
+    for t, n in ((Q, "Q"), (K, "K"), (V, "V")):
+        _need(t, torch.bfloat16, n, 3)
+    H, Nq, d = Q.shape
+    Nk = K.shape[1]
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    O = _out((H, Nq, d), torch.bfloat16, Q.device, out, "O")
+    if want_lse or lse is not None:
+        lse = _out((H, Nq), torch.float32, Q.device, lse, "lse")
+    st = _lib_handle().zb_dense_attn(_ptr(Q), Nq, _ptr(K), _ptr(V), Nk, H, d, float(scale), _ptr(O),
+                                     _ptr(lse), _stream())
+    _check(st, "zb_dense_attn")
+    return (O, lse) if lse is not None else O
+
+
+def linear_state_workspace_bytes(heads: int, n_tokens: int, head_dim: int = HEAD_DIM) -> int:
+    return int(_lib_handle().zb_linear_state_workspace_bytes(heads, n_tokens, head_dim))
+
+
+def affine_fit_workspace_bytes(heads: int, rows: int, head_dim: int = HEAD_DIM) -> int:
+    return int(_lib_handle().zb_affine_fit_workspace_bytes(heads, rows, head_dim))
+
+
+def _ws(nbytes: int, device, ws: Optional[torch.Tensor]) -> torch.Tensor:
+    if ws is not None and ws.numel() * ws.element_size() >= nbytes:
+        return ws
+    return torch.empty(max(nbytes, 16), dtype=torch.uint8, device=device)
+
+
+def zb_linear_state(K, V, S: Optional[torch.Tensor] = None, z: Optional[torch.Tensor] = None,
+                    ws: Optional[torch.Tensor] = None):
+    """S = phi(K)^T V [H, d, d] and z = sum phi(K) [H, d] (fp32)."""
+    _need(K, torch.bfloat16, "K", 3)
+    _need(V, torch.bfloat16, "V", 3)
+    H, N, d = K.shape
+    S = _out((H, d, d), torch.float32, K.device, S, "S")
+    z = _out((H, d), torch.float32, K.device, z, "z")
+    need = linear_state_workspace_bytes(H, N, d)
+    ws = _ws(need, K.device, ws)
+    st = _lib_handle().zb_linear_state(_ptr(K), _ptr(V), H, N, d, _ptr(S), _ptr(z), _ptr(ws),
+                                       ws.numel() * ws.element_size(), _stream())
+    _check(st, "zb_linear_state")
+    return S, z
+
+
+def zb_linear_apply(Q, S, z, A: Optional[torch.Tensor] = None, b: Optional[torch.Tensor] = None,
+                    out: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """O = (phi(Q) S / (phi(Q) . z)) A + b (bf16)."""
+    _need(Q, torch.bfloat16, "Q", 3)
+    _need(S, torch.float32, "S", 3)
+    _need(z, torch.float32, "z", 2)
+    if A is not None:
+        _need(A, torch.float32, "A", 3)
+    if b is not None:
+        _need(b, torch.float32, "b", 2)
+    H, N, d = Q.shape
+    O = _out((H, N, d), torch.bfloat16, Q.device, out, "O")
+    st = _lib_handle().zb_linear_apply(_ptr(Q), H, N, d, _ptr(S), _ptr(z), _ptr(A), _ptr(b), _ptr(O),
+                                       _stream())
+    _check(st, "zb_linear_apply")
+    return O
+
+
+def zb_affine_fit(X, Y, A: Optional[torch.Tensor] = None, b: Optional[torch.Tensor] = None,
+                  ws: Optional[torch.Tensor] = None):
+    """Least-squares [A; b] of [X 1] [A; b] = Y per head (X, Y bf16 [H, R, d])."""
+    _need(X, torch.bfloat16, "X", 3)
+    _need(Y, torch.bfloat16, "Y", 3)
+    H, R, d = X.shape
+    A = _out((H, d, d), torch.float32, X.device, A, "A")
+    b = _out((H, d), torch.float32, X.device, b, "b")
+    ws = _ws(affine_fit_workspace_bytes(H, R, d), X.device, ws)
+    st = _lib_handle().zb_affine_fit(_ptr(X), _ptr(Y), H, R, d, _ptr(A), _ptr(b), _ptr(ws),
+                                     ws.numel() * ws.element_size(), _stream())
+    _check(st, "zb_affine_fit")
+    return A, b
+
+
+def zb_gather_tiles(X, tile: int, tiles: torch.Tensor, out: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """Whole tiles of X [H, N, d] (tile indices: int32 CUDA tensor) -> [H, n*tile, d]."""
+    _need(X, torch.bfloat16, "X", 3)
+    _need(tiles, torch.int32, "tiles", 1)
+    H, N, d = X.shape
+    n = tiles.numel()
+    O = _out((H, n * tile, d), torch.bfloat16, X.device, out, "out")
+    st = _lib_handle().zb_gather_tiles(_ptr(X), _lib.ZbShape(H, N, d, tile), _ptr(tiles), n, _ptr(O),
+                                       _stream())
+    _check(st, "zb_gather_tiles")
+    return O
+
+
+def zb_last_device_status() -> None:
+    """Synchronise the current stream and raise if a kernel recorded a device-side error."""
+    st = _lib_handle().zb_last_device_status(_stream())
+    _check(st, "device status")
+
+
+class HybridLayer:
+    """Preallocated buffers for one hybrid global-attention layer shape.
+
+    ``sparse(Q, K, V)`` runs the tile-sparse stage (landmarks, selection,
+    attention), ``calibrate(Q, K, V)`` fits (A, b) of the linear stage against
+    dense attention on whole calibration tiles, ``linear(Q, K, V)`` runs the
+    fitted linear stage.  Outputs live in the object's buffers and are
+    overwritten by the next call.
+    """
+
+    def __init__(self, heads: int, n_tokens: int, tile: int, k: int, calib_tiles: Sequence[int],
+                 device="cuda", scale: Optional[float] = None):
+        d = HEAD_DIM
+        self.heads, self.n_tokens, self.tile, self.k, self.d = heads, n_tokens, tile, k, d
+        self.T = n_tiles(n_tokens, tile)
+        self.scale = 1.0 / math.sqrt(d) if scale is None else scale
+        dev = torch.device(device)
+        H, N, T = heads, n_tokens, self.T
+        self.lm = Landmarks(torch.empty(H, T, d, dtype=torch.float64, device=dev),
+                            torch.empty(H, T, d, dtype=torch.float64, device=dev),
+                            torch.empty(H, T, d, dtype=torch.bfloat16, device=dev),
+                            torch.empty(H, T, d, dtype=torch.bfloat16, device=dev))
+        self.idx = torch.empty(H, T, k, dtype=torch.int32, device=dev)
+        self.O_sparse = torch.empty(H, N, d, dtype=torch.bfloat16, device=dev)
+        self.O_linear = torch.empty(H, N, d, dtype=torch.bfloat16, device=dev)
+        self.S = torch.empty(H, d, d, dtype=torch.float32, device=dev)
+        self.z = torch.empty(H, d, dtype=torch.float32, device=dev)
+        self.ws_lin = torch.empty(max(linear_state_workspace_bytes(H, N, d), 16), dtype=torch.uint8, device=dev)
+        self.calib = torch.as_tensor(list(calib_tiles), dtype=torch.int32).to(dev)
+        R = len(calib_tiles) * tile
+        self.R = R
+        self.Qc = torch.empty(H, R, d, dtype=torch.bfloat16, device=dev)
+        self.Xc = torch.empty(H, R, d, dtype=torch.bfloat16, device=dev)
+        self.Yc = torch.empty(H, R, d, dtype=torch.bfloat16, device=dev)
+        self.A = torch.empty(H, d, d, dtype=torch.float32, device=dev)
+        self.b = torch.empty(H, d, dtype=torch.float32, device=dev)
+        self.ws_fit = torch.empty(max(affine_fit_workspace_bytes(H, max(R, d + 1), d), 16), dtype=torch.uint8,
+                                  device=dev)
+
+    # kernel launches of each method
+    LAUNCHES = {
+        "sparse": LAUNCHES_PER_CALL["zb_landmark_build"] + LAUNCHES_PER_CALL["zb_tile_score_topk"]
+        + LAUNCHES_PER_CALL["zb_tile_sparse_attn"],
+        "calibrate": LAUNCHES_PER_CALL["zb_linear_state"] + LAUNCHES_PER_CALL["zb_gather_tiles"]
+        + LAUNCHES_PER_CALL["zb_dense_attn"] + LAUNCHES_PER_CALL["zb_linear_apply"]
+        + LAUNCHES_PER_CALL["zb_affine_fit"],
+        "linear": LAUNCHES_PER_CALL["zb_linear_apply"],
+    }
+
+    def sparse(self, Q, K, V) -> torch.Tensor:
+        zb_landmark_build(Q, K, V, self.tile, out=self.lm)
+        zb_tile_score_topk(self.lm.Qbar, self.lm.Kbar, self.n_tokens, self.tile, self.k, out=self.idx)
+        return zb_tile_sparse_attn(Q, K, V, self.lm.Kbar_bf16, self.lm.Vbar_bf16, self.idx, self.k,
+                                   self.tile, True, self.scale, out=self.O_sparse)
+
+    def calibrate(self, Q, K, V):
+        zb_linear_state(K, V, self.S, self.z, self.ws_lin)
+        zb_gather_tiles(Q, self.tile, self.calib, out=self.Qc)
+        zb_dense_attn(self.Qc, K, V, self.scale, out=self.Yc)
+        zb_linear_apply(self.Qc, self.S, self.z, None, None, out=self.Xc)
+        zb_affine_fit(self.Xc, self.Yc, self.A, self.b, self.ws_fit)
+        return self.A, self.b
+
+    def linear(self, Q, K, V, refresh_state: bool = False) -> torch.Tensor:
+        if refresh_state:
+            zb_linear_state(K, V, self.S, self.z, self.ws_lin)
+        return zb_linear_apply(Q, self.S, self.z, self.A, self.b, out=self.O_linear)
+
+    def step(self, Q, K, V):
+        """One pass of the whole hot path: both stage types on the same input."""
+        o_s = self.sparse(Q, K, V)
+        self.calibrate(Q, K, V)
+        o_l = self.linear(Q, K, V)
+        return o_s, o_l
+
+    @property
+    def launches_per_step(self) -> int:
+        return self.LAUNCHES["sparse"] + self.LAUNCHES["calibrate"] + self.LAUNCHES["linear"]

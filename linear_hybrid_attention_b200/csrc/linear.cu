@@ -1,0 +1,530 @@
+// Linear attention (elu+1 feature map) with the per-head affine correction.
+//
+// "Zebra3D: Efficient Hybrid Foundation Models For Scalable 3D Reconstruction",
+// Abstract: tolerant stages use linear attention; a closed-form affine fit
+// makes the conversion training-free.  "Zebra3D speeds up 3D reconstruction by
+// up to 7.1x on 1024 frames without training from scratch", section "How
+// Zebra3D works": the linear parts are corrected by an affine map fitted in
+// closed form.  Reading used (the pages give no formula): non-causal linear
+// attention with phi(x) = elu(x) + 1 on unscaled q, k:
+//   S = sum_r phi(k_r)^T v_r,  z = sum_r phi(k_r),
+//   O_r = (phi(q_r) S / (phi(q_r) . z)) A + b.
+//
+// Both passes stream HBM once and put the d x d products on tcgen05:
+//  * state: one CTA per (head pair, token chunk).  A 128-token step loads K
+//    and V of two heads by TMA, applies phi to K in place (shared memory, same
+//    swizzled layout) while summing z, and issues
+//        D[128 x 128] += [phi(K_h0)^T ; phi(K_h1)^T] . [V_h0 | V_h1]
+//    (both operands MN-major); the diagonal 64 x 64 blocks are S_h0, S_h1.
+//    Per-CTA partials are added in a fixed order by a second kernel.
+//  * apply: persistent CTAs over (head, 128-token tile); B = [ (S A)^T ; z ;
+//    0 ] (80 x 64, bf16) is built in shared memory once per head, each tile
+//    computes D[128 x 80] = phi(Q) B^T on the tensor core, and the epilogue
+//    forms D[:, :64] / D[:, 64] + b.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include "zb_common.cuh"
+#include "zb_host.h"
+
+namespace zb {
+namespace lin {
+
+constexpr int HD = 64;
+constexpr int TILE = 128;
+constexpr uint32_t TILE_BYTES = TILE * HD * 2;  // 16 KB
+constexpr int TARGET_CTAS = 148;                // one wave on a B200
+
+// ------------------------------------------------------------ geometry ----
+struct StateGeom {
+    int pairs, chunks, tiles_per_chunk, n_tiles;
+};
+
+inline StateGeom state_geom(int heads, long long n) {
+    StateGeom g;
+    g.n_tiles = static_cast<int>((n + TILE - 1) / TILE);
+    g.pairs = (heads + 1) / 2;
+    int chunks = TARGET_CTAS / g.pairs;
+    if (chunks < 1) chunks = 1;
+    if (chunks > g.n_tiles) chunks = g.n_tiles;
+    g.tiles_per_chunk = (g.n_tiles + chunks - 1) / chunks;
+    g.chunks = (g.n_tiles + g.tiles_per_chunk - 1) / g.tiles_per_chunk;
+    return g;
+}
+
+constexpr size_t PARTIAL_FLOATS = 2 * (HD * HD + HD);  // per CTA: S and z of two heads
+
+inline size_t state_ws_bytes(int heads, long long n) {
+    const StateGeom g = state_geom(heads, n);
+    return static_cast<size_t>(g.pairs) * g.chunks * PARTIAL_FLOATS * sizeof(float);
+}
+
+// phi(x) = elu(x) + 1
+__device__ __forceinline__ float phi(float x) { return x > 0.f ? x + 1.f : __expf(x); }
+
+// ============================================================== state ====
+constexpr int ST_STAGES = 3;
+constexpr int ST_THREADS = 128;
+
+struct StateSmem {
+    uint8_t buf[ST_STAGES][4][TILE_BYTES];  // [stage][K0, K1, V0, V1]
+    float zred[4][2][HD];
+    uint64_t full[ST_STAGES], empty[ST_STAGES], done;
+    uint32_t tmem_base;
+    int abort_flag;
+};
+
+__global__ void __launch_bounds__(ST_THREADS, 1)
+linear_state_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
+                    int heads, long long n, StateGeom geo, float* __restrict__ partial, int* status,
+                    unsigned long long timeout_ns) {
+    extern __shared__ uint8_t smem_raw[];
+    StateSmem& sm = *reinterpret_cast<StateSmem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int pair = blockIdx.x / geo.chunks;
+    const int chunk = blockIdx.x % geo.chunks;
+    const int h0 = 2 * pair;
+    const int h1 = min(2 * pair + 1, heads - 1);
+    const int t_begin = chunk * geo.tiles_per_chunk;
+    const int t_end = min(geo.n_tiles, t_begin + geo.tiles_per_chunk);
+    const int steps = t_end - t_begin;
+    const WaitCtx wc{status, &sm.abort_flag, timeout_ns};
+
+    if (tid == 0) {
+        sm.abort_flag = 0;
+        for (int s = 0; s < ST_STAGES; ++s) {
+            mbar_init(smem_addr(&sm.full[s]), 1);
+            mbar_init(smem_addr(&sm.empty[s]), 1);
+        }
+        mbar_init(smem_addr(&sm.done), 1);
+        fence_mbar_init();
+        tma_prefetch_desc(&tm_k);
+        tma_prefetch_desc(&tm_v);
+    }
+    if (warp == 0) tmem_alloc(smem_addr(&sm.tmem_base), 128);
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = sm.tmem_base;
+
+    auto issue_load = [&](int step) {
+        const int s = step % ST_STAGES;
+        const uint32_t bar = smem_addr(&sm.full[s]);
+        const int row = (t_begin + step) * TILE;
+        mbar_arrive_expect_tx(bar, 4 * TILE_BYTES);
+        tma_load_3d(smem_addr(sm.buf[s][0]), &tm_k, bar, 0, row, h0);
+        tma_load_3d(smem_addr(sm.buf[s][1]), &tm_k, bar, 0, row, h1);
+        tma_load_3d(smem_addr(sm.buf[s][2]), &tm_v, bar, 0, row, h0);
+        tma_load_3d(smem_addr(sm.buf[s][3]), &tm_v, bar, 0, row, h1);
+    };
+    uint32_t issued = 0;  // loads issued by thread 0
+    if (tid == 0) {
+        for (int st = 0; st < ST_STAGES - 1 && st < steps; ++st) issue_load(st), ++issued;
+    }
+
+    constexpr uint32_t IDESC = idesc_bf16(128, 128, 1, 1);
+    const int cg = tid & 7;        // logical 16-byte feature group
+    const int rbase = tid >> 3;    // rows rbase + 16 m
+    float z0[8], z1[8];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) z0[e] = z1[e] = 0.f;
+    bool ok = true;
+    int consumed = 0;  // loads whose full barrier was waited on
+
+    for (int st = 0; st < steps; ++st) {
+        const int s = st % ST_STAGES;
+        // a failed wait is not a break: every thread must reach the block barrier
+        bool good = mbar_wait(smem_addr(&sm.full[s]), (st / ST_STAGES) & 1, wc);
+        if (good) {
+            consumed = st + 1;
+            const long long row0 = static_cast<long long>(t_begin + st) * TILE;
+            // phi(K) in place for both heads; rows past n become 0 (no contribution)
+#pragma unroll
+            for (int hh = 0; hh < 2; ++hh) {
+                uint8_t* kt = sm.buf[s][hh];
+#pragma unroll
+                for (int m = 0; m < 8; ++m) {
+                    const int r = rbase + 16 * m;
+                    uint4* p = reinterpret_cast<uint4*>(kt + r * 128 + ((cg ^ (r & 7)) << 4));
+                    uint4 v = *p;
+                    uint32_t w[4] = {v.x, v.y, v.z, v.w};
+                    const bool valid = row0 + r < n;
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const float a = valid ? phi(bf16_lo(w[e])) : 0.f;
+                        const float b = valid ? phi(bf16_hi(w[e])) : 0.f;
+                        w[e] = pack_bf16x2(a, b);
+                        // z sums the bf16-rounded features that the MMA uses
+                        if (hh == 0) { z0[2 * e] += bf16_lo(w[e]); z0[2 * e + 1] += bf16_hi(w[e]); }
+                        else { z1[2 * e] += bf16_lo(w[e]); z1[2 * e + 1] += bf16_hi(w[e]); }
+                    }
+                    *p = make_uint4(w[0], w[1], w[2], w[3]);
+                }
+            }
+        }
+        fence_proxy_async_smem();
+        if (__syncthreads_or(!good)) { ok = false; break; }
+        if (tid == 0) {
+            tc_fence_after();
+            const uint32_t a0 = smem_addr(sm.buf[s][0]);
+            const uint32_t b0 = smem_addr(sm.buf[s][2]);
+#pragma unroll
+            for (int kk = 0; kk < TILE / 16; ++kk) {
+                const uint64_t ad = sdesc_sw128(a0 + kk * 2048, TILE_BYTES, 1024);
+                const uint64_t bd = sdesc_sw128(b0 + kk * 2048, TILE_BYTES, 1024);
+                umma_ss(tmem, ad, bd, IDESC, (st > 0 || kk > 0) ? 1u : 0u);
+            }
+            umma_commit(smem_addr(&sm.empty[s]));
+            // refill the stage used by the previous step once its MMA is done;
+            // a failed wait surfaces at the next block barrier via the abort flag
+            const int nxt = st + ST_STAGES - 1;
+            if (nxt < steps) {
+                const int ps = nxt % ST_STAGES;
+                bool free_ok = true;
+                if (nxt >= ST_STAGES)
+                    free_ok = mbar_wait(smem_addr(&sm.empty[ps]), ((nxt / ST_STAGES) - 1) & 1, wc);
+                if (free_ok) issue_load(nxt), ++issued;
+            }
+        }
+    }
+
+    // ---- drain: no MMA may run and no TMA may write once we read and free
+    {
+        volatile int no_abort = 0;
+        const WaitCtx w2{status, &no_abort, timeout_ns};
+        if (tid == 0) {
+            umma_commit(smem_addr(&sm.done));
+            for (uint32_t q = static_cast<uint32_t>(consumed); q < issued; ++q)
+                mbar_wait(smem_addr(&sm.full[q % ST_STAGES]), (q / ST_STAGES) & 1, w2);
+        }
+        if (!mbar_wait(smem_addr(&sm.done), 0, w2)) ok = false;
+        if (sm.abort_flag) ok = false;
+    }
+    tc_fence_after();
+    float* part = partial + static_cast<size_t>(blockIdx.x) * PARTIAL_FLOATS;
+    if (steps > 0 && ok) {
+        const int hs = tid >> 6;   // head slot of this TMEM lane
+        const int f = tid & 63;    // feature row
+        uint32_t r[64];
+        const uint32_t ta = tmem + (static_cast<uint32_t>(warp * 32) << 16) + hs * 64;
+        tmem_ld32(ta, sub32(r, 0));
+        tmem_ld32(ta + 32, sub32(r, 32));
+        tmem_wait_ld_dep(sub32(r, 0));
+        tmem_wait_ld_dep(sub32(r, 32));
+        float4* dst = reinterpret_cast<float4*>(part + hs * (HD * HD) + f * HD);
+#pragma unroll
+        for (int c = 0; c < 16; ++c)
+            dst[c] = make_float4(__uint_as_float(r[4 * c]), __uint_as_float(r[4 * c + 1]),
+                                 __uint_as_float(r[4 * c + 2]), __uint_as_float(r[4 * c + 3]));
+    } else {
+        for (int e = tid; e < 2 * HD * HD; e += ST_THREADS) part[e] = 0.f;
+    }
+    // z: lanes cg, cg+8, cg+16, cg+24 of a warp share a feature group
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+#pragma unroll
+        for (int o = 8; o <= 16; o <<= 1) {
+            z0[e] += __shfl_xor_sync(0xffffffffu, z0[e], o);
+            z1[e] += __shfl_xor_sync(0xffffffffu, z1[e], o);
+        }
+    }
+    if (lane < 8) {
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+            sm.zred[warp][0][cg * 8 + e] = z0[e];
+            sm.zred[warp][1][cg * 8 + e] = z1[e];
+        }
+    }
+    __syncthreads();
+    {
+        const int hs = tid >> 6, f = tid & 63;
+        float zz = 0.f;
+#pragma unroll
+        for (int w = 0; w < 4; ++w) zz += sm.zred[w][hs][f];
+        part[2 * HD * HD + hs * HD + f] = (steps > 0 && ok) ? zz : 0.f;
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 0) {
+        tc_fence_after();
+        tmem_dealloc(tmem, 128);
+    }
+}
+
+// Fixed-order sum of the per-CTA partials: S[h], z[h].
+__global__ void linear_state_reduce_kernel(const float* __restrict__ partial, int heads, StateGeom geo,
+                                           float* __restrict__ S, float* __restrict__ z) {
+    const int h = blockIdx.x;
+    const int pair = h >> 1, slot = h & 1;
+    for (int e = threadIdx.x; e < HD * HD + HD; e += blockDim.x) {
+        const size_t off = e < HD * HD ? static_cast<size_t>(slot) * HD * HD + e
+                                       : 2 * HD * HD + static_cast<size_t>(slot) * HD + (e - HD * HD);
+        float acc = 0.f;
+        for (int c = 0; c < geo.chunks; ++c)
+            acc += partial[static_cast<size_t>(pair * geo.chunks + c) * PARTIAL_FLOATS + off];
+        if (e < HD * HD) S[static_cast<size_t>(h) * HD * HD + e] = acc;
+        else z[static_cast<size_t>(h) * HD + (e - HD * HD)] = acc;
+    }
+}
+
+// ============================================================== apply ====
+constexpr int AP_STAGES = 4;
+constexpr int AP_THREADS = 128;
+constexpr int BN_ROWS = 80;  // 64 columns of S A, one of z, 15 of zeros
+constexpr uint32_t B_BYTES = BN_ROWS * 128;
+
+struct ApplySmem {
+    uint8_t q[AP_STAGES][TILE_BYTES];
+    uint8_t bop[2][B_BYTES];
+    float bvec[2][HD];
+    uint64_t full[AP_STAGES], mma_done[2], drain;
+    uint32_t tmem_base;
+    int abort_flag;
+};
+
+__global__ void __launch_bounds__(AP_THREADS, 2)
+linear_apply_kernel(const __grid_constant__ CUtensorMap tm_q, int heads, long long n_q,
+                    const float* __restrict__ S, const float* __restrict__ z,
+                    const float* __restrict__ A, const float* __restrict__ bias,
+                    uint16_t* __restrict__ O, int* status, unsigned long long timeout_ns) {
+    extern __shared__ uint8_t smem_raw[];
+    ApplySmem& sm = *reinterpret_cast<ApplySmem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int Tn = static_cast<int>((n_q + TILE - 1) / TILE);
+    const long long n_items = static_cast<long long>(heads) * Tn;
+    const long long per = (n_items + gridDim.x - 1) / gridDim.x;
+    const long long first = static_cast<long long>(blockIdx.x) * per;
+    const long long last = min(n_items, first + per);
+    const int cnt = first < last ? static_cast<int>(last - first) : 0;
+    const WaitCtx wc{status, &sm.abort_flag, timeout_ns};
+
+    if (tid == 0) {
+        sm.abort_flag = 0;
+        for (int s = 0; s < AP_STAGES; ++s) mbar_init(smem_addr(&sm.full[s]), 1);
+        for (int s = 0; s < 2; ++s) mbar_init(smem_addr(&sm.mma_done[s]), 1);
+        mbar_init(smem_addr(&sm.drain), 1);
+        fence_mbar_init();
+        tma_prefetch_desc(&tm_q);
+    }
+    if (warp == 0) tmem_alloc(smem_addr(&sm.tmem_base), 256);
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = sm.tmem_base;
+
+    auto issue_load = [&](int it) {
+        const long long item = first + it;
+        const int h = static_cast<int>(item / Tn), t = static_cast<int>(item % Tn);
+        const int s = it % AP_STAGES;
+        const uint32_t bar = smem_addr(&sm.full[s]);
+        mbar_arrive_expect_tx(bar, TILE_BYTES);
+        tma_load_3d(smem_addr(sm.q[s]), &tm_q, bar, 0, t * TILE, h);
+    };
+    uint32_t issued = 0;
+    if (tid == 0)
+        for (int it = 0; it < AP_STAGES && it < cnt; ++it) issue_load(it), ++issued;
+
+    constexpr uint32_t IDESC = idesc_bf16(128, BN_ROWS, 0, 0);
+    const int cg = tid & 7, rbase = tid >> 3;
+    const uint32_t lane_addr = static_cast<uint32_t>(warp * 32) << 16;
+    int h_prev = -1;
+    int consumed = 0;
+    bool ok = true;
+
+    // epilogue of item `it`: O row = D[:64] / D[64] + b
+    auto epilogue = [&](int it) -> bool {
+        const int buf = it & 1;
+        if (!mbar_wait(smem_addr(&sm.mma_done[buf]), (it >> 1) & 1, wc)) return false;
+        tc_fence_after();
+        uint32_t r[96];
+        const uint32_t ta = tmem + lane_addr + buf * 128;
+        tmem_ld32(ta, sub32(r, 0));
+        tmem_ld32(ta + 32, sub32(r, 32));
+        tmem_ld32(ta + 64, sub32(r, 64));
+        tmem_wait_ld_dep(sub32(r, 0));
+        tmem_wait_ld_dep(sub32(r, 32));
+        tmem_wait_ld_dep(sub32(r, 64));
+        tc_fence_before();
+        const long long item = first + it;
+        const int h = static_cast<int>(item / Tn), t = static_cast<int>(item % Tn);
+        const long long row = static_cast<long long>(t) * TILE + tid;
+        if (row < n_q) {
+            const float inv = 1.f / __uint_as_float(r[64]);
+            uint4* dst = reinterpret_cast<uint4*>(O + (static_cast<long long>(h) * n_q + row) * HD);
+            const float* bb = sm.bvec[h & 1];
+#pragma unroll
+            for (int c = 0; c < HD / 8; ++c) {
+                float o[8];
+#pragma unroll
+                for (int e = 0; e < 8; ++e) o[e] = fmaf(__uint_as_float(r[c * 8 + e]), inv, bb[c * 8 + e]);
+                dst[c] = make_uint4(pack_bf16x2(o[0], o[1]), pack_bf16x2(o[2], o[3]),
+                                    pack_bf16x2(o[4], o[5]), pack_bf16x2(o[6], o[7]));
+            }
+        }
+        return true;
+    };
+
+    for (int it = 0; it < cnt; ++it) {
+        const long long item = first + it;
+        const int h = static_cast<int>(item / Tn);
+        if (h != h_prev) {
+            // B operand of head h into buffer (h & 1): rows n < 64 hold (S A)[:, n],
+            // row 64 holds z, rows 65..79 zero; K-major, 128-byte swizzle.
+            uint8_t* bo = sm.bop[h & 1];
+            const float* Sh = S + static_cast<size_t>(h) * HD * HD;
+            const float* Ah = A ? A + static_cast<size_t>(h) * HD * HD : nullptr;
+            {
+                const int ncol = tid & 63;       // output column n
+                const int khalf = tid >> 6;      // rows k in [32 khalf, 32 khalf + 32)
+                float acol[HD];
+#pragma unroll
+                for (int m = 0; m < HD; ++m) acol[m] = Ah ? __ldg(Ah + m * HD + ncol) : (m == ncol ? 1.f : 0.f);
+                for (int kq = 0; kq < 32; kq += 2) {
+                    float v2[2];
+#pragma unroll
+                    for (int u = 0; u < 2; ++u) {
+                        const int k = khalf * 32 + kq + u;
+                        const float* srow = Sh + k * HD;
+                        float acc = 0.f;
+#pragma unroll
+                        for (int m = 0; m < HD; ++m) acc = fmaf(__ldg(srow + m), acol[m], acc);
+                        v2[u] = acc;
+                    }
+                    const int k = khalf * 32 + kq;  // even: both land in one 32-bit word
+                    const int off = ncol * 128 + ((((k >> 3) ^ (ncol & 7))) << 4) + (k & 7) * 2;
+                    *reinterpret_cast<uint32_t*>(bo + off) = pack_bf16x2(v2[0], v2[1]);
+                }
+            }
+            for (int e = tid; e < 16 * HD / 2; e += AP_THREADS) {
+                // rows 64..79: z then zeros, two values per word
+                const int rr = 64 + e / (HD / 2);
+                const int k = (e % (HD / 2)) * 2;
+                const float a = rr == 64 ? z[static_cast<size_t>(h) * HD + k] : 0.f;
+                const float b = rr == 64 ? z[static_cast<size_t>(h) * HD + k + 1] : 0.f;
+                const int off = rr * 128 + ((((k >> 3) ^ (rr & 7))) << 4) + (k & 7) * 2;
+                *reinterpret_cast<uint32_t*>(bo + off) = pack_bf16x2(a, b);
+            }
+            if (tid < HD) sm.bvec[h & 1][tid] = bias ? bias[static_cast<size_t>(h) * HD + tid] : 0.f;
+            h_prev = h;
+        }
+        const int s = it % AP_STAGES;
+        if (!mbar_wait(smem_addr(&sm.full[s]), (it / AP_STAGES) & 1, wc)) ok = false;
+        else consumed = it + 1;
+        if (ok) {
+            uint8_t* qt = sm.q[s];
+#pragma unroll
+            for (int m = 0; m < 8; ++m) {
+                const int r = rbase + 16 * m;
+                uint4* p = reinterpret_cast<uint4*>(qt + r * 128 + ((cg ^ (r & 7)) << 4));
+                uint4 v = *p;
+                uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+                for (int e = 0; e < 4; ++e) w[e] = pack_bf16x2(phi(bf16_lo(w[e])), phi(bf16_hi(w[e])));
+                *p = make_uint4(w[0], w[1], w[2], w[3]);
+            }
+        }
+        fence_proxy_async_smem();
+        if (__syncthreads_or(!ok)) { ok = false; break; }
+        if (tid == 0) {
+            tc_fence_after();
+            const uint32_t a0 = smem_addr(sm.q[s]);
+            const uint32_t b0 = smem_addr(sm.bop[h & 1]);
+            const uint32_t d = tmem + (it & 1) * 128;
+#pragma unroll
+            for (int kk = 0; kk < HD / 16; ++kk) {
+                const uint64_t ad = sdesc_sw128(a0 + kk * 32, 16, 1024);
+                const uint64_t bd = sdesc_sw128(b0 + kk * 32, 16, 1024);
+                umma_ss(d, ad, bd, IDESC, kk > 0 ? 1u : 0u);
+            }
+            umma_commit(smem_addr(&sm.mma_done[it & 1]));
+        }
+        if (it >= 1) {
+            if (!epilogue(it - 1)) ok = false;
+            // the stage of item it-1 is free (its MMA is done): refill it
+            if (tid == 0 && ok && it - 1 + AP_STAGES < cnt) issue_load(it - 1 + AP_STAGES), ++issued;
+        }
+    }
+    if (ok && cnt > 0) {
+        if (!epilogue(cnt - 1)) ok = false;
+    }
+    // drain: no MMA may run and no TMA may write once TMEM and smem are released
+    if (tid == 0) {
+        volatile int no_abort = 0;
+        const WaitCtx w2{status, &no_abort, timeout_ns};
+        umma_commit(smem_addr(&sm.drain));
+        mbar_wait(smem_addr(&sm.drain), 0, w2);
+        for (uint32_t q = static_cast<uint32_t>(consumed); q < issued; ++q)
+            mbar_wait(smem_addr(&sm.full[q % AP_STAGES]), (q / AP_STAGES) & 1, w2);
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 0) {
+        tc_fence_after();
+        tmem_dealloc(tmem, 256);
+    }
+}
+
+}  // namespace lin
+}  // namespace zb
+
+using namespace zb;
+
+extern "C" size_t zb_linear_state_workspace_bytes(int32_t heads, int64_t n_tokens, int32_t head_dim) {
+    if (heads < 1 || n_tokens < 1 || head_dim != 64) return 0;
+    return lin::state_ws_bytes(heads, n_tokens);
+}
+
+extern "C" zb_status zb_linear_state(const uint16_t* K, const uint16_t* V, int32_t heads,
+                                     int64_t n_tokens, int32_t head_dim, float* S, float* z,
+                                     void* ws, size_t ws_bytes, void* stream) {
+    if (heads < 1 || n_tokens < 1) return ZB_ERR_SHAPE;
+    if (head_dim != 64) return ZB_ERR_UNSUPPORTED;
+    if (n_tokens > (1ll << 31) - 256) return ZB_ERR_UNSUPPORTED;
+    if (!K || !V || !S || !z) return ZB_ERR_NULL;
+    if (!aligned16(K) || !aligned16(V) || !aligned16(S) || !aligned16(z) || !aligned16(ws)) return ZB_ERR_ALIGN;
+    const size_t need = lin::state_ws_bytes(heads, n_tokens);
+    if (!ws || ws_bytes < need) return ZB_ERR_WORKSPACE;
+    DeviceInfo dev;
+    zb_status e = current_device(&dev);
+    if (e != ZB_OK) return e;
+    CUtensorMap mk, mv;
+    if ((e = make_map_bf16_3d(&mk, K, 64, n_tokens, heads, lin::TILE)) != ZB_OK) return e;
+    if ((e = make_map_bf16_3d(&mv, V, 64, n_tokens, heads, lin::TILE)) != ZB_OK) return e;
+    const lin::StateGeom geo = lin::state_geom(heads, n_tokens);
+    const size_t smem = sizeof(lin::StateSmem) + 1024;
+    if (cudaFuncSetAttribute(lin::linear_state_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(smem)) != cudaSuccess)
+        return ZB_ERR_CUDA;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    float* part = static_cast<float*>(ws);
+    lin::linear_state_kernel<<<geo.pairs * geo.chunks, lin::ST_THREADS, smem, st>>>(
+        mk, mv, heads, n_tokens, geo, part, dev.status, wait_timeout_ns());
+    if (cudaGetLastError() != cudaSuccess) return ZB_ERR_CUDA;
+    lin::linear_state_reduce_kernel<<<heads, 256, 0, st>>>(part, heads, geo, S, z);
+    return cudaGetLastError() == cudaSuccess ? ZB_OK : ZB_ERR_CUDA;
+}
+
+extern "C" zb_status zb_linear_apply(const uint16_t* Q, int32_t heads, int64_t n_q,
+                                     int32_t head_dim, const float* S, const float* z,
+                                     const float* A, const float* b, uint16_t* O, void* stream) {
+    if (heads < 1 || n_q < 1) return ZB_ERR_SHAPE;
+    if (head_dim != 64) return ZB_ERR_UNSUPPORTED;
+    if (n_q > (1ll << 31) - 256) return ZB_ERR_UNSUPPORTED;
+    if (!Q || !S || !z || !O) return ZB_ERR_NULL;
+    if (!aligned16(Q) || !aligned16(S) || !aligned16(z) || !aligned16(A) || !aligned16(b) || !aligned16(O))
+        return ZB_ERR_ALIGN;
+    DeviceInfo dev;
+    zb_status e = current_device(&dev);
+    if (e != ZB_OK) return e;
+    CUtensorMap mq;
+    if ((e = make_map_bf16_3d(&mq, Q, 64, n_q, heads, lin::TILE)) != ZB_OK) return e;
+    const size_t smem = sizeof(lin::ApplySmem) + 1024;
+    if (cudaFuncSetAttribute(lin::linear_apply_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(smem)) != cudaSuccess)
+        return ZB_ERR_CUDA;
+    const long long items = static_cast<long long>(heads) * ((n_q + lin::TILE - 1) / lin::TILE);
+    const long long grid = items < 2ll * dev.sm_count ? items : 2ll * dev.sm_count;
+    lin::linear_apply_kernel<<<static_cast<unsigned>(grid), lin::AP_THREADS, smem, static_cast<cudaStream_t>(stream)>>>(
+        mq, heads, n_q, S, z, A, b, O, dev.status, wait_timeout_ns());
+    return cudaGetLastError() == cudaSuccess ? ZB_OK : ZB_ERR_CUDA;
+}

@@ -1,0 +1,114 @@
+"""The C ABI on the host: the library builds and loads, exports every function
+that include/zb.h declares, and rejects bad arguments before touching the GPU.
+CPU only: no call here reaches a CUDA API (validation runs first)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "zb.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from linear_hybrid_attention_b200 import build, _lib
+    build.build()
+    return _lib.load()
+
+
+def _declared():
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(zb_[a-z0-9_]+)\s*\(", src)))
+
+
+def test_header_declares_the_calls():
+    names = _declared()
+    for n in ["zb_landmark_build", "zb_tile_score_topk", "zb_tile_sparse_attn", "zb_dense_attn",
+              "zb_linear_state", "zb_linear_apply", "zb_affine_fit", "zb_gather_tiles",
+              "zb_last_device_status", "zb_status_string", "zb_abi_version"]:
+        assert n in names
+
+
+def test_every_declared_symbol_is_exported(lib):
+    for n in _declared():
+        assert hasattr(lib, n), n
+    from linear_hybrid_attention_b200 import _lib
+    assert set(_declared()) == set(_lib.PROTOTYPES)
+
+
+def test_version_and_status_strings(lib):
+    assert lib.zb_abi_version() == 100
+    for code, name in [(0, "ZB_OK"), (2, "ZB_ERR_SHAPE"), (7, "ZB_ERR_TIMEOUT"), (9, "ZB_ERR_INDEX")]:
+        assert lib.zb_status_string(code).decode().startswith(name)
+    assert b"unknown" in lib.zb_status_string(1234)
+
+
+def test_workspace_sizes(lib):
+    n = lib.zb_linear_state_workspace_bytes(16, 1024 * 1374, 64)
+    assert 0 < n < 64 * 2**20
+    assert lib.zb_linear_state_workspace_bytes(16, 1000, 32) == 0
+    assert lib.zb_affine_fit_workspace_bytes(16, 4096, 64) == 16 * (128 + 16 * 2 * 4096) * 8
+    assert lib.zb_affine_fit_workspace_bytes(0, 4096, 64) == 0
+
+
+def _shape(H=2, N=256, d=64, t=64):
+    from linear_hybrid_attention_b200._lib import ZbShape
+    return ZbShape(H, N, d, t)
+
+
+FAKE = 0x10000  # 16-byte aligned, never dereferenced: validation fails first
+
+
+def test_validation_errors_before_launch(lib):
+    S = _shape()
+    # unsupported head_dim / tile, bad sizes
+    assert lib.zb_landmark_build(FAKE, FAKE, FAKE, _shape(d=32), FAKE, FAKE, FAKE, FAKE, None) == 4
+    assert lib.zb_landmark_build(FAKE, FAKE, FAKE, _shape(t=96), FAKE, FAKE, FAKE, FAKE, None) == 4
+    assert lib.zb_landmark_build(FAKE, FAKE, FAKE, _shape(N=0), FAKE, FAKE, FAKE, FAKE, None) == 2
+    assert lib.zb_landmark_build(FAKE, None, FAKE, S, FAKE, FAKE, FAKE, FAKE, None) == 1
+    assert lib.zb_landmark_build(FAKE, FAKE, FAKE, S, None, FAKE, FAKE, FAKE, None) == 1
+    assert lib.zb_landmark_build(FAKE + 8, FAKE, FAKE, S, FAKE, FAKE, FAKE, FAKE, None) == 3
+    # selection: k out of range, null output
+    assert lib.zb_tile_score_topk(FAKE, FAKE, S, 5, FAKE, None) == 2
+    assert lib.zb_tile_score_topk(FAKE, FAKE, S, -1, FAKE, None) == 2
+    assert lib.zb_tile_score_topk(FAKE, FAKE, S, 2, None, None) == 1
+    assert lib.zb_tile_score_topk(FAKE, FAKE, S, 0, None, None) == 0  # nothing to do
+    # sparse attention
+    a = (FAKE, FAKE, FAKE, FAKE, FAKE, FAKE)
+    assert lib.zb_tile_sparse_attn(*a, 5, 1, 0.125, S, FAKE, None, None) == 2          # k > T
+    assert lib.zb_tile_sparse_attn(*a, 0, 0, 0.125, S, FAKE, None, None) == 2          # no keys
+    assert lib.zb_tile_sparse_attn(*a, 2, 1, -1.0, S, FAKE, None, None) == 2           # scale
+    assert lib.zb_tile_sparse_attn(FAKE, FAKE, FAKE, None, FAKE, FAKE, 2, 1, 0.125, S, FAKE, None, None) == 1
+    assert lib.zb_tile_sparse_attn(FAKE, FAKE, FAKE, FAKE, FAKE, None, 2, 1, 0.125, S, FAKE, None, None) == 1
+    assert lib.zb_tile_sparse_attn(*a, 2, 1, 0.125, S, FAKE + 4, None, None) == 3
+    assert lib.zb_tile_sparse_attn(*a, 2, 1, 0.125, _shape(N=128 * 40000), FAKE, None, None) == 4  # T > 32768
+    # dense
+    assert lib.zb_dense_attn(FAKE, 0, FAKE, FAKE, 10, 2, 64, 0.125, FAKE, None, None) == 2
+    assert lib.zb_dense_attn(FAKE, 10, FAKE, FAKE, 10, 2, 128, 0.125, FAKE, None, None) == 4
+    # linear
+    need = lib.zb_linear_state_workspace_bytes(2, 256, 64)
+    assert lib.zb_linear_state(FAKE, FAKE, 2, 256, 64, FAKE, FAKE, FAKE, need - 1, None) == 5
+    assert lib.zb_linear_state(FAKE, FAKE, 2, 256, 64, FAKE, FAKE, None, need, None) == 5
+    assert lib.zb_linear_state(FAKE, None, 2, 256, 64, FAKE, FAKE, FAKE, need, None) == 1
+    assert lib.zb_linear_apply(FAKE, 2, 256, 64, FAKE, None, None, None, FAKE, None) == 1
+    assert lib.zb_linear_apply(FAKE, 2, 256, 64, FAKE, FAKE, FAKE + 2, None, FAKE, None) == 3
+    # affine fit: too few rows, workspace
+    assert lib.zb_affine_fit(FAKE, FAKE, 2, 64, 64, FAKE, FAKE, FAKE, 1 << 30, None) == 2
+    wsn = lib.zb_affine_fit_workspace_bytes(2, 300, 64)
+    assert lib.zb_affine_fit(FAKE, FAKE, 2, 300, 64, FAKE, FAKE, FAKE, wsn - 8, None) == 5
+    # gather
+    assert lib.zb_gather_tiles(FAKE, S, FAKE, 0, FAKE, None) == 2
+    assert lib.zb_gather_tiles(FAKE, S, None, 2, FAKE, None) == 1
+
+
+def test_binding_refuses_cpu_tensors():
+    import torch
+    import linear_hybrid_attention_b200 as zb
+    x = torch.zeros(1, 64, 64, dtype=torch.bfloat16)
+    with pytest.raises(ValueError, match="CUDA"):
+        zb.zb_landmark_build(x, x, x, 64)
+    with pytest.raises(ValueError, match="CUDA"):
+        zb.zb_linear_state(x, x)

@@ -1,0 +1,111 @@
+"""GPU parity: landmarks (bit-exact fp64 means) and tile selection (bit-exact sets)."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import synth
+from tests.gpu_helpers import bf16_round_f64, host, sync_ok, workload
+
+pytestmark = pytest.mark.gpu
+
+CASES = [
+    ("tiny", {}),                                       # t = 64, T = 4, k = 2
+    ("views32", {"heads": 3, "n_tokens": 5000}),        # ragged last tile (8 rows), odd heads
+    ("views32", {}),                                    # full 32-view stage: T = 344, k = 69
+]
+
+
+def _ids(c):
+    return c[0] + ("-" + "-".join(f"{k}{v}" for k, v in c[1].items()) if c[1] else "")
+
+
+@pytest.fixture(scope="module", params=CASES, ids=[_ids(c) for c in CASES])
+def case(request):
+    import linear_hybrid_attention_b200 as zb
+    name, over = request.param
+    w = workload(name, **over)
+    Q, K, V = synth.make_qkv(w, device="cuda")
+    lm = zb.zb_landmark_build(Q, K, V, w.tile)
+    idx = zb.zb_tile_score_topk(lm.Qbar, lm.Kbar, w.n_tokens, w.tile, w.k)
+    sync_ok()
+    Qb = oracle.landmark_means(host(Q), w.tile)
+    Kb = oracle.landmark_means(host(K), w.tile)
+    Vb = oracle.landmark_means(host(V), w.tile)
+    return w, (Q, K, V), lm, idx, (Qb, Kb, Vb)
+
+
+def test_landmark_means_bit_exact(case):
+    w, _, lm, _, (Qb, Kb, Vb) = case
+    assert np.array_equal(lm.Qbar.cpu().numpy(), Qb)
+    assert np.array_equal(lm.Kbar.cpu().numpy(), Kb)
+
+
+def test_landmark_bf16_correctly_rounded(case):
+    w, _, lm, _, (Qb, Kb, Vb) = case
+    assert np.array_equal(host(lm.Kbar_bf16), bf16_round_f64(Kb))
+    assert np.array_equal(host(lm.Vbar_bf16), bf16_round_f64(Vb))
+
+
+def test_selection_bit_exact(case):
+    w, _, _, idx, (Qb, Kb, _) = case
+    ref = oracle.select_tiles(oracle.tile_scores(Qb, Kb), w.k)
+    got = idx.cpu().numpy().astype(np.int64)
+    if not np.array_equal(got, ref):
+        bad = np.argwhere((got != ref).any(-1))
+        scores = oracle.tile_scores(Qb, Kb)
+        h, i = bad[0]
+        s = np.sort(scores[h, i])[::-1]
+        raise AssertionError(f"{len(bad)} rows differ; first (h={h}, i={i}); k-th/k+1-th score gap "
+                             f"{s[w.k - 1] - s[w.k]:.3e}")
+
+
+def test_selection_keeps_planted_tiles_tiny():
+    import linear_hybrid_attention_b200 as zb
+    w = workload("tiny")
+    Q, K, V = synth.make_qkv(w, device="cuda")
+    lm = zb.zb_landmark_build(Q, K, V, w.tile)
+    idx = zb.zb_tile_score_topk(lm.Qbar, lm.Kbar, w.n_tokens, w.tile, w.k).cpu().numpy()
+    hh, ii, jj = synth.planted_pairs(w, synth.default_seed(w))
+    for h, i, j in zip(hh, ii, jj):
+        assert j in idx[h, i]
+
+
+@pytest.mark.parametrize("k", [1, 17, 39, 40])
+def test_selection_edge_budgets(k):
+    import linear_hybrid_attention_b200 as zb
+    w = workload("views32", heads=2, n_tokens=5000)
+    Q, K, V = synth.make_qkv(w, device="cuda", seed=77)
+    lm = zb.zb_landmark_build(Q, K, V, w.tile)
+    idx = zb.zb_tile_score_topk(lm.Qbar, lm.Kbar, w.n_tokens, w.tile, k)
+    sync_ok()
+    ref = oracle.select_tiles(oracle.tile_scores(oracle.landmark_means(host(Q), w.tile),
+                                                 oracle.landmark_means(host(K), w.tile)), k)
+    assert np.array_equal(idx.cpu().numpy(), ref)
+
+
+def test_selection_ties_go_to_lower_index():
+    # zero queries: every score is 0 (or -0), so the k lowest indices are kept
+    import linear_hybrid_attention_b200 as zb
+    H, N, t, k = 2, 1000, 64, 5
+    Qbar = torch.zeros(H, 16, 64, dtype=torch.float64, device="cuda")
+    Kbar = torch.randn(H, 16, 64, dtype=torch.float64, device="cuda")
+    Qbar[1, :, 0] = -0.0
+    idx = zb.zb_tile_score_topk(Qbar, Kbar, N, t, k)
+    sync_ok()
+    assert (idx.cpu() == torch.arange(k, dtype=torch.int32)).all()
+
+
+def test_gather_tiles():
+    import linear_hybrid_attention_b200 as zb
+    w = workload("views32", heads=2, n_tokens=1000)   # T = 8, last tile 104 rows
+    Q, _, _ = synth.make_qkv(w, device="cuda")
+    tiles = torch.tensor([7, 0, 3], dtype=torch.int32, device="cuda")
+    out = zb.zb_gather_tiles(Q, w.tile, tiles)
+    sync_ok()
+    q = Q.cpu()
+    o = out.cpu()
+    assert torch.equal(o[:, :104], q[:, 896:1000])
+    assert (o[:, 104:128] == 0).all()
+    assert torch.equal(o[:, 128:256], q[:, 0:128])
+    assert torch.equal(o[:, 256:384], q[:, 384:512])
