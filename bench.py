@@ -1,0 +1,413 @@
+"""Benchmark of the Zebra3D hybrid global-attention layer on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload views1024] [--impl reference]
+
+One step = one pass of the whole hot path on one synthetic 1,024-view input
+(16 heads x 1,406,976 tokens, d = 64, bf16): the tile-sparse stage (landmark
+means, fp64 tile selection keeping 6% of key tiles, tile-sparse attention with
+landmarks) and the linear stage (elu+1 state, dense attention on 4,096
+calibration rows, closed-form affine fit, fitted linear attention on all
+rows).  The metric is hybrid-layer throughput with half the layers linear
+(0.5L): tokens / (0.5 t_linear + 0.5 t_sparse) = 2 N / t_step, in Mtokens/s.
+
+Prints ONE JSON line on rank 0.  Under torchrun every rank runs its own
+independent input (weak scaling, no collective on the data path).
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+import torch  # noqa: E402
+
+import synth  # noqa: E402
+from linear_hybrid_attention_b200 import replicas  # noqa: E402
+
+METRIC = "hybrid global-attn layer Mtokens/s at 1,024 views; % bf16 TC peak / % HBM BW"
+UNIT = "Mtokens/s"
+
+
+# ------------------------------------------------------------------ peaks ----
+def measured_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return {"hbm_gbs": d["hbm_gbs"], "bf16_tflops": d["bf16_tflops"],
+                "bf16_tflops_sustained": d.get("bf16_tflops_sustained", d["bf16_tflops"]),
+                "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
+
+
+# ----------------------------------------------------------------- clocks ----
+class ClockSampler:
+    """nvidia-smi sampling of SM clock and throttle reasons during the timed region."""
+
+    FIELDS = ("index,uuid,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index: int):
+        self.proc = None
+        self.path = None
+        try:
+            props = torch.cuda.get_device_properties(device_index)
+            u = str(getattr(props, "uuid", ""))
+            self.uuid = u if u.startswith("GPU-") else ("GPU-" + u if u else "")
+        except Exception:
+            self.uuid = ""
+
+    def start(self):
+        try:
+            fd, self.path = tempfile.mkstemp(suffix=".csv")
+            os.close(fd)
+            cmd = ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits", "-lms", "200"]
+            if self.uuid:
+                cmd += ["-i", self.uuid]
+            self.proc = subprocess.Popen(cmd, stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        rows = []
+        try:
+            with open(self.path) as f:
+                for line in f:
+                    parts = [p.strip() for p in line.split(",")]
+                    if len(parts) >= 10:
+                        rows.append(parts)
+            os.remove(self.path)
+        except Exception:
+            return None
+        if not rows:
+            return None
+        sm = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        smax = [float(r[3]) for r in rows if r[3].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[6 + i].lower().startswith("active")})
+        loaded = [s for s in sm if smax and s > 0.5 * max(smax)] or sm
+        return {"sm_mhz": statistics.median(loaded) if loaded else None,
+                "sm_max_mhz": max(smax) if smax else None, "reasons": reasons, "samples": len(rows)}
+
+
+# --------------------------------------------------------------- CPU oracle ----
+def oracle_sample(w, Q, K, V, calib_tiles, sample_tiles=4, calib_rows=16, head=0):
+    """Time the fp64 oracle on a bounded sample of one head and extrapolate.
+
+    Fixed per-head work (landmark means, linear state, calibration dense rows +
+    unfitted linear rows + fit) and per-query-tile work (selection row, sparse
+    attention, fitted linear output) are timed on `sample_tiles` query tiles and
+    `calib_rows` calibration rows of one head, then scaled to the full job.
+    Returns (extrapolated seconds per step, description, cores)."""
+    import oracle
+    cores = len(os.sched_getaffinity(0))
+    d = w.head_dim
+    s = 1.0 / math.sqrt(d)
+    t0 = time.perf_counter()
+    q = synth.to_f64(Q[head:head + 1])
+    k = synth.to_f64(K[head:head + 1])
+    v = synth.to_f64(V[head:head + 1])
+    t_load = time.perf_counter() - t0
+    # --- fixed per-head work
+    t0 = time.perf_counter()
+    Qb = oracle.landmark_means(q, w.tile)
+    Kb = oracle.landmark_means(k, w.tile)
+    S, z = oracle.linear_state(k, v)
+    t_fixed = time.perf_counter() - t0
+    rows = oracle.calibration_rows(w.n_tokens, w.tile, calib_tiles)
+    sub = rows[:calib_rows]
+    t0 = time.perf_counter()
+    Y = np.concatenate([oracle.dense_attention(q[:, sub[c:c + 16]], k, v, s)
+                        for c in range(0, len(sub), 16)], axis=1)
+    X = oracle.linear_attention(q[:, sub], k, v)
+    t_cal = (time.perf_counter() - t0) * (len(rows) / len(sub))
+    # the fit itself is timed at the full calibration size (the values of the
+    # tiled rows do not matter for its cost; a small jitter keeps it full-rank)
+    reps = -(-len(rows) // len(sub))
+    jit = 1e-3 * np.random.default_rng(0).standard_normal((1, len(rows), d))
+    Xf = np.tile(X, (1, reps, 1))[:, : len(rows)] + jit
+    Yf = np.tile(Y, (1, reps, 1))[:, : len(rows)]
+    t0 = time.perf_counter()
+    A, b = oracle.affine_fit(Xf, Yf)
+    t_fit = time.perf_counter() - t0
+    # --- per-query-tile work
+    tiles = list(np.linspace(0, w.n_tiles - 1, sample_tiles).astype(int))
+    t0 = time.perf_counter()
+    sc = oracle.tile_scores(Qb[:, tiles], Kb)
+    idx_s = oracle.select_tiles(sc, w.k)
+    idx = np.zeros((1, w.n_tiles, w.k), dtype=np.int64)
+    idx[0, tiles] = idx_s[0]
+    oracle.sparse_attention(q, k, v, w.tile, idx, s, query_tiles=tiles)
+    qrows = oracle.calibration_rows(w.n_tokens, w.tile, tiles)
+    oracle.linear_apply(q[:, qrows], S, z, A, b)
+    t_tiles = time.perf_counter() - t0
+    per_head = t_fixed + t_cal + t_fit + t_tiles * (w.n_tiles / sample_tiles)
+    total = per_head * w.heads
+    desc = (f"fp64 oracle on head {head}: landmarks + linear state of the head, {len(sub)} of {len(rows)} "
+            f"calibration rows, {sample_tiles} of {w.n_tiles} query tiles (selection, sparse attention, "
+            f"fitted linear); extrapolated to {w.heads} heads x {w.n_tiles} tiles "
+            f"(sample time {t_fixed + t_cal / (len(rows) / len(sub)) + t_fit + t_tiles:.1f} s, "
+            f"load {t_load:.1f} s)")
+    return total, desc, cores
+
+
+# ------------------------------------------------------------------- main ----
+def selected_flops(idx_cpu: np.ndarray, n_tokens: int, tile: int, d: int) -> float:
+    """4 * d * sum over (h, i, j in sel) n_i * n_j: the algorithmic FLOPs of QK^T and PV."""
+    T = idx_cpu.shape[1]
+    n = np.full(T, tile, dtype=np.float64)
+    n[-1] = n_tokens - (T - 1) * tile
+    per_row = n[idx_cpu].sum(axis=-1)  # [H, T]
+    return float(4.0 * d * (per_row * n[None, :]).sum())
+
+
+def run_reference(args, w):
+    rank, _, world = replicas.env_rank()
+    if rank != 0:
+        return 0
+    Q, K, V = synth.make_qkv(w, device="cpu" if not torch.cuda.is_available() else "cuda")
+    calib = synth.calibration_tiles(w.n_tiles, w.calib_tiles)
+    times = []
+    desc = cores = None
+    for _ in range(args.warmup + args.steps):
+        t, desc, cores = oracle_sample(w, Q, K, V, calib, sample_tiles=2, calib_rows=8)
+        times.append(t)
+    t = statistics.median(times[args.warmup:]) if args.steps else times[-1]
+    value = 2 * w.n_tokens / t / 1e6
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": t * 1e3, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": config_dict(w),
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle", "sample": desc},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def config_dict(w):
+    return {"workload": f"{w.name}: {w.n_tokens // synth.TOKENS_PER_VIEW} views x {synth.TOKENS_PER_VIEW} "
+                        f"tokens = {w.n_tokens} tokens, {w.heads} heads, d={w.head_dim}, bf16; tile "
+                        f"{w.tile}, keep {w.k}/{w.n_tiles} key tiles + landmarks; linear elu+1 with affine "
+                        f"fit on {len(synth.calibration_tiles(w.n_tiles, w.calib_tiles)) * w.tile} rows; "
+                        f"0.5L/0.5S hybrid",
+            "heads": w.heads, "n_tokens": w.n_tokens, "head_dim": w.head_dim, "tile": w.tile, "k": w.k,
+            "linear_fraction": 0.5, "l2": "inputs larger than L2 (each of Q, K, V, O is "
+            f"{w.heads * w.n_tokens * w.head_dim * 2 / 1e9:.2f} GB)"}
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=5)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--workload", default="views1024", choices=sorted(synth.WORKLOADS))
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--keep-frac", type=float, default=None, help="override the kept fraction of key tiles")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu", action="store_true")
+    ap.add_argument("--profile", action="store_true", help="short run for profilers: no JSON extras")
+    args = ap.parse_args()
+
+    w = synth.WORKLOADS[args.workload]
+    if args.keep_frac is not None:
+        import dataclasses
+        w = dataclasses.replace(w, keep_frac=args.keep_frac, k_fixed=None)
+    if w.k is None:
+        import dataclasses
+        w = dataclasses.replace(w, keep_frac=0.06)
+    if args.impl == "reference":
+        return run_reference(args, w)
+
+    rank, local_rank, world = replicas.env_rank()
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py needs a CUDA device (libzb has no CPU path)")
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    if world > 1:
+        import datetime
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                             device_id=dev)
+    import linear_hybrid_attention_b200 as zb
+    zb._lib.load()
+
+    seed = replicas.rank_seed(synth.default_seed(w), rank)
+    Q, K, V = synth.make_qkv(w, device=dev, seed=seed)
+    calib = synth.calibration_tiles(w.n_tiles, w.calib_tiles)
+    layer = zb.HybridLayer(w.heads, w.n_tokens, w.tile, w.k, calib, device=dev)
+    stream = torch.cuda.current_stream()
+
+    # per-kernel events around each call of the step (same stream as the kernels)
+    names = ["landmark", "topk", "sparse_attn", "linear_state", "calib_dense", "calib_rest", "linear_apply"]
+
+    def step(ev=None):
+        def mark(i):
+            if ev is not None:
+                ev[i].record(stream)
+        mark(0)
+        zb.zb_landmark_build(Q, K, V, w.tile, out=layer.lm)
+        mark(1)
+        zb.zb_tile_score_topk(layer.lm.Qbar, layer.lm.Kbar, w.n_tokens, w.tile, w.k, out=layer.idx)
+        mark(2)
+        zb.zb_tile_sparse_attn(Q, K, V, layer.lm.Kbar_bf16, layer.lm.Vbar_bf16, layer.idx, w.k, w.tile, True,
+                               layer.scale, out=layer.O_sparse)
+        mark(3)
+        zb.zb_linear_state(K, V, layer.S, layer.z, layer.ws_lin)
+        mark(4)
+        zb.zb_gather_tiles(Q, w.tile, layer.calib, out=layer.Qc)
+        zb.zb_dense_attn(layer.Qc, K, V, layer.scale, out=layer.Yc)
+        mark(5)
+        zb.zb_linear_apply(layer.Qc, layer.S, layer.z, None, None, out=layer.Xc)
+        zb.zb_affine_fit(layer.Xc, layer.Yc, layer.A, layer.b, layer.ws_fit)
+        mark(6)
+        zb.zb_linear_apply(Q, layer.S, layer.z, layer.A, layer.b, out=layer.O_linear)
+        mark(7)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    zb.zb_last_device_status()
+    if args.profile:
+        step()
+        torch.cuda.synchronize()
+        zb.zb_last_device_status()
+        if rank == 0:
+            print(json.dumps({"profile_run": True, "workload": w.name}))
+        return 0
+
+    events = [[torch.cuda.Event(enable_timing=True) for _ in range(8)] for _ in range(args.steps)]
+    clocks = ClockSampler(local_rank)
+    replicas.barrier(dev)
+    torch.cuda.synchronize()
+    clocks.start()
+    t_start = torch.cuda.Event(enable_timing=True)
+    t_end = torch.cuda.Event(enable_timing=True)
+    t_start.record(stream)
+    for s in range(args.steps):
+        step(events[s])
+    t_end.record(stream)
+    torch.cuda.synchronize()
+    clk = clocks.stop()
+    replicas.barrier(dev)
+    zb.zb_last_device_status()
+    secs = t_start.elapsed_time(t_end) / 1e3
+    tokens_per_step = 2.0 * w.n_tokens  # both stage types of the 0.5L hybrid layer
+    tput, t_max = replicas.job_throughput(tokens_per_step, args.steps, secs, dev)
+    ms_per_step = t_max / args.steps * 1e3
+
+    per = {n: [] for n in names}
+    for ev in events:
+        for i, n in enumerate(names):
+            per[n].append(ev[i].elapsed_time(ev[i + 1]) / 1e3)
+    kt = {n: statistics.mean(v) for n, v in per.items()}
+
+    peaks = measured_peaks()
+    idx_cpu = layer.idx.cpu().numpy()
+    flops = selected_flops(idx_cpu, w.n_tokens, w.tile, w.head_dim)
+    sparse_tf = flops / kt["sparse_attn"] / 1e12
+    H, N, d = w.heads, w.n_tokens, w.head_dim
+    tensor_bytes = H * N * d * 2
+    lm_bytes = 3 * tensor_bytes                      # reads Q, K, V once
+    lin_state_bytes = 2 * tensor_bytes               # reads K, V
+    lin_apply_bytes = 2 * tensor_bytes               # reads Q, writes O
+    hbm = peaks["hbm_gbs"]
+    roofline = {"kernel": "zb_tile_sparse_attn", "bound": "tensor", "achieved": sparse_tf,
+                "peak": peaks["bf16_tflops_sustained"], "unit": "TFLOP/s",
+                "frac": sparse_tf / peaks["bf16_tflops_sustained"], "traffic": None,
+                "peak_kind": f"bf16 sustained ({peaks['source']}); kernel runs inside a long step",
+                "frac_of_burst": sparse_tf / peaks["bf16_tflops"],
+                "algorithmic": f"{flops:.4e} FLOP per launch = 4*d*sum n_i*n_j over kept (query tile, key tile) pairs"}
+    kernel_rooflines = {
+        "zb_landmark_build": {"bound": "hbm", "achieved": lm_bytes / kt["landmark"] / 1e9, "peak": hbm,
+                              "unit": "GB/s", "frac": lm_bytes / kt["landmark"] / 1e9 / hbm, "ms": kt["landmark"] * 1e3},
+        "zb_linear_state": {"bound": "hbm", "achieved": lin_state_bytes / kt["linear_state"] / 1e9, "peak": hbm,
+                            "unit": "GB/s", "frac": lin_state_bytes / kt["linear_state"] / 1e9 / hbm,
+                            "ms": kt["linear_state"] * 1e3},
+        "zb_linear_apply": {"bound": "hbm", "achieved": lin_apply_bytes / kt["linear_apply"] / 1e9, "peak": hbm,
+                            "unit": "GB/s", "frac": lin_apply_bytes / kt["linear_apply"] / 1e9 / hbm,
+                            "ms": kt["linear_apply"] * 1e3},
+        "zb_linear_attn (state + apply)": {
+            "bound": "hbm", "achieved": (lin_state_bytes + lin_apply_bytes) / (kt["linear_state"] + kt["linear_apply"]) / 1e9,
+            "peak": hbm, "unit": "GB/s",
+            "frac": (lin_state_bytes + lin_apply_bytes) / (kt["linear_state"] + kt["linear_apply"]) / 1e9 / hbm},
+        "zb_tile_score_topk": {"ms": kt["topk"] * 1e3, "bound": "alu (fp64)", "note": "reported only"},
+        "calibration (dense 4,096 rows + fit)": {"ms": (kt["calib_dense"] + kt["calib_rest"]) * 1e3},
+    }
+    stage_ms = {"sparse_stage": (kt["landmark"] + kt["topk"] + kt["sparse_attn"]) * 1e3,
+                "linear_stage": (kt["linear_state"] + kt["calib_dense"] + kt["calib_rest"] + kt["linear_apply"]) * 1e3,
+                "linear_stage_without_fit": (kt["linear_state"] + kt["linear_apply"]) * 1e3}
+
+    # ------------------------------------------------------------ e2e ----
+    e2e = None
+    if not args.no_e2e:
+        pin = [torch.empty(t.shape, dtype=t.dtype, pin_memory=True) for t in (Q, K, V)]
+        outs = [torch.empty(Q.shape, dtype=Q.dtype, pin_memory=True) for _ in range(2)]
+        for p, t in zip(pin, (Q, K, V)):
+            p.copy_(t)
+        e2e_steps = max(1, min(args.steps, 3))
+
+        def e2e_step():
+            for p, t in zip(pin, (Q, K, V)):
+                t.copy_(p, non_blocking=True)
+            step()
+            outs[0].copy_(layer.O_sparse, non_blocking=True)
+            outs[1].copy_(layer.O_linear, non_blocking=True)
+
+        e2e_step()
+        torch.cuda.synchronize()
+        replicas.barrier(dev)
+        a = torch.cuda.Event(enable_timing=True)
+        bb = torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(e2e_steps):
+            e2e_step()
+        bb.record(stream)
+        torch.cuda.synchronize()
+        replicas.barrier(dev)
+        e_secs = a.elapsed_time(bb) / 1e3
+        e_tput, _ = replicas.job_throughput(tokens_per_step, e2e_steps, e_secs, dev)
+        e2e = {"value": e_tput / 1e6, "unit": UNIT, "h2d_bytes_per_step": 3 * tensor_bytes,
+               "d2h_bytes_per_step": 2 * tensor_bytes, "steps": e2e_steps,
+               "api": "HybridLayer C-ABI calls with inputs copied from pinned host memory and both "
+                      "outputs copied back inside the timed region"}
+        del pin, outs
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu:
+        t_cpu, desc, cores = oracle_sample(w, Q, K, V, calib)
+        cpu = {"value": tokens_per_step / t_cpu / 1e6, "unit": UNIT, "cores": cores, "kind": "oracle",
+               "sample": desc}
+
+    if rank == 0:
+        line = {"metric": METRIC, "value": tput / 1e6, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+                "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
+                "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+                "config": config_dict(w), "e2e": e2e, "gpu_launches": layer.launches_per_step * args.steps,
+                "roofline": roofline, "kernel_roofline": kernel_rooflines, "stage_ms": stage_ms,
+                "kernel_ms": {n: v * 1e3 for n, v in kt.items()}, "clocks": clk, "cpu_baseline": cpu,
+                "peaks": peaks}
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        torch.distributed.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -45,7 +45,7 @@ import numpy as np
 __all__ = [
     "tile_lengths", "landmark_means", "tile_scores", "select_tiles",
     "sparse_attention", "dense_attention", "elu_plus_one", "linear_state",
-    "linear_attention", "linear_attention_quadratic", "affine_fit",
+    "linear_apply", "linear_attention", "linear_attention_quadratic", "affine_fit",
     "affine_apply", "calibration_rows",
 ]
 
@@ -224,11 +224,15 @@ def linear_attention(Q, K, V, A=None, b=None) -> np.ndarray:
     [ABS]'s page).
     """
     S, z = linear_state(K, V)
+    return linear_apply(Q, S, z, A, b)
+
+
+def linear_apply(Q, S, z, A=None, b=None) -> np.ndarray:
+    """Output of the linear stage from a given state: (phi(q) S / (phi(q) . z)) A + b."""
     fq = elu_plus_one(Q)
-    num = np.matmul(fq, S)
-    den = np.matmul(fq, z[..., None])
-    O = num / den
-    return affine_apply(O, A, b)
+    num = np.matmul(fq, _f64(S))
+    den = np.matmul(fq, _f64(z)[..., None])
+    return affine_apply(num / den, A, b)
 
 
 def linear_attention_quadratic(Q, K, V) -> np.ndarray:
