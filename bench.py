@@ -264,7 +264,8 @@ def main():
         mark(0)
         zb.zb_landmark_build(Q, K, V, w.tile, out=layer.lm)
         mark(1)
-        zb.zb_tile_score_topk(layer.lm.Qbar, layer.lm.Kbar, w.n_tokens, w.tile, w.k, out=layer.idx)
+        zb.zb_tile_score_topk(layer.lm.Qbar, layer.lm.Kbar, w.n_tokens, w.tile, w.k, out=layer.idx,
+                              ws=layer.ws_topk)
         mark(2)
         zb.zb_tile_sparse_attn(Q, K, V, layer.lm.Kbar_bf16, layer.lm.Vbar_bf16, layer.idx, w.k, w.tile, True,
                                layer.scale, out=layer.O_sparse)

@@ -95,12 +95,18 @@ zb_status zb_landmark_build(const uint16_t* Q, const uint16_t* K, const uint16_t
  * mean-pooled reading.  The budget k is the kept share of the key tiles (the
  * y in "xL/yS" of the Table 20 caption is the dropped share).
  *   in : Qbar, Kbar fp64 [H][T][d];  0 <= k <= T
+ *   ws : scratch for the fp64 score matrix of a group of heads; at least
+ *        T*T*8 bytes (one head per pass), up to H*T*T*8 (all heads in one
+ *        pass).  zb_tile_score_topk_workspace_bytes() gives a default (4
+ *        heads).  Not needed (may be NULL) when k == 0 or k == T.
  *   out: idx int32 [H][T][k]
- * Needs no workspace.  Errors: ZB_ERR_NULL, ZB_ERR_SHAPE, ZB_ERR_ALIGN,
- * ZB_ERR_UNSUPPORTED (T > 32768), ZB_ERR_CUDA.
+ * Errors: ZB_ERR_NULL, ZB_ERR_SHAPE, ZB_ERR_ALIGN, ZB_ERR_UNSUPPORTED (T > 32768),
+ * ZB_ERR_WORKSPACE, ZB_ERR_CUDA.
  */
+size_t zb_tile_score_topk_workspace_bytes(zb_shape s);
 zb_status zb_tile_score_topk(const double* Qbar, const double* Kbar, zb_shape s,
-                             int32_t k, int32_t* idx, void* stream);
+                             int32_t k, int32_t* idx, void* ws, size_t ws_bytes,
+                             void* stream);
 
 /*
  * Tile-sparse softmax attention with landmarks (Figure 1 (a) caption; section

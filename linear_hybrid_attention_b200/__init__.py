@@ -35,7 +35,7 @@ HEAD_DIM = 64
 
 # kernels each entry point launches (for counting launches in a timed region)
 LAUNCHES_PER_CALL = {
-    "zb_landmark_build": 1, "zb_tile_score_topk": 1, "zb_tile_sparse_attn": 1, "zb_dense_attn": 1,
+    "zb_landmark_build": 1, "zb_tile_score_topk": 2, "zb_tile_sparse_attn": 1, "zb_dense_attn": 1,
     "zb_linear_state": 2, "zb_linear_apply": 1, "zb_affine_fit": 3, "zb_gather_tiles": 1,
 }
 
@@ -123,15 +123,22 @@ def zb_landmark_build(Q: Optional[torch.Tensor], K: torch.Tensor, V: torch.Tenso
     return Landmarks(Qbar, Kbar, Kb, Vb)
 
 
+def topk_workspace_bytes(heads: int, n_tokens: int, tile: int, head_dim: int = HEAD_DIM) -> int:
+    return int(_lib_handle().zb_tile_score_topk_workspace_bytes(_lib.ZbShape(heads, n_tokens, head_dim, tile)))
+
+
 def zb_tile_score_topk(Qbar: torch.Tensor, Kbar: torch.Tensor, n_tokens: int, tile: int, k: int,
-                       out: Optional[torch.Tensor] = None) -> torch.Tensor:
+                       out: Optional[torch.Tensor] = None, ws: Optional[torch.Tensor] = None) -> torch.Tensor:
     """Indices [H, T, k] (int32, ascending) of the k best key tiles per query tile."""
     _need(Qbar, torch.float64, "Qbar", 3)
     _need(Kbar, torch.float64, "Kbar", 3)
     H, T, d = Kbar.shape
     idx = _out((H, T, k), torch.int32, Kbar.device, out, "idx")
+    need = topk_workspace_bytes(H, n_tokens, tile, d) if 0 < k < T else 0
+    wsb = _ws(need, Kbar.device, ws) if need else None
     st = _lib_handle().zb_tile_score_topk(_ptr(Qbar), _ptr(Kbar), _lib.ZbShape(H, n_tokens, d, tile),
-                                          int(k), _ptr(idx), _stream())
+                                          int(k), _ptr(idx), _ptr(wsb),
+                                          0 if wsb is None else wsb.numel() * wsb.element_size(), _stream())
     _check(st, "zb_tile_score_topk")
     return idx
 
@@ -287,6 +294,7 @@ class HybridLayer:
                             torch.empty(H, T, d, dtype=torch.bfloat16, device=dev),
                             torch.empty(H, T, d, dtype=torch.bfloat16, device=dev))
         self.idx = torch.empty(H, T, k, dtype=torch.int32, device=dev)
+        self.ws_topk = torch.empty(max(topk_workspace_bytes(H, N, tile, d), 16), dtype=torch.uint8, device=dev)
         self.O_sparse = torch.empty(H, N, d, dtype=torch.bfloat16, device=dev)
         self.O_linear = torch.empty(H, N, d, dtype=torch.bfloat16, device=dev)
         self.S = torch.empty(H, d, d, dtype=torch.float32, device=dev)
@@ -315,7 +323,8 @@ class HybridLayer:
 
     def sparse(self, Q, K, V) -> torch.Tensor:
         zb_landmark_build(Q, K, V, self.tile, out=self.lm)
-        zb_tile_score_topk(self.lm.Qbar, self.lm.Kbar, self.n_tokens, self.tile, self.k, out=self.idx)
+        zb_tile_score_topk(self.lm.Qbar, self.lm.Kbar, self.n_tokens, self.tile, self.k, out=self.idx,
+                           ws=self.ws_topk)
         return zb_tile_sparse_attn(Q, K, V, self.lm.Kbar_bf16, self.lm.Vbar_bf16, self.idx, self.k,
                                    self.tile, True, self.scale, out=self.O_sparse)
 

@@ -25,7 +25,8 @@ PROTOTYPES = {
     "zb_abi_version": (c_i32, []),
     "zb_status_string": (ctypes.c_char_p, [c_i32]),
     "zb_landmark_build": (c_i32, [c_vp, c_vp, c_vp, ZbShape, c_vp, c_vp, c_vp, c_vp, c_vp]),
-    "zb_tile_score_topk": (c_i32, [c_vp, c_vp, ZbShape, c_i32, c_vp, c_vp]),
+    "zb_tile_score_topk_workspace_bytes": (c_sz, [ZbShape]),
+    "zb_tile_score_topk": (c_i32, [c_vp, c_vp, ZbShape, c_i32, c_vp, c_vp, c_sz, c_vp]),
     "zb_tile_sparse_attn": (c_i32, [c_vp, c_vp, c_vp, c_vp, c_vp, c_vp, c_i32, c_i32, c_f32, ZbShape,
                                     c_vp, c_vp, c_vp]),
     "zb_dense_attn": (c_i32, [c_vp, c_i64, c_vp, c_vp, c_i64, c_i32, c_i32, c_f32, c_vp, c_vp, c_vp]),

@@ -356,42 +356,57 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                 }
                 tc_fence_before();
                 mbar_arrive(smem_addr(&sm.s_free[b]));
-                // logits in log2 units, masked
-                float mx = -INFINITY;
-                if (st < p.k) {
+                // ---- row max (tree of 3-input max; no long dependency chain)
+                // Selected tiles: max of the raw scores, scaled afterwards
+                // (scale > 0).  Landmark chunks: x = s * scale + bias first,
+                // bias = log2(n_j), or -inf for selected / out-of-range tiles.
+                const bool is_lm = st >= p.k;
+                const uint64_t c2 = f2_pack(p.scale_log2, p.scale_log2);
+                if (!is_lm) {
                     const int valid = (st == p.k - 1) ? last_valid : p.tk;
-                    if (valid >= BN) {
+                    if (valid < BN) {
 #pragma unroll
-                        for (int e = 0; e < BN; ++e) {
-                            x[e] *= p.scale_log2;
-                            mx = fmaxf(mx, x[e]);
-                        }
-                    } else {
-#pragma unroll
-                        for (int e = 0; e < BN; ++e) {
-                            x[e] = e < valid ? x[e] * p.scale_log2 : -INFINITY;
-                            mx = fmaxf(mx, x[e]);
-                        }
+                        for (int e = 0; e < BN; ++e)
+                            if (e >= valid) x[e] = -INFINITY;
                     }
                 } else {
-                    const int c = st - p.k;
-                    const int j0 = c * BN;
+                    const int j0 = (st - p.k) * BN;
 #pragma unroll
                     for (int w = 0; w < BN / 32; ++w) {
                         const int jw = j0 + w * 32;
-                        const uint32_t bits = (jw < p.Tk) ? bm[jw >> 5] : 0xFFFFFFFFu;
+                        uint32_t bits = (jw < p.Tk) ? bm[jw >> 5] : 0xFFFFFFFFu;
+                        if (jw + 32 > p.Tk) {  // the chunk runs past the last tile
+                            const int keep = p.Tk - jw;
+                            bits |= keep <= 0 ? 0xFFFFFFFFu : (0xFFFFFFFFu << keep);
+                        }
 #pragma unroll
-                        for (int e = 0; e < 32; ++e) {
+                        for (int e = 0; e < 32; e += 2) {
                             const int j = jw + e;
-                            float bias = (j == p.Tk - 1) ? p.log2_last : p.log2_tk;
-                            if (j >= p.Tk || ((bits >> e) & 1u)) bias = -INFINITY;
-                            const float v = fmaf(x[w * 32 + e], p.scale_log2, bias);
-                            x[w * 32 + e] = v;
-                            mx = fmaxf(mx, v);
+                            float b0 = (j == p.Tk - 1) ? p.log2_last : p.log2_tk;
+                            float b1 = (j + 1 == p.Tk - 1) ? p.log2_last : p.log2_tk;
+                            if ((bits >> e) & 1u) b0 = -INFINITY;
+                            if ((bits >> (e + 1)) & 1u) b1 = -INFINITY;
+                            float v0, v1;
+                            f2_unpack(f2_fma(f2_pack(x[w * 32 + e], x[w * 32 + e + 1]), c2, f2_pack(b0, b1)), v0, v1);
+                            x[w * 32 + e] = v0;
+                            x[w * 32 + e + 1] = v1;
                         }
                     }
                 }
-                // lazy rescale: keep the old max unless the new one exceeds it by > 8
+                float mx;
+                {
+                    float g[8];
+#pragma unroll
+                    for (int q = 0; q < 8; ++q) {
+                        float t = fmax3(x[16 * q], x[16 * q + 1], x[16 * q + 2]);
+#pragma unroll
+                        for (int e = 3; e < 15; e += 2) t = fmax3(t, x[16 * q + e], x[16 * q + e + 1]);
+                        g[q] = fmaxf(t, x[16 * q + 15]);
+                    }
+                    mx = fmax3(fmax3(g[0], g[1], g[2]), fmax3(g[3], g[4], g[5]), fmaxf(g[6], g[7]));
+                }
+                if (!is_lm) mx *= p.scale_log2;
+                // ---- lazy rescale: keep the old max unless the new one exceeds it by > 8
                 const float m_new = fmaxf(m, mx);
                 const bool rescale = m_new > m + RESCALE_THRESHOLD;
                 float alpha = 1.f;
@@ -401,16 +416,35 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                     l *= alpha;
                 }
                 const float msub = (m == -INFINITY) ? 0.f : m;
+                // ---- p = 2^(x - m): 3 of every 8 pairs on the FMA pipes, the
+                // rest on MUFU; packed fp32x2 arithmetic; 4 independent sums
                 uint32_t pk[BN / 2];
-                float rs = 0.f;
+                const uint64_t nm2 = f2_pack(-msub, -msub);
+                uint64_t acc[4] = {0ull, 0ull, 0ull, 0ull};
 #pragma unroll
-                for (int e = 0; e < BN; e += 2) {
-                    const float p0 = ex2(x[e] - msub);
-                    const float p1 = ex2(x[e + 1] - msub);
-                    rs += p0 + p1;
-                    pk[e / 2] = pack_bf16x2(p0, p1);
+                for (int q = 0; q < BN / 2; ++q) {
+                    const uint64_t xin = f2_pack(x[2 * q], x[2 * q + 1]);
+                    const uint64_t xs = is_lm ? f2_add(xin, nm2) : f2_fma(xin, c2, nm2);
+                    uint64_t pv;
+                    if ((q & 7) < 3) {
+                        pv = f2_exp2_poly(xs);
+                    } else {
+                        float a0, a1;
+                        f2_unpack(xs, a0, a1);
+                        pv = f2_pack(ex2(a0), ex2(a1));
+                    }
+                    acc[q & 3] = f2_add(acc[q & 3], pv);
+                    float p0, p1;
+                    f2_unpack(pv, p0, p1);
+                    pk[q] = pack_bf16x2(p0, p1);
                 }
-                l += rs;
+                {
+                    float s0, s1, s2, s3;
+                    f2_unpack(f2_add(f2_add(acc[0], acc[1]), f2_add(acc[2], acc[3])), s0, s1);
+                    (void)s2;
+                    (void)s3;
+                    l += s0 + s1;
+                }
                 // P buffer b is free once PV of step gg-2 is done
                 if (!mbar_wait(smem_addr(&sm.p_free[b]), (buse & 1) ^ 1, wc)) { ok = false; break; }
                 if (rescale && st > 0) {

@@ -45,80 +45,139 @@ __device__ __forceinline__ uint16_t f64_to_bf16_rne(double x) {
     return static_cast<uint16_t>(__float_as_uint(f) >> 16);
 }
 
-__global__ void __launch_bounds__(THREADS)
+// Persistent landmark kernel: one CTA per SM walks (head, tile) items
+// round-robin.  Thread 0 copies the Q, K, V runs of an item (n_j rows x 128 B
+// each, contiguous) into a LM_STAGES-deep shared-memory ring with bulk copies;
+// warp w sums rows [16 w, 16 w + 16) of each tensor, lane l columns 2l, 2l+1,
+// in fp64 (exact for bf16 inputs unless a tile spans > ~38 binades); the 8
+// warp partials are added in a fixed order by 192 threads, one output each.
+constexpr int LM_STAGES = 4;
+constexpr uint32_t RUN_BYTES = 128 * HD * 2;  // one full tile of one tensor
+
+struct LmSmem {
+    uint8_t buf[LM_STAGES][3][RUN_BYTES];
+    double part[2][THREADS / 32][3][HD];
+    uint64_t full[LM_STAGES];
+    int abort_flag;
+};
+
+__global__ void __launch_bounds__(THREADS, 1)
 landmark_kernel(const uint16_t* __restrict__ Q, const uint16_t* __restrict__ K,
                 const uint16_t* __restrict__ V, int heads, long long N, int tile, int T,
                 double* __restrict__ Qbar, double* __restrict__ Kbar, uint16_t* __restrict__ Kb16,
-                uint16_t* __restrict__ Vb16) {
-    __shared__ double part[3][THREADS / 32][8][8];  // [tensor][warp][col group][col]
-    const int tid = threadIdx.x;
-    const int cg = tid & 7;          // 16-byte column group (8 columns)
-    const int rs = tid >> 3;         // row slot 0..31
-    const int warp = tid >> 5, lane = tid & 31;
+                uint16_t* __restrict__ Vb16, int* status, unsigned long long timeout_ns) {
+    extern __shared__ uint8_t smem_raw[];
+    LmSmem& sm = *reinterpret_cast<LmSmem*>((reinterpret_cast<uintptr_t>(smem_raw) + 127) & ~uintptr_t(127));
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const bool do_q = Q != nullptr;
+    const int nt = do_q ? 3 : 2;         // tensors copied per item
+    const int t0 = do_q ? 0 : 1;         // first tensor slot used (0 = Q, 1 = K, 2 = V)
     const long long total = static_cast<long long>(heads) * T;
-    for (long long w = blockIdx.x; w < total; w += gridDim.x) {
-        const int h = static_cast<int>(w / T);
-        const int j = static_cast<int>(w % T);
-        const long long r0 = static_cast<long long>(j) * tile;
-        const int n = static_cast<int>(min(static_cast<long long>(tile), N - r0));
-        const long long base = (static_cast<long long>(h) * N + r0) * HD;
-        double aq[8] = {0, 0, 0, 0, 0, 0, 0, 0}, ak[8] = {0, 0, 0, 0, 0, 0, 0, 0},
-               av[8] = {0, 0, 0, 0, 0, 0, 0, 0};
-        // issue all loads of this thread first, then accumulate (memory-level parallelism)
-        uint4 lq[4], lk[4], lv[4];
+    const long long first = blockIdx.x;
+    const int cnt = first < total ? static_cast<int>((total - 1 - first) / gridDim.x + 1) : 0;
+    const WaitCtx wc{status, &sm.abort_flag, timeout_ns};
+    if (tid == 0) {
+        sm.abort_flag = 0;
+        for (int s = 0; s < LM_STAGES; ++s) mbar_init(smem_addr(&sm.full[s]), 1);
+        fence_mbar_init();
+    }
+    __syncthreads();
+
+    auto item_of = [&](int it, int& h, int& j, int& n) {
+        const long long w = first + static_cast<long long>(it) * gridDim.x;
+        h = static_cast<int>(w / T);
+        j = static_cast<int>(w % T);
+        n = static_cast<int>(min(static_cast<long long>(tile), N - static_cast<long long>(j) * tile));
+    };
+    auto issue = [&](int it) {
+        int h, j, n;
+        item_of(it, h, j, n);
+        const int s = it % LM_STAGES;
+        const uint32_t bar = smem_addr(&sm.full[s]);
+        const uint32_t bytes = static_cast<uint32_t>(n) * HD * 2;
+        const long long off = (static_cast<long long>(h) * N + static_cast<long long>(j) * tile) * HD;
+        mbar_arrive_expect_tx(bar, bytes * nt);
+        if (do_q) bulk_load(smem_addr(sm.buf[s][0]), Q + off, bytes, bar);
+        bulk_load(smem_addr(sm.buf[s][1]), K + off, bytes, bar);
+        bulk_load(smem_addr(sm.buf[s][2]), V + off, bytes, bar);
+    };
+    int issued = 0;
+    if (tid == 0)
+        for (int it = 0; it < LM_STAGES && it < cnt; ++it) issue(it), ++issued;
+
+    int consumed = 0;
+    for (int it = 0; it < cnt; ++it) {
+        const int s = it % LM_STAGES;
+        int h, j, n;
+        item_of(it, h, j, n);
+        const bool good = mbar_wait(smem_addr(&sm.full[s]), (it / LM_STAGES) & 1, wc);
+        if (good) consumed = it + 1;
+        const int r0 = warp * 16;
+        const int rows = good ? max(0, min(16, n - r0)) : 0;
 #pragma unroll
-        for (int m = 0; m < 4; ++m) {
-            const int r = rs + 32 * m;
-            const bool in = r < n;
-            const long long off = base + static_cast<long long>(r) * HD + cg * 8;
-            lk[m] = in ? __ldg(reinterpret_cast<const uint4*>(K + off)) : make_uint4(0, 0, 0, 0);
-            lv[m] = in ? __ldg(reinterpret_cast<const uint4*>(V + off)) : make_uint4(0, 0, 0, 0);
-            lq[m] = (in && do_q) ? __ldg(reinterpret_cast<const uint4*>(Q + off)) : make_uint4(0, 0, 0, 0);
-        }
+        for (int t = 0; t < 3; ++t) {
+            double a0 = 0.0, a1 = 0.0;
+            if (t >= t0) {
+                const uint32_t* src = reinterpret_cast<const uint32_t*>(sm.buf[s][t]) + r0 * (HD / 2) + lane;
+                if (rows == 16) {
+                    // all loads first, then a tree of adds (sums are exact, order-free)
+                    uint32_t wv[16];
 #pragma unroll
-        for (int m = 0; m < 4; ++m) {
-            add8(ak, lk[m]);
-            add8(av, lv[m]);
-            if (do_q) add8(aq, lq[m]);
-        }
-        // reduce over the 4 row slots of this warp that share cg (lanes cg, cg+8, cg+16, cg+24)
+                    for (int r = 0; r < 16; ++r) wv[r] = src[r * (HD / 2)];
+                    double l[8], h[8];
 #pragma unroll
-        for (int c = 0; c < 8; ++c) {
+                    for (int r = 0; r < 8; ++r) {
+                        l[r] = static_cast<double>(bf16_lo(wv[2 * r])) + static_cast<double>(bf16_lo(wv[2 * r + 1]));
+                        h[r] = static_cast<double>(bf16_hi(wv[2 * r])) + static_cast<double>(bf16_hi(wv[2 * r + 1]));
+                    }
 #pragma unroll
-            for (int o = 8; o <= 16; o <<= 1) {
-                ak[c] += __shfl_xor_sync(0xffffffffu, ak[c], o);
-                av[c] += __shfl_xor_sync(0xffffffffu, av[c], o);
-                aq[c] += __shfl_xor_sync(0xffffffffu, aq[c], o);
+                    for (int w = 4; w >= 1; w >>= 1)
+#pragma unroll
+                        for (int r = 0; r < w; ++r) {
+                            l[r] += l[r + w];
+                            h[r] += h[r + w];
+                        }
+                    a0 = l[0];
+                    a1 = h[0];
+                } else {
+                    for (int r = 0; r < rows; ++r) {
+                        const uint32_t wv = src[r * (HD / 2)];
+                        a0 += static_cast<double>(bf16_lo(wv));
+                        a1 += static_cast<double>(bf16_hi(wv));
+                    }
+                }
             }
+            sm.part[it & 1][warp][t][2 * lane] = a0;
+            sm.part[it & 1][warp][t][2 * lane + 1] = a1;
         }
-        if (lane < 8) {
-#pragma unroll
-            for (int c = 0; c < 8; ++c) {
-                part[0][warp][cg][c] = aq[c];
-                part[1][warp][cg][c] = ak[c];
-                part[2][warp][cg][c] = av[c];
-            }
-        }
-        __syncthreads();
+        fence_proxy_async_smem();  // our reads of buf[s] precede the next bulk write into it
+        if (__syncthreads_or(!good)) break;
+        if (tid == 0 && it + LM_STAGES < cnt) issue(it + LM_STAGES), ++issued;
         if (tid < 3 * HD) {
-            const int t = tid / HD;       // 0 = Q, 1 = K, 2 = V
-            const int col = tid % HD;
-            double s = 0.0;
+            const int t = tid / HD, col = tid % HD;
+            if (t >= t0) {
+                double acc = 0.0;
 #pragma unroll
-            for (int wp = 0; wp < THREADS / 32; ++wp) s += part[t][wp][col >> 3][col & 7];
-            const double mean = s / static_cast<double>(n);
-            const long long o = (static_cast<long long>(h) * T + j) * HD + col;
-            if (t == 0) {
-                if (do_q) Qbar[o] = mean;
-            } else if (t == 1) {
-                Kbar[o] = mean;
-                Kb16[o] = f64_to_bf16_rne(mean);
-            } else {
-                Vb16[o] = f64_to_bf16_rne(mean);
+                for (int wp = 0; wp < THREADS / 32; ++wp) acc += sm.part[it & 1][wp][t][col];
+                const double mean = acc / static_cast<double>(n);
+                const long long o = (static_cast<long long>(h) * T + j) * HD + col;
+                if (t == 0) {
+                    Qbar[o] = mean;
+                } else if (t == 1) {
+                    Kbar[o] = mean;
+                    Kb16[o] = f64_to_bf16_rne(mean);
+                } else {
+                    Vb16[o] = f64_to_bf16_rne(mean);
+                }
             }
         }
-        __syncthreads();
+    }
+    // leave no bulk copy in flight
+    if (tid == 0) {
+        volatile int no_abort = 0;
+        const WaitCtx w2{status, &no_abort, timeout_ns};
+        for (int q = consumed; q < issued; ++q)
+            mbar_wait(smem_addr(&sm.full[q % LM_STAGES]), (q / LM_STAGES) & 1, w2);
     }
 }
 
@@ -164,9 +223,14 @@ extern "C" zb_status zb_landmark_build(const uint16_t* Q, const uint16_t* K, con
     if ((e = current_device(&dev)) != ZB_OK) return e;
     const int T = static_cast<int>(n_tiles(s));
     const long long total = static_cast<long long>(s.heads) * T;
-    const long long grid = total < 8ll * dev.sm_count ? total : 8ll * dev.sm_count;
-    lmk::landmark_kernel<<<static_cast<unsigned>(grid), lmk::THREADS, 0, static_cast<cudaStream_t>(stream)>>>(
-        Q, K, V, s.heads, s.n_tokens, s.tile, T, Qbar, Kbar, Kbar_bf16, Vbar_bf16);
+    const long long grid = total < dev.sm_count ? total : dev.sm_count;
+    const size_t smem = sizeof(lmk::LmSmem) + 128;
+    if (cudaFuncSetAttribute(lmk::landmark_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(smem)) != cudaSuccess)
+        return ZB_ERR_CUDA;
+    lmk::landmark_kernel<<<static_cast<unsigned>(grid), lmk::THREADS, smem, static_cast<cudaStream_t>(stream)>>>(
+        Q, K, V, s.heads, s.n_tokens, s.tile, T, Qbar, Kbar, Kbar_bf16, Vbar_bf16, dev.status,
+        wait_timeout_ns());
     return cudaGetLastError() == cudaSuccess ? ZB_OK : ZB_ERR_CUDA;
 }
 

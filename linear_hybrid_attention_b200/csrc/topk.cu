@@ -6,10 +6,15 @@
 // Reading used: score(i, j) = Qbar_i . Kbar_j in fp64, the k largest kept,
 // equal scores resolved toward the lower key-tile index, output ascending.
 //
-// One CTA scores R query tiles of one head against all T key tiles (scores
-// kept in shared memory as fp64), then, row by row, finds the k-th largest
-// score with an 8-bit-digit radix select on order-preserving 64-bit keys, and
-// writes the kept indices in ascending order with block-wide prefix sums.
+// Two kernels per group of heads (as many heads as the workspace holds):
+//  * score_gemm_kernel: register-tiled fp64 GEMM, 128 x 128 scores per CTA,
+//    8 x 8 per thread, full d = 64 staged (transposed) in shared memory; each
+//    score is one FMA chain over d in index order.  Scores go to the workspace.
+//  * select_kernel: one CTA per (head, query tile); the T scores are copied to
+//    shared memory, the k-th largest is found by an 8-bit-digit radix select on
+//    order-preserving 64-bit keys (warp-aggregated histogram atomics, early
+//    exit once the bucket holds exactly the remaining count), and the kept
+//    indices are written in ascending order with two block-wide prefix sums.
 #include <cuda_runtime.h>
 
 #include "zb_common.cuh"
@@ -18,10 +23,12 @@
 namespace zb {
 namespace topk {
 
-constexpr int THREADS = 256;
 constexpr int HD = 64;
-constexpr size_t SCORE_SMEM_BUDGET = 200 * 1024;
-constexpr int MAX_ROWS = 32;
+constexpr int GT = 128;            // GEMM CTA tile (rows and columns)
+constexpr int GTHREADS = 256;
+constexpr int STHREADS = 512;
+constexpr int MAX_T = 32768;
+constexpr size_t SMEM_SCORE_LIMIT = 200 * 1024;  // scores kept in smem up to this size
 
 // Order-preserving map of an fp64 value to uint64 (larger value -> larger key);
 // -0.0 is folded onto +0.0 so that they tie.
@@ -31,8 +38,63 @@ __device__ __forceinline__ unsigned long long order_key(double s) {
     return (u >> 63) ? ~u : (u | 0x8000000000000000ull);
 }
 
-// Block-wide exclusive prefix sum of one int per thread; returns the exclusive
-// value, writes the block total to *total.  Uses `scratch` (>= THREADS/32 ints).
+// ------------------------------------------------------------- GEMM ----
+// grid: (ceil(T/128) column blocks, ceil(T/128) row blocks, heads in group).
+// Shared memory holds the 128-row blocks of Qbar and Kbar transposed, with a
+// row stride of 129 doubles so that the transposing stores and the inner-loop
+// reads are bank-conflict free; thread (ty, tx) owns rows ty + 16 a and
+// columns tx + 16 b (a, b < 8), so a warp reads 16 consecutive doubles.
+constexpr int GS = GT + 1;
+
+__global__ void __launch_bounds__(GTHREADS)
+score_gemm_kernel(const double* __restrict__ Qbar, const double* __restrict__ Kbar, int T, int h0,
+                  double* __restrict__ scores) {
+    extern __shared__ __align__(16) uint8_t smem_raw[];
+    double* qt = reinterpret_cast<double*>(smem_raw);  // [64][129]
+    double* kt = qt + HD * GS;                         // [64][129]
+    const int h = h0 + blockIdx.z;
+    const int i0 = blockIdx.y * GT, j0 = blockIdx.x * GT;
+    const double* qh = Qbar + static_cast<long long>(h) * T * HD;
+    const double* kh = Kbar + static_cast<long long>(h) * T * HD;
+    for (int e = threadIdx.x; e < GT * HD; e += GTHREADS) {
+        const int r = e / HD, c = e % HD;  // coalesced global reads
+        qt[c * GS + r] = (i0 + r < T) ? qh[static_cast<long long>(i0 + r) * HD + c] : 0.0;
+        kt[c * GS + r] = (j0 + r < T) ? kh[static_cast<long long>(j0 + r) * HD + c] : 0.0;
+    }
+    __syncthreads();
+    const int ty = threadIdx.x >> 4, tx = threadIdx.x & 15;
+    double acc[8][8];
+#pragma unroll
+    for (int a = 0; a < 8; ++a)
+#pragma unroll
+        for (int b = 0; b < 8; ++b) acc[a][b] = 0.0;
+#pragma unroll 2
+    for (int c = 0; c < HD; ++c) {
+        double qv[8], kv[8];
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+            qv[u] = qt[c * GS + ty + 16 * u];
+            kv[u] = kt[c * GS + tx + 16 * u];
+        }
+#pragma unroll
+        for (int a = 0; a < 8; ++a)
+#pragma unroll
+            for (int b = 0; b < 8; ++b) acc[a][b] = fma(qv[a], kv[b], acc[a][b]);
+    }
+    double* out = scores + static_cast<long long>(blockIdx.z) * T * T;
+#pragma unroll
+    for (int a = 0; a < 8; ++a) {
+        const int i = i0 + ty + 16 * a;
+        if (i >= T) continue;
+#pragma unroll
+        for (int b = 0; b < 8; ++b) {
+            const int j = j0 + tx + 16 * b;
+            if (j < T) out[static_cast<long long>(i) * T + j] = acc[a][b];
+        }
+    }
+}
+
+// Block-wide exclusive prefix sum of one int per thread (STHREADS threads).
 __device__ __forceinline__ int block_excl_scan(int v, int* scratch, int* total) {
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     int x = v;
@@ -45,7 +107,7 @@ __device__ __forceinline__ int block_excl_scan(int v, int* scratch, int* total) 
     __syncthreads();
     int wsum = 0, tot = 0;
 #pragma unroll
-    for (int w = 0; w < THREADS / 32; ++w) {
+    for (int w = 0; w < STHREADS / 32; ++w) {
         const int s = scratch[w];
         if (w < warp) wsum += s;
         tot += s;
@@ -55,164 +117,173 @@ __device__ __forceinline__ int block_excl_scan(int v, int* scratch, int* total) 
     return wsum + x - v;
 }
 
-__global__ void __launch_bounds__(THREADS)
-score_topk_kernel(const double* __restrict__ Qbar, const double* __restrict__ Kbar, int heads,
-                  int T, int k, int rows_per_cta, int32_t* __restrict__ idx) {
+// ----------------------------------------------------------- select ----
+// grid: heads in group x T rows.  Scores of the row in shared memory when they
+// fit (`in_smem`), else read from the workspace on every pass.
+__global__ void __launch_bounds__(STHREADS)
+select_kernel(const double* __restrict__ scores, int T, int k, int h0, int in_smem,
+              int32_t* __restrict__ idx) {
     extern __shared__ __align__(16) uint8_t smem_raw[];
-    double* qs = reinterpret_cast<double*>(smem_raw);                 // [R][64]
-    double* sc = qs + static_cast<size_t>(rows_per_cta) * HD;        // [R][T]
     __shared__ unsigned int hist[256];
-    __shared__ int scan_scratch[THREADS / 32];
+    __shared__ int scan_scratch[STHREADS / 32];
     __shared__ int sel_bucket, sel_above;
-
     const int tid = threadIdx.x;
-    const int blocks_per_head = (T + rows_per_cta - 1) / rows_per_cta;
-    const int h = blockIdx.x / blocks_per_head;
-    const int i0 = (blockIdx.x % blocks_per_head) * rows_per_cta;
-    const int R = min(rows_per_cta, T - i0);
-    const double* qh = Qbar + (static_cast<long long>(h) * T + i0) * HD;
-    const double* kh = Kbar + static_cast<long long>(h) * T * HD;
-
-    for (int e = tid; e < R * HD; e += THREADS) qs[e] = qh[e];
-    __syncthreads();
-
-    // ---- scores: thread owns key tiles j = tid, tid + 256, ...; fp64 FMA chain over d
-    for (int j = tid; j < T; j += THREADS) {
-        double acc[MAX_ROWS];
-#pragma unroll
-        for (int r = 0; r < MAX_ROWS; ++r) acc[r] = 0.0;
-        const double2* kj = reinterpret_cast<const double2*>(kh + static_cast<long long>(j) * HD);
-#pragma unroll 4
-        for (int c2 = 0; c2 < HD / 2; ++c2) {
-            const double2 kv = __ldg(kj + c2);
-#pragma unroll
-            for (int r = 0; r < MAX_ROWS; ++r) {
-                if (r < R) {
-                    const double2 qv = reinterpret_cast<const double2*>(qs + r * HD)[c2];
-                    acc[r] = fma(qv.x, kv.x, acc[r]);
-                    acc[r] = fma(qv.y, kv.y, acc[r]);
-                }
-            }
-        }
-#pragma unroll
-        for (int r = 0; r < MAX_ROWS; ++r)
-            if (r < R) sc[static_cast<size_t>(r) * T + j] = acc[r];
-    }
-    __syncthreads();
-
-    for (int r = 0; r < R; ++r) {
-        const double* row = sc + static_cast<size_t>(r) * T;
-        int32_t* out = idx + (static_cast<long long>(h) * T + i0 + r) * static_cast<long long>(k);
-        if (k == 0) continue;
-        if (k == T) {
-            for (int j = tid; j < T; j += THREADS) out[j] = j;
-            continue;
-        }
-        // ---- radix select of the k-th largest key, 8 bits per pass from the top
-        unsigned long long prefix = 0, mask = 0;
-        int need = k;
-        for (int shift = 56; shift >= 0; shift -= 8) {
-            for (int b = tid; b < 256; b += THREADS) hist[b] = 0u;
-            __syncthreads();
-            // uniform trip count: every lane reaches the warp-collective calls
-            for (int j0 = 0; j0 < T; j0 += THREADS) {
-                const int j = j0 + tid;
-                const unsigned long long key = j < T ? order_key(row[j]) : 0ull;
-                const bool m = j < T && (key & mask) == prefix;
-                const unsigned int digit = static_cast<unsigned int>((key >> shift) & 0xFFu);
-                const unsigned int active = __ballot_sync(0xffffffffu, m);
-                if (m) {
-                    const unsigned int peers = __match_any_sync(active, digit);
-                    if ((__ffs(peers) - 1) == (tid & 31)) atomicAdd(&hist[digit], __popc(peers));
-                }
-            }
-            __syncthreads();
-            if (tid < 32) {
-                // lane l owns bins 8l..8l+7; find the bin holding the need-th largest
-                unsigned int c[8], lsum = 0;
-#pragma unroll
-                for (int e = 0; e < 8; ++e) lsum += (c[e] = hist[tid * 8 + e]);
-                // inclusive suffix sum over lanes: x = sum of lanes >= tid
-                unsigned int x = lsum;
-#pragma unroll
-                for (int o = 1; o < 32; o <<= 1) {
-                    const unsigned int y = __shfl_down_sync(0xffffffffu, x, o);
-                    if (tid + o < 32) x += y;
-                }
-                const unsigned int suffix = x - lsum;  // sum of lanes > tid
-                if (suffix < static_cast<unsigned int>(need) && suffix + lsum >= static_cast<unsigned int>(need)) {
-                    unsigned int run = suffix;
-                    for (int e = 7; e >= 0; --e) {
-                        if (run + c[e] >= static_cast<unsigned int>(need)) {
-                            sel_bucket = tid * 8 + e;
-                            sel_above = static_cast<int>(run);
-                            break;
-                        }
-                        run += c[e];
-                    }
-                }
-            }
-            __syncthreads();
-            const int bsel = sel_bucket;
-            need -= sel_above;
-            prefix |= static_cast<unsigned long long>(bsel) << shift;
-            mask |= 0xFFull << shift;
-            const bool done = static_cast<int>(hist[bsel]) == need;
-            __syncthreads();
-            if (done) break;
-        }
-        // ---- write kept indices ascending: keys above the prefix, plus the
-        // first `need` (lowest j) keys equal to it
-        int run_eq = 0, run_sel = 0;
-        for (int j0 = 0; j0 < T; j0 += THREADS) {
-            const int j = j0 + tid;
-            bool gt = false, eq = false;
-            if (j < T) {
-                const unsigned long long km = order_key(row[j]) & mask;
-                gt = km > prefix;
-                eq = km == prefix;
-            }
-            int tot_eq;
-            const int eq_rank = run_eq + block_excl_scan(eq ? 1 : 0, scan_scratch, &tot_eq);
-            const bool sel = gt || (eq && eq_rank < need);
-            int tot_sel;
-            const int pos = run_sel + block_excl_scan(sel ? 1 : 0, scan_scratch, &tot_sel);
-            if (sel) out[pos] = j;
-            run_eq += tot_eq;
-            run_sel += tot_sel;
-        }
+    const int hl = blockIdx.x / T, i = blockIdx.x % T;
+    const double* grow = scores + (static_cast<long long>(hl) * T + i) * T;
+    const double* row = grow;
+    if (in_smem) {
+        double* srow = reinterpret_cast<double*>(smem_raw);
+        for (int j = tid; j < T; j += STHREADS) srow[j] = grow[j];
+        row = srow;
         __syncthreads();
     }
+    int32_t* out = idx + (static_cast<long long>(h0 + hl) * T + i) * static_cast<long long>(k);
+
+    // ---- radix select of the k-th largest key, 8 bits per pass from the top
+    unsigned long long prefix = 0, mask = 0;
+    int need = k;
+    for (int shift = 56; shift >= 0; shift -= 8) {
+        for (int b = tid; b < 256; b += STHREADS) hist[b] = 0u;
+        __syncthreads();
+        for (int j0 = 0; j0 < T; j0 += STHREADS) {  // uniform trip count (warp collectives)
+            const int j = j0 + tid;
+            const unsigned long long key = j < T ? order_key(row[j]) : 0ull;
+            const bool m = j < T && (key & mask) == prefix;
+            const unsigned int digit = static_cast<unsigned int>((key >> shift) & 0xFFu);
+            const unsigned int active = __ballot_sync(0xffffffffu, m);
+            if (m) {
+                const unsigned int peers = __match_any_sync(active, digit);
+                if ((__ffs(peers) - 1) == (tid & 31)) atomicAdd(&hist[digit], __popc(peers));
+            }
+        }
+        __syncthreads();
+        if (tid < 32) {
+            unsigned int c[8], lsum = 0;
+#pragma unroll
+            for (int e = 0; e < 8; ++e) lsum += (c[e] = hist[tid * 8 + e]);
+            unsigned int x = lsum;  // inclusive suffix sum over lanes
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const unsigned int y = __shfl_down_sync(0xffffffffu, x, o);
+                if (tid + o < 32) x += y;
+            }
+            const unsigned int suffix = x - lsum;
+            if (suffix < static_cast<unsigned int>(need) && x >= static_cast<unsigned int>(need)) {
+                unsigned int run = suffix;
+                for (int e = 7; e >= 0; --e) {
+                    if (run + c[e] >= static_cast<unsigned int>(need)) {
+                        sel_bucket = tid * 8 + e;
+                        sel_above = static_cast<int>(run);
+                        break;
+                    }
+                    run += c[e];
+                }
+            }
+        }
+        __syncthreads();
+        const int bsel = sel_bucket;
+        need -= sel_above;
+        prefix |= static_cast<unsigned long long>(bsel) << shift;
+        mask |= 0xFFull << shift;
+        const bool done = static_cast<int>(hist[bsel]) == need;
+        __syncthreads();
+        if (done) break;
+    }
+
+    // ---- ascending output: each thread owns a contiguous range of j
+    const int per = (T + STHREADS - 1) / STHREADS;
+    const int jb = tid * per, je = min(T, jb + per);
+    int n_eq = 0;
+    for (int j = jb; j < je; ++j) n_eq += ((order_key(row[j]) & mask) == prefix) ? 1 : 0;
+    int tot;
+    const int eq_rank = block_excl_scan(n_eq, scan_scratch, &tot);
+    int n_sel = 0;
+    {
+        int r = eq_rank;
+        for (int j = jb; j < je; ++j) {
+            const unsigned long long km = order_key(row[j]) & mask;
+            if (km > prefix) ++n_sel;
+            else if (km == prefix) n_sel += (r++ < need) ? 1 : 0;
+        }
+    }
+    int pos = block_excl_scan(n_sel, scan_scratch, &tot);
+    {
+        int r = eq_rank;
+        for (int j = jb; j < je; ++j) {
+            const unsigned long long km = order_key(row[j]) & mask;
+            bool sel = km > prefix;
+            if (km == prefix) sel = (r++ < need);
+            if (sel) out[pos++] = j;
+        }
+    }
 }
+
+__global__ void iota_kernel(int32_t* __restrict__ idx, long long rows, int T) {
+    const long long total = rows * T;
+    for (long long e = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; e < total;
+         e += static_cast<long long>(gridDim.x) * blockDim.x)
+        idx[e] = static_cast<int32_t>(e % T);
+}
+
+inline size_t head_bytes(long long T) { return static_cast<size_t>(T) * static_cast<size_t>(T) * sizeof(double); }
 
 }  // namespace topk
 }  // namespace zb
 
 using namespace zb;
 
+extern "C" size_t zb_tile_score_topk_workspace_bytes(zb_shape s) {
+    if (check_shape(s) != ZB_OK) return 0;
+    const long long T = n_tiles(s);
+    const int heads = s.heads < 4 ? s.heads : 4;  // up to 4 heads per pass by default
+    return topk::head_bytes(T) * heads;
+}
+
 extern "C" zb_status zb_tile_score_topk(const double* Qbar, const double* Kbar, zb_shape s,
-                                        int32_t k, int32_t* idx, void* stream) {
+                                        int32_t k, int32_t* idx, void* ws, size_t ws_bytes,
+                                        void* stream) {
     zb_status e = check_shape(s);
     if (e != ZB_OK) return e;
     if (!Qbar || !Kbar || (!idx && k > 0)) return ZB_ERR_NULL;
     const long long T = n_tiles(s);
-    if (T > 32768) return ZB_ERR_UNSUPPORTED;
+    if (T > topk::MAX_T) return ZB_ERR_UNSUPPORTED;
     if (k < 0 || k > T) return ZB_ERR_SHAPE;
-    if (!aligned16(Qbar) || !aligned16(Kbar) || !aligned16(idx)) return ZB_ERR_ALIGN;
+    if (!aligned16(Qbar) || !aligned16(Kbar) || !aligned16(idx) || !aligned16(ws)) return ZB_ERR_ALIGN;
     if (k == 0) return ZB_OK;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (k == T) {  // keep-all: every row is 0..T-1, no scoring needed
+        DeviceInfo dev;
+        if ((e = current_device(&dev)) != ZB_OK) return e;
+        topk::iota_kernel<<<4 * dev.sm_count, 256, 0, st>>>(idx, static_cast<long long>(s.heads) * T,
+                                                            static_cast<int>(T));
+        return cudaGetLastError() == cudaSuccess ? ZB_OK : ZB_ERR_CUDA;
+    }
+    if (!ws || ws_bytes < topk::head_bytes(T)) return ZB_ERR_WORKSPACE;
     DeviceInfo dev;
     if ((e = current_device(&dev)) != ZB_OK) return e;
-    long long R = static_cast<long long>(topk::SCORE_SMEM_BUDGET / (static_cast<size_t>(T) * 8 + 64 * 8));
-    if (R > topk::MAX_ROWS) R = topk::MAX_ROWS;
-    if (R > T) R = T;
-    if (R < 1) return ZB_ERR_UNSUPPORTED;
-    const size_t smem = static_cast<size_t>(R) * (static_cast<size_t>(T) + 64) * 8;
-    if (cudaFuncSetAttribute(topk::score_topk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             static_cast<int>(smem)) != cudaSuccess)
+    const size_t fit = ws_bytes / topk::head_bytes(T);
+    const int per_pass = static_cast<int>(fit < static_cast<size_t>(s.heads) ? fit : static_cast<size_t>(s.heads));
+    const size_t gsmem = 2 * topk::HD * topk::GS * sizeof(double);
+    const size_t row_bytes = static_cast<size_t>(T) * sizeof(double);
+    const int in_smem = row_bytes <= topk::SMEM_SCORE_LIMIT ? 1 : 0;
+    const size_t ssmem = in_smem ? row_bytes : 0;
+    if (cudaFuncSetAttribute(topk::score_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(gsmem)) != cudaSuccess ||
+        cudaFuncSetAttribute(topk::select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(ssmem > 0 ? ssmem : 16)) != cudaSuccess)
         return ZB_ERR_CUDA;
-    const long long grid = static_cast<long long>(s.heads) * ((T + R - 1) / R);
-    if (grid > 0x7FFFFFFFll) return ZB_ERR_UNSUPPORTED;
-    topk::score_topk_kernel<<<static_cast<unsigned>(grid), topk::THREADS, smem, static_cast<cudaStream_t>(stream)>>>(
-        Qbar, Kbar, s.heads, static_cast<int>(T), k, static_cast<int>(R), idx);
-    return cudaGetLastError() == cudaSuccess ? ZB_OK : ZB_ERR_CUDA;
+    double* scores = static_cast<double*>(ws);
+    const int blocks = static_cast<int>((T + topk::GT - 1) / topk::GT);
+    for (int h0 = 0; h0 < s.heads; h0 += per_pass) {
+        const int hn = (s.heads - h0) < per_pass ? (s.heads - h0) : per_pass;
+        topk::score_gemm_kernel<<<dim3(blocks, blocks, hn), topk::GTHREADS, gsmem, st>>>(
+            Qbar, Kbar, static_cast<int>(T), h0, scores);
+        if (cudaGetLastError() != cudaSuccess) return ZB_ERR_CUDA;
+        const long long rows = static_cast<long long>(hn) * T;
+        if (rows > 0x7FFFFFFFll) return ZB_ERR_UNSUPPORTED;
+        topk::select_kernel<<<static_cast<unsigned>(rows), topk::STHREADS, ssmem, st>>>(
+            scores, static_cast<int>(T), k, h0, in_smem, idx);
+        if (cudaGetLastError() != cudaSuccess) return ZB_ERR_CUDA;
+    }
+    return ZB_OK;
 }

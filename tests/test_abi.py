@@ -52,6 +52,8 @@ def test_workspace_sizes(lib):
     assert lib.zb_linear_state_workspace_bytes(16, 1000, 32) == 0
     assert lib.zb_affine_fit_workspace_bytes(16, 4096, 64) == 16 * (128 + 16 * 2 * 4096) * 8
     assert lib.zb_affine_fit_workspace_bytes(0, 4096, 64) == 0
+    assert lib.zb_tile_score_topk_workspace_bytes(_shape(H=16, N=1024 * 1374, t=128)) == 4 * 10992 ** 2 * 8
+    assert lib.zb_tile_score_topk_workspace_bytes(_shape(H=2, N=256, t=64)) == 2 * 16 * 8
 
 
 def _shape(H=2, N=256, d=64, t=64):
@@ -72,10 +74,12 @@ def test_validation_errors_before_launch(lib):
     assert lib.zb_landmark_build(FAKE, FAKE, FAKE, S, None, FAKE, FAKE, FAKE, None) == 1
     assert lib.zb_landmark_build(FAKE + 8, FAKE, FAKE, S, FAKE, FAKE, FAKE, FAKE, None) == 3
     # selection: k out of range, null output
-    assert lib.zb_tile_score_topk(FAKE, FAKE, S, 5, FAKE, None) == 2
-    assert lib.zb_tile_score_topk(FAKE, FAKE, S, -1, FAKE, None) == 2
-    assert lib.zb_tile_score_topk(FAKE, FAKE, S, 2, None, None) == 1
-    assert lib.zb_tile_score_topk(FAKE, FAKE, S, 0, None, None) == 0  # nothing to do
+    assert lib.zb_tile_score_topk(FAKE, FAKE, S, 5, FAKE, FAKE, 1 << 20, None) == 2
+    assert lib.zb_tile_score_topk(FAKE, FAKE, S, -1, FAKE, FAKE, 1 << 20, None) == 2
+    assert lib.zb_tile_score_topk(FAKE, FAKE, S, 2, None, FAKE, 1 << 20, None) == 1
+    assert lib.zb_tile_score_topk(FAKE, FAKE, S, 2, FAKE, None, 1 << 20, None) == 5    # no workspace
+    assert lib.zb_tile_score_topk(FAKE, FAKE, S, 2, FAKE, FAKE, 4 * 4 * 8 - 8, None) == 5
+    assert lib.zb_tile_score_topk(FAKE, FAKE, S, 0, None, None, 0, None) == 0  # nothing to do
     # sparse attention
     a = (FAKE, FAKE, FAKE, FAKE, FAKE, FAKE)
     assert lib.zb_tile_sparse_attn(*a, 5, 1, 0.125, S, FAKE, None, None) == 2          # k > T
