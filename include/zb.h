@@ -198,6 +198,34 @@ zb_status zb_affine_fit(const uint16_t* X, const uint16_t* Y, int32_t heads,
                         void* ws, size_t ws_bytes, void* stream);
 
 /*
+ * Linear-attention state without a workspace.  The paper has no counterpart:
+ * this is a service entry point of the library.  Same result as
+ * zb_linear_state, for callers that cannot allocate device memory at call
+ * time (a process whose device memory is reserved by another allocator, or a
+ * latency-critical loop where an allocation and its implicit synchronisation
+ * are not allowed).  The per-CTA partial states go to a fixed scratch array
+ * inside the library (zb_linear_state_static_scratch_bytes() = 8 MiB), held
+ * on every GPU that loads the library until the process exits.
+ *   in : K, V bf16 [H][N][d]
+ *   out: S fp32 [H][d][d], z fp32 [H][d]
+ *   - Allocates nothing and needs no workspace.
+ *   - The first call on a device looks up the scratch array's device address
+ *     (with that device current); make that first call before any stream
+ *     capture.
+ *   - Every call shares the one scratch array: calls that overlap on the GPU
+ *     (other streams, other threads) race and must be serialised by the
+ *     caller.  A call overwrites all the scratch it reads, so the contents
+ *     left by an earlier call do not matter.
+ * Errors: ZB_ERR_NULL, ZB_ERR_SHAPE, ZB_ERR_ALIGN, ZB_ERR_UNSUPPORTED (also
+ * when the partial states of the shape exceed the scratch: more than 504
+ * heads), ZB_ERR_CUDA.
+ */
+size_t zb_linear_state_static_scratch_bytes(void);
+zb_status zb_linear_state_static(const uint16_t* K, const uint16_t* V, int32_t heads,
+                                 int64_t n_tokens, int32_t head_dim, float* S, float* z,
+                                 void* stream);
+
+/*
  * Copy whole tiles of a [H][N][d] bf16 tensor into a compact buffer (the
  * calibration rows of the affine fit are whole query tiles).
  *   in : X bf16 [H][N][d];  tiles int32 [n_tiles] DEVICE array, each in [0, T)

@@ -24,6 +24,8 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 
+#include <mutex>
+
 #include "zb_common.cuh"
 #include "zb_host.h"
 
@@ -526,5 +528,78 @@ extern "C" zb_status zb_linear_apply(const uint16_t* Q, int32_t heads, int64_t n
     const long long grid = items < 2ll * dev.sm_count ? items : 2ll * dev.sm_count;
     lin::linear_apply_kernel<<<static_cast<unsigned>(grid), lin::AP_THREADS, smem, static_cast<cudaStream_t>(stream)>>>(
         mq, heads, n_q, S, z, A, b, O, dev.status, wait_timeout_ns());
+    return cudaGetLastError() == cudaSuccess ? ZB_OK : ZB_ERR_CUDA;
+}
+
+// ======================================= linear state without a workspace ====
+// zb_linear_state needs a caller-allocated workspace for the per-CTA partial
+// states.  Some callers cannot allocate device memory when they call the
+// layer: a serving process whose device memory is reserved up front by
+// another framework's allocator, or a latency-critical loop where cudaMalloc
+// (which may synchronise the device) is not allowed.  zb_linear_state_static
+// gives them the same result without any workspace: the partials live in the
+// file-scope array below, a fixed 8 MiB that every GPU which loads this
+// library holds until the process exits.
+namespace zb {
+namespace lin {
+
+constexpr size_t kStaticScratchBytes = size_t(8) << 20;
+static __device__ __align__(256) unsigned char g_state_scratch[kStaticScratchBytes];
+
+namespace {
+std::mutex g_static_mu;
+float* g_static_ptr[64] = {};  // device address of g_state_scratch, per device
+}  // namespace
+
+// Device address of the scratch array on the current device; looked up once per
+// device with that device current (the first call on a device does this).
+static zb_status static_scratch(int device, float** out) {
+    if (device < 0 || device >= 64) return ZB_ERR_DEVICE;
+    std::lock_guard<std::mutex> lock(g_static_mu);
+    if (!g_static_ptr[device]) {
+        void* p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_state_scratch) != cudaSuccess || p == nullptr) return ZB_ERR_CUDA;
+        g_static_ptr[device] = static_cast<float*>(p);
+    }
+    *out = g_static_ptr[device];
+    return ZB_OK;
+}
+
+}  // namespace lin
+}  // namespace zb
+
+extern "C" size_t zb_linear_state_static_scratch_bytes(void) { return zb::lin::kStaticScratchBytes; }
+
+extern "C" zb_status zb_linear_state_static(const uint16_t* K, const uint16_t* V, int32_t heads,
+                                            int64_t n_tokens, int32_t head_dim, float* S, float* z,
+                                            void* stream) {
+    using namespace zb;
+    if (heads < 1 || n_tokens < 1) return ZB_ERR_SHAPE;
+    if (head_dim != 64) return ZB_ERR_UNSUPPORTED;
+    if (n_tokens > (1ll << 31) - 256) return ZB_ERR_UNSUPPORTED;
+    if (!K || !V || !S || !z) return ZB_ERR_NULL;
+    if (!aligned16(K) || !aligned16(V) || !aligned16(S) || !aligned16(z)) return ZB_ERR_ALIGN;
+    // the partial states of this shape must fit the fixed scratch
+    if (lin::state_ws_bytes(heads, n_tokens) > lin::kStaticScratchBytes) return ZB_ERR_UNSUPPORTED;
+    DeviceInfo dev;
+    zb_status e = current_device(&dev);
+    if (e != ZB_OK) return e;
+    float* part = nullptr;
+    if ((e = lin::static_scratch(dev.device, &part)) != ZB_OK) return e;
+    CUtensorMap mk, mv;
+    if ((e = make_map_bf16_3d(&mk, K, 64, n_tokens, heads, lin::TILE)) != ZB_OK) return e;
+    if ((e = make_map_bf16_3d(&mv, V, 64, n_tokens, heads, lin::TILE)) != ZB_OK) return e;
+    const lin::StateGeom geo = lin::state_geom(heads, n_tokens);
+    const size_t smem = sizeof(lin::StateSmem) + 1024;
+    if (cudaFuncSetAttribute(lin::linear_state_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(smem)) != cudaSuccess)
+        return ZB_ERR_CUDA;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    // Every CTA writes its whole partial slot (zeros when it has no tokens), so
+    // nothing left in the scratch by an earlier call is read.
+    lin::linear_state_kernel<<<geo.pairs * geo.chunks, lin::ST_THREADS, smem, st>>>(
+        mk, mv, heads, n_tokens, geo, part, dev.status, wait_timeout_ns());
+    if (cudaGetLastError() != cudaSuccess) return ZB_ERR_CUDA;
+    lin::linear_state_reduce_kernel<<<heads, 256, 0, st>>>(part, heads, geo, S, z);
     return cudaGetLastError() == cudaSuccess ? ZB_OK : ZB_ERR_CUDA;
 }
