@@ -273,9 +273,9 @@ def main():
         zb.zb_linear_state(K, V, layer.S, layer.z, layer.ws_lin)
         mark(4)
         zb.zb_gather_tiles(Q, w.tile, layer.calib, out=layer.Qc)
-        zb.zb_dense_attn(layer.Qc, K, V, layer.scale, out=layer.Yc)
+        zb.zb_dense_attn(layer.Qc, K, V, layer.scale, out=layer.Yc, out_fp32=True)
         mark(5)
-        zb.zb_linear_apply(layer.Qc, layer.S, layer.z, None, None, out=layer.Xc)
+        zb.zb_linear_apply(layer.Qc, layer.S, layer.z, None, None, out=layer.Xc, out_fp32=True)
         zb.zb_affine_fit(layer.Xc, layer.Yc, layer.A, layer.b, layer.ws_fit)
         mark(6)
         zb.zb_linear_apply(Q, layer.S, layer.z, layer.A, layer.b, out=layer.O_linear)

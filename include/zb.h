@@ -137,13 +137,14 @@ zb_status zb_tile_sparse_attn(const uint16_t* Q, const uint16_t* K, const uint16
  * zb_tile_sparse_attn with every key tile kept and no landmarks; queries and
  * keys may have different lengths.
  *   in : Q bf16 [H][n_q][d];  K, V bf16 [H][n_kv][d]
- *   out: O bf16 [H][n_q][d];  lse fp32 [H][n_q] (may be NULL)
+ *   out: O [H][n_q][d], bf16 (out_fp32 == 0) or fp32 (out_fp32 != 0);
+ *        lse fp32 [H][n_q] (may be NULL)
  * Errors: ZB_ERR_NULL, ZB_ERR_SHAPE, ZB_ERR_ALIGN, ZB_ERR_UNSUPPORTED, ZB_ERR_CUDA.
  */
 zb_status zb_dense_attn(const uint16_t* Q, int64_t n_q, const uint16_t* K,
                         const uint16_t* V, int64_t n_kv, int32_t heads,
-                        int32_t head_dim, float scale, uint16_t* O, float* lse,
-                        void* stream);
+                        int32_t head_dim, float scale, void* O, int32_t out_fp32,
+                        float* lse, void* stream);
 
 /*
  * Linear-attention state (Abstract: linear attention for tolerant stages):
@@ -166,24 +167,32 @@ zb_status zb_linear_state(const uint16_t* K, const uint16_t* V, int32_t heads,
  * Linear-attention output with the per-head affine map (section "How Zebra3D
  * works": the linear parts are corrected by a closed-form affine map):
  *   O_r = (phi(q_r) S / (phi(q_r) . z)) A + b      (row vectors)
- * computed as phi(q_r) (S A) / (phi(q_r) . z) + b: S A and z are rounded to
- * bf16 for the tensor-core product, the division and + b are fp32.
+ * computed around the centre c = 1^T S / 1^T z (the output for phi(q) = 1):
+ *   O_r = phi(q_r) ((S - z c^T) A) / (phi(q_r) . z) + (c A + b),
+ * an exact identity that keeps rounded intermediates small.
+ *   out_fp32 == 0: bf16 O; (S - z c^T) A and z are rounded to bf16 for the
+ *                  tensor-core product, the division and the bias are fp32.
+ *   out_fp32 != 0: fp32 O computed on the CUDA cores in fp32 (meant for
+ *                  calibration-sized row sets such as the affine fit's X).
  *   in : Q bf16 [H][n_q][d];  S fp32 [H][d][d];  z fp32 [H][d];
  *        A fp32 [H][d][d] or NULL (identity);  b fp32 [H][d] or NULL (zero)
- *   out: O bf16 [H][n_q][d]
+ *   out: O [H][n_q][d] (bf16 or fp32, see above)
  * Errors: ZB_ERR_NULL, ZB_ERR_SHAPE, ZB_ERR_ALIGN, ZB_ERR_UNSUPPORTED, ZB_ERR_CUDA.
  */
 zb_status zb_linear_apply(const uint16_t* Q, int32_t heads, int64_t n_q,
                           int32_t head_dim, const float* S, const float* z,
-                          const float* A, const float* b, uint16_t* O, void* stream);
+                          const float* A, const float* b, void* O, int32_t out_fp32,
+                          void* stream);
 
 /*
  * Closed-form affine fit (Abstract: closed-form affine fitting makes the
  * conversion training-free; Table 3 (a) of "Zebra3D: Efficient Hybrid
  * Foundation Models ..." compares no fit with fitted variants): per head, the
- * least-squares solution of [X 1] [A; b] = Y over R calibration rows.  Solved
- * in fp64: row means, centred Gram matrices, Cholesky factorisation.
- *   in : X bf16 [H][R][d] (unfitted linear output), Y bf16 [H][R][d] (dense
+ * least-squares solution of [X 1] [A; b] = Y over R calibration rows, with a
+ * vanishing ridge lam = 1e-8 * max_i ((X - mean X)^T (X - mean X))_ii on A so
+ * that calibration outputs varying in fewer than d directions stay solvable.
+ * Solved in fp64: row means, centred Gram matrices, Cholesky factorisation.
+ *   in : X fp32 [H][R][d] (unfitted linear output), Y fp32 [H][R][d] (dense
  *        output on the same rows);  R >= d + 1;  ws of >=
  *        zb_affine_fit_workspace_bytes() bytes
  *   out: A fp32 [H][d][d], b fp32 [H][d]
@@ -193,7 +202,7 @@ zb_status zb_linear_apply(const uint16_t* Q, int32_t heads, int64_t n_q,
  * ZB_ERR_WORKSPACE, ZB_ERR_CUDA.
  */
 size_t zb_affine_fit_workspace_bytes(int32_t heads, int64_t rows, int32_t head_dim);
-zb_status zb_affine_fit(const uint16_t* X, const uint16_t* Y, int32_t heads,
+zb_status zb_affine_fit(const float* X, const float* Y, int32_t heads,
                         int64_t rows, int32_t head_dim, float* A, float* b,
                         void* ws, size_t ws_bytes, void* stream);
 

@@ -172,19 +172,19 @@ def zb_tile_sparse_attn(Q, K, V, Kbar_bf16, Vbar_bf16, idx, k: int, tile: int,
 
 
 def zb_dense_attn(Q, K, V, scale: Optional[float] = None, out: Optional[torch.Tensor] = None,
-                  lse: Optional[torch.Tensor] = None, want_lse: bool = False):
-    """Dense softmax attention softmax(scale Q K^T) V on the tensor cores."""
+                  lse: Optional[torch.Tensor] = None, want_lse: bool = False, out_fp32: bool = False):
+    """Dense softmax attention softmax(scale Q K^T) V on the tensor cores (bf16 or fp32 O)."""
     for t, n in ((Q, "Q"), (K, "K"), (V, "V")):
         _need(t, torch.bfloat16, n, 3)
     H, Nq, d = Q.shape
     Nk = K.shape[1]
     if scale is None:
         scale = 1.0 / math.sqrt(d)
-    O = _out((H, Nq, d), torch.bfloat16, Q.device, out, "O")
+    O = _out((H, Nq, d), torch.float32 if out_fp32 else torch.bfloat16, Q.device, out, "O")
     if want_lse or lse is not None:
         lse = _out((H, Nq), torch.float32, Q.device, lse, "lse")
     st = _lib_handle().zb_dense_attn(_ptr(Q), Nq, _ptr(K), _ptr(V), Nk, H, d, float(scale), _ptr(O),
-                                     _ptr(lse), _stream())
+                                     1 if out_fp32 else 0, _ptr(lse), _stream())
     _check(st, "zb_dense_attn")
     return (O, lse) if lse is not None else O
 
@@ -220,8 +220,8 @@ def zb_linear_state(K, V, S: Optional[torch.Tensor] = None, z: Optional[torch.Te
 
 
 def zb_linear_apply(Q, S, z, A: Optional[torch.Tensor] = None, b: Optional[torch.Tensor] = None,
-                    out: Optional[torch.Tensor] = None) -> torch.Tensor:
-    """O = (phi(Q) S / (phi(Q) . z)) A + b (bf16)."""
+                    out: Optional[torch.Tensor] = None, out_fp32: bool = False) -> torch.Tensor:
+    """O = (phi(Q) S / (phi(Q) . z)) A + b: bf16 on the tensor cores, or fp32 on the CUDA cores."""
     _need(Q, torch.bfloat16, "Q", 3)
     _need(S, torch.float32, "S", 3)
     _need(z, torch.float32, "z", 2)
@@ -230,18 +230,18 @@ def zb_linear_apply(Q, S, z, A: Optional[torch.Tensor] = None, b: Optional[torch
     if b is not None:
         _need(b, torch.float32, "b", 2)
     H, N, d = Q.shape
-    O = _out((H, N, d), torch.bfloat16, Q.device, out, "O")
+    O = _out((H, N, d), torch.float32 if out_fp32 else torch.bfloat16, Q.device, out, "O")
     st = _lib_handle().zb_linear_apply(_ptr(Q), H, N, d, _ptr(S), _ptr(z), _ptr(A), _ptr(b), _ptr(O),
-                                       _stream())
+                                       1 if out_fp32 else 0, _stream())
     _check(st, "zb_linear_apply")
     return O
 
 
 def zb_affine_fit(X, Y, A: Optional[torch.Tensor] = None, b: Optional[torch.Tensor] = None,
                   ws: Optional[torch.Tensor] = None):
-    """Least-squares [A; b] of [X 1] [A; b] = Y per head (X, Y bf16 [H, R, d])."""
-    _need(X, torch.bfloat16, "X", 3)
-    _need(Y, torch.bfloat16, "Y", 3)
+    """Least-squares [A; b] of [X 1] [A; b] = Y per head (vanishing ridge), X, Y fp32 [H, R, d]."""
+    _need(X, torch.float32, "X", 3)
+    _need(Y, torch.float32, "Y", 3)
     H, R, d = X.shape
     A = _out((H, d, d), torch.float32, X.device, A, "A")
     b = _out((H, d), torch.float32, X.device, b, "b")
@@ -304,8 +304,8 @@ class HybridLayer:
         R = len(calib_tiles) * tile
         self.R = R
         self.Qc = torch.empty(H, R, d, dtype=torch.bfloat16, device=dev)
-        self.Xc = torch.empty(H, R, d, dtype=torch.bfloat16, device=dev)
-        self.Yc = torch.empty(H, R, d, dtype=torch.bfloat16, device=dev)
+        self.Xc = torch.empty(H, R, d, dtype=torch.float32, device=dev)
+        self.Yc = torch.empty(H, R, d, dtype=torch.float32, device=dev)
         self.A = torch.empty(H, d, d, dtype=torch.float32, device=dev)
         self.b = torch.empty(H, d, dtype=torch.float32, device=dev)
         self.ws_fit = torch.empty(max(affine_fit_workspace_bytes(H, max(R, d + 1), d), 16), dtype=torch.uint8,
@@ -331,8 +331,8 @@ class HybridLayer:
     def calibrate(self, Q, K, V):
         zb_linear_state(K, V, self.S, self.z, self.ws_lin)
         zb_gather_tiles(Q, self.tile, self.calib, out=self.Qc)
-        zb_dense_attn(self.Qc, K, V, self.scale, out=self.Yc)
-        zb_linear_apply(self.Qc, self.S, self.z, None, None, out=self.Xc)
+        zb_dense_attn(self.Qc, K, V, self.scale, out=self.Yc, out_fp32=True)
+        zb_linear_apply(self.Qc, self.S, self.z, None, None, out=self.Xc, out_fp32=True)
         zb_affine_fit(self.Xc, self.Yc, self.A, self.b, self.ws_fit)
         return self.A, self.b
 

@@ -29,12 +29,12 @@ PROTOTYPES = {
     "zb_tile_score_topk": (c_i32, [c_vp, c_vp, ZbShape, c_i32, c_vp, c_vp, c_sz, c_vp]),
     "zb_tile_sparse_attn": (c_i32, [c_vp, c_vp, c_vp, c_vp, c_vp, c_vp, c_i32, c_i32, c_f32, ZbShape,
                                     c_vp, c_vp, c_vp]),
-    "zb_dense_attn": (c_i32, [c_vp, c_i64, c_vp, c_vp, c_i64, c_i32, c_i32, c_f32, c_vp, c_vp, c_vp]),
+    "zb_dense_attn": (c_i32, [c_vp, c_i64, c_vp, c_vp, c_i64, c_i32, c_i32, c_f32, c_vp, c_i32, c_vp, c_vp]),
     "zb_linear_state_workspace_bytes": (c_sz, [c_i32, c_i64, c_i32]),
     "zb_linear_state": (c_i32, [c_vp, c_vp, c_i32, c_i64, c_i32, c_vp, c_vp, c_vp, c_sz, c_vp]),
     "zb_linear_state_static_scratch_bytes": (c_sz, []),
     "zb_linear_state_static": (c_i32, [c_vp, c_vp, c_i32, c_i64, c_i32, c_vp, c_vp, c_vp]),
-    "zb_linear_apply": (c_i32, [c_vp, c_i32, c_i64, c_i32, c_vp, c_vp, c_vp, c_vp, c_vp, c_vp]),
+    "zb_linear_apply": (c_i32, [c_vp, c_i32, c_i64, c_i32, c_vp, c_vp, c_vp, c_vp, c_vp, c_i32, c_vp]),
     "zb_affine_fit_workspace_bytes": (c_sz, [c_i32, c_i64, c_i32]),
     "zb_affine_fit": (c_i32, [c_vp, c_vp, c_i32, c_i64, c_i32, c_vp, c_vp, c_vp, c_sz, c_vp]),
     "zb_gather_tiles": (c_i32, [c_vp, ZbShape, c_vp, c_i32, c_vp, c_vp]),

@@ -8,10 +8,11 @@
 // descent.  Reading used: per head, least squares of [X 1] [A; b] = Y over the
 // calibration rows (row vectors, y = x A + b).
 //
-// Solved in fp64 through centred normal equations, which give the same
-// minimiser as the uncentred system but a better-conditioned matrix:
+// Solved in fp64 through centred normal equations (the intercept absorbs the
+// means) with a vanishing ridge on A that keeps degenerate calibration sets
+// solvable:
 //   xm, ym = column means;  G = (X - xm)^T (X - xm);  C = (X - xm)^T (Y - ym);
-//   G A = C (Cholesky),  b = ym - xm A.
+//   lam = 1e-8 * max_i G_ii;  (G + lam I) A = C (Cholesky);  b = ym - xm A.
 // Three kernels: column means per head; Gram partials per (head, 256-row
 // chunk); fixed-order reduction + Cholesky + two triangular solves per head.
 #include <cuda_runtime.h>
@@ -25,6 +26,7 @@ namespace aff {
 constexpr int HD = 64;
 constexpr int CHUNK = 256;
 constexpr int BATCH = 32;  // rows staged in shared memory at a time
+constexpr double RIDGE_REL = 1e-8;
 
 inline long long n_chunks(long long rows) { return (rows + CHUNK - 1) / CHUNK; }
 
@@ -32,22 +34,19 @@ inline size_t ws_bytes(int heads, long long rows) {
     return static_cast<size_t>(heads) * (2 * HD + n_chunks(rows) * 2 * HD * HD) * sizeof(double);
 }
 
-__device__ __forceinline__ double bf(uint16_t v) {
-    return static_cast<double>(__uint_as_float(static_cast<uint32_t>(v) << 16));
-}
 
 // ws layout per head: [means: 2 x 64][partials: chunks x 2 x 64 x 64]
-__global__ void __launch_bounds__(256) affine_means_kernel(const uint16_t* __restrict__ X, const uint16_t* __restrict__ Y,
+__global__ void __launch_bounds__(256) affine_means_kernel(const float* __restrict__ X, const float* __restrict__ Y,
                                     long long rows, double* __restrict__ ws, long long nch) {
     const int h = blockIdx.x;
     const int c = threadIdx.x & 63, r0 = threadIdx.x >> 6;
     __shared__ double red[2][4][HD];
     double sx = 0.0, sy = 0.0;
-    const uint16_t* xh = X + static_cast<long long>(h) * rows * HD;
-    const uint16_t* yh = Y + static_cast<long long>(h) * rows * HD;
+    const float* xh = X + static_cast<long long>(h) * rows * HD;
+    const float* yh = Y + static_cast<long long>(h) * rows * HD;
     for (long long r = r0; r < rows; r += 4) {
-        sx += bf(xh[r * HD + c]);
-        sy += bf(yh[r * HD + c]);
+        sx += static_cast<double>(xh[r * HD + c]);
+        sy += static_cast<double>(yh[r * HD + c]);
     }
     red[0][r0][c] = sx;
     red[1][r0][c] = sy;
@@ -59,7 +58,7 @@ __global__ void __launch_bounds__(256) affine_means_kernel(const uint16_t* __res
     }
 }
 
-__global__ void __launch_bounds__(256) affine_gram_kernel(const uint16_t* __restrict__ X, const uint16_t* __restrict__ Y,
+__global__ void __launch_bounds__(256) affine_gram_kernel(const float* __restrict__ X, const float* __restrict__ Y,
                                    long long rows, double* __restrict__ ws, long long nch) {
     const int h = blockIdx.y;
     const long long ch = blockIdx.x;
@@ -75,8 +74,8 @@ __global__ void __launch_bounds__(256) affine_gram_kernel(const uint16_t* __rest
     double g[16], cc[16];
 #pragma unroll
     for (int e = 0; e < 16; ++e) g[e] = cc[e] = 0.0;
-    const uint16_t* xh = X + static_cast<long long>(h) * rows * HD;
-    const uint16_t* yh = Y + static_cast<long long>(h) * rows * HD;
+    const float* xh = X + static_cast<long long>(h) * rows * HD;
+    const float* yh = Y + static_cast<long long>(h) * rows * HD;
     const long long rbeg = ch * CHUNK;
     const long long rend = min(rows, rbeg + CHUNK);
     __syncthreads();
@@ -85,8 +84,8 @@ __global__ void __launch_bounds__(256) affine_gram_kernel(const uint16_t* __rest
             const int rr = e / HD, col = e % HD;
             const long long r = r0 + rr;
             const bool in = r < rend;
-            xs[rr][col] = in ? bf(xh[r * HD + col]) - mx[col] : 0.0;
-            ys[rr][col] = in ? bf(yh[r * HD + col]) - my[col] : 0.0;
+            xs[rr][col] = in ? static_cast<double>(xh[r * HD + col]) - mx[col] : 0.0;
+            ys[rr][col] = in ? static_cast<double>(yh[r * HD + col]) - my[col] : 0.0;
         }
         __syncthreads();
 #pragma unroll 4
@@ -130,6 +129,14 @@ __global__ void __launch_bounds__(HD) affine_solve_kernel(const double* __restri
     }
     if (t == 0) singular = 0;
     __syncthreads();
+    // vanishing ridge: lam = RIDGE_REL * max_i G_ii (every thread computes it)
+    {
+        double gmax = 0.0;
+        for (int i = 0; i < HD; ++i) gmax = fmax(gmax, G[i][i]);
+        __syncthreads();
+        G[t][t] += RIDGE_REL * gmax;
+        __syncthreads();
+    }
     // Cholesky G = L L^T in place (lower triangle), right-looking
     for (int j = 0; j < HD; ++j) {
         if (t == 0) {
@@ -179,7 +186,7 @@ extern "C" size_t zb_affine_fit_workspace_bytes(int32_t heads, int64_t rows, int
     return aff::ws_bytes(heads, rows);
 }
 
-extern "C" zb_status zb_affine_fit(const uint16_t* X, const uint16_t* Y, int32_t heads, int64_t rows,
+extern "C" zb_status zb_affine_fit(const float* X, const float* Y, int32_t heads, int64_t rows,
                                    int32_t head_dim, float* A, float* b, void* ws, size_t ws_bytes,
                                    void* stream) {
     if (heads < 1) return ZB_ERR_SHAPE;

@@ -279,6 +279,7 @@ struct ApplySmem {
     uint8_t q[AP_STAGES][TILE_BYTES];
     uint8_t bop[2][B_BYTES];
     float bvec[2][HD];
+    float cvec[HD];
     uint64_t full[AP_STAGES], mma_done[2], drain;
     uint32_t tmem_base;
     int abort_flag;
@@ -370,11 +371,30 @@ linear_apply_kernel(const __grid_constant__ CUtensorMap tm_q, int heads, long lo
         const long long item = first + it;
         const int h = static_cast<int>(item / Tn);
         if (h != h_prev) {
-            // B operand of head h into buffer (h & 1): rows n < 64 hold (S A)[:, n],
-            // row 64 holds z, rows 65..79 zero; K-major, 128-byte swizzle.
+            // B operand of head h into buffer (h & 1), K-major, 128-byte swizzle:
+            // rows n < 64 hold ((S - z c^T) A)[:, n], row 64 holds z, rows
+            // 65..79 zero; the bias becomes b' = c A + b.  Centring on
+            // c = 1^T S / 1^T z (the output for phi(q) = 1) is an exact identity
+            // (phi(q) z c^T / (phi(q) . z) = c^T) that keeps the bf16 operand
+            // small, so rounding it does not cancel against b'.
             uint8_t* bo = sm.bop[h & 1];
             const float* Sh = S + static_cast<size_t>(h) * HD * HD;
+            const float* zh = z + static_cast<size_t>(h) * HD;
             const float* Ah = A ? A + static_cast<size_t>(h) * HD * HD : nullptr;
+            if (tid < HD) {
+                float cs = 0.f, zs = 0.f;
+                for (int k = 0; k < HD; ++k) {
+                    cs += __ldg(Sh + k * HD + tid);
+                    zs += __ldg(zh + k);
+                }
+                sm.cvec[tid] = cs / zs;
+            }
+            __syncthreads();
+            if (tid < HD) {
+                float ca = 0.f;
+                for (int m = 0; m < HD; ++m) ca = fmaf(sm.cvec[m], Ah ? __ldg(Ah + m * HD + tid) : (m == tid ? 1.f : 0.f), ca);
+                sm.bvec[h & 1][tid] = ca + (bias ? bias[static_cast<size_t>(h) * HD + tid] : 0.f);
+            }
             {
                 const int ncol = tid & 63;       // output column n
                 const int khalf = tid >> 6;      // rows k in [32 khalf, 32 khalf + 32)
@@ -387,9 +407,10 @@ linear_apply_kernel(const __grid_constant__ CUtensorMap tm_q, int heads, long lo
                     for (int u = 0; u < 2; ++u) {
                         const int k = khalf * 32 + kq + u;
                         const float* srow = Sh + k * HD;
+                        const float zk = __ldg(zh + k);
                         float acc = 0.f;
 #pragma unroll
-                        for (int m = 0; m < HD; ++m) acc = fmaf(__ldg(srow + m), acol[m], acc);
+                        for (int m = 0; m < HD; ++m) acc = fmaf(fmaf(-zk, sm.cvec[m], __ldg(srow + m)), acol[m], acc);
                         v2[u] = acc;
                     }
                     const int k = khalf * 32 + kq;  // even: both land in one 32-bit word
@@ -406,7 +427,6 @@ linear_apply_kernel(const __grid_constant__ CUtensorMap tm_q, int heads, long lo
                 const int off = rr * 128 + ((((k >> 3) ^ (rr & 7))) << 4) + (k & 7) * 2;
                 *reinterpret_cast<uint32_t*>(bo + off) = pack_bf16x2(a, b);
             }
-            if (tid < HD) sm.bvec[h & 1][tid] = bias ? bias[static_cast<size_t>(h) * HD + tid] : 0.f;
             h_prev = h;
         }
         const int s = it % AP_STAGES;
@@ -466,6 +486,83 @@ linear_apply_kernel(const __grid_constant__ CUtensorMap tm_q, int heads, long lo
     }
 }
 
+// fp32 output on the CUDA cores, for calibration-sized row sets: one thread
+// per query row, (S - z c^T), z and A staged in shared memory in fp32,
+//   x_c = phi(q) (S - z c^T) / (phi(q) . z)   (= linear output - c)
+//   o   = x_c A + (c A + b)
+// with c = 1^T S / 1^T z, the same centring as the tensor-core path.
+__global__ void __launch_bounds__(128)
+linear_apply_f32_kernel(const uint16_t* __restrict__ Q, int heads, long long n_q, const float* __restrict__ S,
+                        const float* __restrict__ z, const float* __restrict__ A,
+                        const float* __restrict__ bias, float* __restrict__ O) {
+    __shared__ float sc[HD][HD];      // S - z c^T
+    __shared__ float am[HD][HD + 1];  // A (identity when absent)
+    __shared__ float zz[HD], cc[HD], bb[HD];
+    const int h = blockIdx.y;
+    const int tid = threadIdx.x;
+    const float* Sh = S + static_cast<size_t>(h) * HD * HD;
+    const float* zh = z + static_cast<size_t>(h) * HD;
+    const float* Ah = A ? A + static_cast<size_t>(h) * HD * HD : nullptr;
+    if (tid < HD) {
+        float cs = 0.f, zs = 0.f;
+        for (int k = 0; k < HD; ++k) {
+            cs += Sh[k * HD + tid];
+            zs += zh[k];
+        }
+        cc[tid] = cs / zs;
+        zz[tid] = zh[tid];
+    }
+    for (int e = tid; e < HD * HD; e += blockDim.x) {
+        const int m = e / HD, n = e % HD;
+        am[m][n] = Ah ? Ah[e] : (m == n ? 1.f : 0.f);
+    }
+    __syncthreads();
+    for (int e = tid; e < HD * HD; e += blockDim.x) {
+        const int k = e / HD, n = e % HD;
+        sc[k][n] = fmaf(-zz[k], cc[n], Sh[e]);
+    }
+    if (tid < HD) {
+        float ca = 0.f;
+        for (int m = 0; m < HD; ++m) ca = fmaf(cc[m], am[m][tid], ca);
+        bb[tid] = ca + (bias ? bias[static_cast<size_t>(h) * HD + tid] : 0.f);
+    }
+    __syncthreads();
+    const long long row = static_cast<long long>(blockIdx.x) * blockDim.x + tid;
+    if (row >= n_q) return;
+    const uint16_t* qr = Q + (static_cast<long long>(h) * n_q + row) * HD;
+    float f[HD];
+    float den = 0.f;
+#pragma unroll
+    for (int c8 = 0; c8 < HD / 8; ++c8) {
+        const uint4 v = __ldg(reinterpret_cast<const uint4*>(qr) + c8);
+        const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            f[c8 * 8 + 2 * e] = phi(bf16_lo(w[e]));
+            f[c8 * 8 + 2 * e + 1] = phi(bf16_hi(w[e]));
+        }
+    }
+#pragma unroll
+    for (int k = 0; k < HD; ++k) den = fmaf(f[k], zz[k], den);
+    const float inv = 1.f / den;
+    float xc[HD];
+#pragma unroll 4
+    for (int n = 0; n < HD; ++n) {
+        float u = 0.f;
+#pragma unroll
+        for (int k = 0; k < HD; ++k) u = fmaf(f[k], sc[k][n], u);
+        xc[n] = u * inv;
+    }
+    float* orow = O + (static_cast<long long>(h) * n_q + row) * HD;
+#pragma unroll 4
+    for (int n = 0; n < HD; ++n) {
+        float o = bb[n];
+#pragma unroll
+        for (int m = 0; m < HD; ++m) o = fmaf(xc[m], am[m][n], o);
+        orow[n] = o;
+    }
+}
+
 }  // namespace lin
 }  // namespace zb
 
@@ -508,7 +605,8 @@ extern "C" zb_status zb_linear_state(const uint16_t* K, const uint16_t* V, int32
 
 extern "C" zb_status zb_linear_apply(const uint16_t* Q, int32_t heads, int64_t n_q,
                                      int32_t head_dim, const float* S, const float* z,
-                                     const float* A, const float* b, uint16_t* O, void* stream) {
+                                     const float* A, const float* b, void* O, int32_t out_fp32,
+                                     void* stream) {
     if (heads < 1 || n_q < 1) return ZB_ERR_SHAPE;
     if (head_dim != 64) return ZB_ERR_UNSUPPORTED;
     if (n_q > (1ll << 31) - 256) return ZB_ERR_UNSUPPORTED;
@@ -518,6 +616,14 @@ extern "C" zb_status zb_linear_apply(const uint16_t* Q, int32_t heads, int64_t n
     DeviceInfo dev;
     zb_status e = current_device(&dev);
     if (e != ZB_OK) return e;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (out_fp32) {
+        const long long blocks = (n_q + 127) / 128;
+        if (blocks > 0x7FFFFFFFll || heads > 65535) return ZB_ERR_UNSUPPORTED;
+        lin::linear_apply_f32_kernel<<<dim3(static_cast<unsigned>(blocks), heads), 128, 0, st>>>(
+            Q, heads, n_q, S, z, A, b, static_cast<float*>(O));
+        return cudaGetLastError() == cudaSuccess ? ZB_OK : ZB_ERR_CUDA;
+    }
     CUtensorMap mq;
     if ((e = make_map_bf16_3d(&mq, Q, 64, n_q, heads, lin::TILE)) != ZB_OK) return e;
     const size_t smem = sizeof(lin::ApplySmem) + 1024;
@@ -526,8 +632,8 @@ extern "C" zb_status zb_linear_apply(const uint16_t* Q, int32_t heads, int64_t n
         return ZB_ERR_CUDA;
     const long long items = static_cast<long long>(heads) * ((n_q + lin::TILE - 1) / lin::TILE);
     const long long grid = items < 2ll * dev.sm_count ? items : 2ll * dev.sm_count;
-    lin::linear_apply_kernel<<<static_cast<unsigned>(grid), lin::AP_THREADS, smem, static_cast<cudaStream_t>(stream)>>>(
-        mq, heads, n_q, S, z, A, b, O, dev.status, wait_timeout_ns());
+    lin::linear_apply_kernel<<<static_cast<unsigned>(grid), lin::AP_THREADS, smem, st>>>(
+        mq, heads, n_q, S, z, A, b, static_cast<uint16_t*>(O), dev.status, wait_timeout_ns());
     return cudaGetLastError() == cudaSuccess ? ZB_OK : ZB_ERR_CUDA;
 }
 

@@ -46,7 +46,7 @@ __all__ = [
     "tile_lengths", "landmark_means", "tile_scores", "select_tiles",
     "sparse_attention", "dense_attention", "elu_plus_one", "linear_state",
     "linear_apply", "linear_attention", "linear_attention_quadratic", "affine_fit",
-    "affine_apply", "calibration_rows",
+    "affine_apply", "calibration_rows", "RIDGE_REL",
 ]
 
 
@@ -252,23 +252,41 @@ def affine_apply(X, A=None, b=None) -> np.ndarray:
     return Y
 
 
-def affine_fit(X, Y):
-    """Closed-form least-squares affine map per head: [A; b] = argmin ||[X 1] W - Y||_F.
+RIDGE_REL = 1e-8
+
+
+def affine_fit(X, Y, ridge_rel: float = RIDGE_REL):
+    """Closed-form affine map per head: [A; b] minimising ||[X 1][A; b] - Y||_F^2 + lam ||A||_F^2.
 
     [ABS], [HOW]: the linear stage's output is corrected by an affine map fitted
     in closed form (no gradient descent) against the dense layer's output on
     calibration rows.  X, Y: [H, R, d] -> A [H, d, d], b [H, d].
-    Solved with an fp64 least-squares routine on the design matrix [X 1].
+
+    Reading: ordinary least squares with an intercept, plus a vanishing ridge
+    lam = ridge_rel * max_i ((X - mean X)^T (X - mean X))_ii on A (not on b).
+    The intercept absorbs the means, so this equals OLS on the centred data,
+    A = argmin ||Xc A - Yc||^2 + lam ||A||^2, b = mean(Y) - mean(X) A.  Without
+    the ridge the problem is singular whenever the calibration outputs vary in
+    fewer than d directions (which the linear stage's outputs often nearly
+    do); the ridge only damps directions carrying under sqrt(ridge_rel) of the
+    largest singular value.  Solved as an augmented least-squares problem
+    [Xc; sqrt(lam) I] A = [Yc; 0] with an fp64 least-squares routine.
     """
     X, Y = _f64(X), _f64(Y)
     H, R, d = X.shape
     A = np.empty((H, d, d), dtype=np.float64)
     b = np.empty((H, d), dtype=np.float64)
     for h in range(H):
-        D = np.concatenate([X[h], np.ones((R, 1))], axis=1)
-        W, *_ = np.linalg.lstsq(D, Y[h], rcond=None)
-        A[h] = W[:d]
-        b[h] = W[d]
+        xm = X[h].mean(axis=0)
+        ym = Y[h].mean(axis=0)
+        Xc = X[h] - xm
+        Yc = Y[h] - ym
+        lam = ridge_rel * float((Xc * Xc).sum(axis=0).max())
+        D = np.concatenate([Xc, np.sqrt(lam) * np.eye(d)], axis=0)
+        T = np.concatenate([Yc, np.zeros((d, Y.shape[-1]))], axis=0)
+        W, *_ = np.linalg.lstsq(D, T, rcond=None)
+        A[h] = W
+        b[h] = ym - xm @ W
     return A, b
 
 

@@ -90,15 +90,15 @@ def test_validation_errors_before_launch(lib):
     assert lib.zb_tile_sparse_attn(*a, 2, 1, 0.125, S, FAKE + 4, None, None) == 3
     assert lib.zb_tile_sparse_attn(*a, 2, 1, 0.125, _shape(N=128 * 40000), FAKE, None, None) == 4  # T > 32768
     # dense
-    assert lib.zb_dense_attn(FAKE, 0, FAKE, FAKE, 10, 2, 64, 0.125, FAKE, None, None) == 2
-    assert lib.zb_dense_attn(FAKE, 10, FAKE, FAKE, 10, 2, 128, 0.125, FAKE, None, None) == 4
+    assert lib.zb_dense_attn(FAKE, 0, FAKE, FAKE, 10, 2, 64, 0.125, FAKE, 0, None, None) == 2
+    assert lib.zb_dense_attn(FAKE, 10, FAKE, FAKE, 10, 2, 128, 0.125, FAKE, 1, None, None) == 4
     # linear
     need = lib.zb_linear_state_workspace_bytes(2, 256, 64)
     assert lib.zb_linear_state(FAKE, FAKE, 2, 256, 64, FAKE, FAKE, FAKE, need - 1, None) == 5
     assert lib.zb_linear_state(FAKE, FAKE, 2, 256, 64, FAKE, FAKE, None, need, None) == 5
     assert lib.zb_linear_state(FAKE, None, 2, 256, 64, FAKE, FAKE, FAKE, need, None) == 1
-    assert lib.zb_linear_apply(FAKE, 2, 256, 64, FAKE, None, None, None, FAKE, None) == 1
-    assert lib.zb_linear_apply(FAKE, 2, 256, 64, FAKE, FAKE, FAKE + 2, None, FAKE, None) == 3
+    assert lib.zb_linear_apply(FAKE, 2, 256, 64, FAKE, None, None, None, FAKE, 0, None) == 1
+    assert lib.zb_linear_apply(FAKE, 2, 256, 64, FAKE, FAKE, FAKE + 2, None, FAKE, 1, None) == 3
     # affine fit: too few rows, workspace
     assert lib.zb_affine_fit(FAKE, FAKE, 2, 64, 64, FAKE, FAKE, FAKE, 1 << 30, None) == 2
     wsn = lib.zb_affine_fit_workspace_bytes(2, 300, 64)

@@ -21,8 +21,9 @@ MUTATIONS = {
     "ties go to the upper index": ("order = np.lexsort((j, -flat[r]))", "order = np.lexsort((-j, -flat[r]))"),
     "softmax scale dropped": ("logit_parts = [scale * q @ K[h, cols].T]", "logit_parts = [q @ K[h, cols].T]"),
     "feature map off by one": ("x + 1.0, np.exp", "x, np.exp"),
-    "fit without intercept": ("D = np.concatenate([X[h], np.ones((R, 1))], axis=1)",
-                              "D = np.concatenate([X[h], np.zeros((R, 1))], axis=1)"),
+    "fit without intercept": ("b[h] = ym - xm @ W", "b[h] = 0.0 * ym"),
+    "ridge on the wrong side": ("D = np.concatenate([Xc, np.sqrt(lam) * np.eye(d)], axis=0)",
+                                "D = np.concatenate([Xc, -np.sqrt(lam) * np.eye(d) + 1.0], axis=0)"),
     "score transposed": ("np.matmul(Qbar, np.swapaxes(Kbar, -1, -2))",
                          "np.swapaxes(np.matmul(Qbar, np.swapaxes(Kbar, -1, -2)), -1, -2)"),
     "ragged tile divided by full size": ("out /= n[None, :, None].astype(np.float64)", "out /= float(tile)"),

@@ -246,25 +246,48 @@ def test_affine_fit_recovers_planted_map():
     b0 = RNG.standard_normal((H, d))
     Y = oracle.affine_apply(X, A0, b0)
     A, b = oracle.affine_fit(X, Y)
+    # the vanishing ridge (1e-8 relative) biases A by O(1e-8)
+    np.testing.assert_allclose(A, A0, rtol=0, atol=1e-6)
+    np.testing.assert_allclose(b, b0, rtol=0, atol=1e-6)
+    A, b = oracle.affine_fit(X, Y, ridge_rel=0.0)
     np.testing.assert_allclose(A, A0, rtol=0, atol=1e-10)
     np.testing.assert_allclose(b, b0, rtol=0, atol=1e-10)
 
 
 def test_affine_fit_identity():
     X = RNG.standard_normal((2, 100, 6))
-    A, b = oracle.affine_fit(X, X)
+    A, b = oracle.affine_fit(X, X, ridge_rel=0.0)
     np.testing.assert_allclose(A, np.broadcast_to(np.eye(6), A.shape), atol=1e-12)
     np.testing.assert_allclose(b, 0, atol=1e-12)
 
 
-def test_affine_fit_residual_orthogonal_to_design():
+def test_affine_fit_normal_equations_with_ridge():
+    # stationarity of ||[X 1] W - Y||^2 + lam ||A||^2:  [X 1]^T E = [lam A; 0]
     X = RNG.standard_normal((2, 300, 5))
     Y = RNG.standard_normal((2, 300, 5))
+    for rr in (0.0, 1e-8, 1e-2):
+        A, b = oracle.affine_fit(X, Y, ridge_rel=rr)
+        E = Y - oracle.affine_apply(X, A, b)
+        for h in range(2):
+            Xc = X[h] - X[h].mean(0)
+            lam = rr * (Xc * Xc).sum(0).max()
+            D = np.concatenate([X[h], np.ones((300, 1))], axis=1)
+            want = np.concatenate([lam * A[h], np.zeros((1, 5))], axis=0)
+            np.testing.assert_allclose(D.T @ E[h], want, atol=1e-9)
+
+
+def test_affine_fit_rank_deficient_calibration_is_finite():
+    # outputs varying in only 2 of 6 directions: plain least squares is singular,
+    # the vanishing ridge gives the minimum-norm-like finite solution that still
+    # reproduces Y on the calibration rows
+    H, R, d = 1, 200, 6
+    basis = RNG.standard_normal((2, d))
+    X = (RNG.standard_normal((H, R, 2)) @ basis) + 0.3
+    A0 = RNG.standard_normal((H, d, d))
+    Y = oracle.affine_apply(X, A0, np.ones((H, d)))
     A, b = oracle.affine_fit(X, Y)
-    E = Y - oracle.affine_apply(X, A, b)
-    for h in range(2):
-        D = np.concatenate([X[h], np.ones((300, 1))], axis=1)
-        np.testing.assert_allclose(D.T @ E[h], 0, atol=1e-10)
+    assert np.isfinite(A).all() and np.abs(A).max() < 1e3
+    np.testing.assert_allclose(oracle.affine_apply(X, A, b), Y, atol=1e-6)
 
 
 def test_calibration_rows():
