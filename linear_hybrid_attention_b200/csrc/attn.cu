@@ -79,7 +79,8 @@ struct Params {
     float log2_tk, log2_last;
     long long n_items;
     const int32_t* idx;
-    uint16_t* O;
+    void* O;
+    int out_fp32;      // 1: O is fp32, else bf16
     float* lse;
     int* status;
     unsigned long long timeout_ns;
@@ -497,15 +498,23 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
             const long long qrow = static_cast<long long>(i) * p.tq + row;
             if (row < p.tq && qrow < p.n_q) {
                 const float inv = 1.f / l;
-                uint4* dst = reinterpret_cast<uint4*>(p.O + (static_cast<long long>(h) * p.n_q + qrow) * HD);
+                const long long orow = (static_cast<long long>(h) * p.n_q + qrow) * HD;
+                if (p.out_fp32) {
+                    float4* dst = reinterpret_cast<float4*>(static_cast<float*>(p.O) + orow);
 #pragma unroll
-                for (int c = 0; c < HD / 8; ++c) {
-                    uint4 v;
-                    v.x = pack_bf16x2(o[c * 8 + 0] * inv, o[c * 8 + 1] * inv);
-                    v.y = pack_bf16x2(o[c * 8 + 2] * inv, o[c * 8 + 3] * inv);
-                    v.z = pack_bf16x2(o[c * 8 + 4] * inv, o[c * 8 + 5] * inv);
-                    v.w = pack_bf16x2(o[c * 8 + 6] * inv, o[c * 8 + 7] * inv);
-                    dst[c] = v;
+                    for (int c = 0; c < HD / 4; ++c)
+                        dst[c] = make_float4(o[c * 4] * inv, o[c * 4 + 1] * inv, o[c * 4 + 2] * inv, o[c * 4 + 3] * inv);
+                } else {
+                    uint4* dst = reinterpret_cast<uint4*>(static_cast<uint16_t*>(p.O) + orow);
+#pragma unroll
+                    for (int c = 0; c < HD / 8; ++c) {
+                        uint4 v;
+                        v.x = pack_bf16x2(o[c * 8 + 0] * inv, o[c * 8 + 1] * inv);
+                        v.y = pack_bf16x2(o[c * 8 + 2] * inv, o[c * 8 + 3] * inv);
+                        v.z = pack_bf16x2(o[c * 8 + 4] * inv, o[c * 8 + 5] * inv);
+                        v.w = pack_bf16x2(o[c * 8 + 6] * inv, o[c * 8 + 7] * inv);
+                        dst[c] = v;
+                    }
                 }
                 if (p.lse) p.lse[static_cast<long long>(h) * p.n_q + qrow] = (m + __log2f(l)) * 0.6931471805599453f;
             }
@@ -529,7 +538,8 @@ static size_t attn_smem_bytes() { return sizeof(attn::Smem) + 1024; }
 static zb_status launch_attn(const uint16_t* Q, const uint16_t* K, const uint16_t* V,
                              const uint16_t* Kb, const uint16_t* Vb, const int32_t* idx, int heads,
                              long long n_q, long long n_kv, int tq, int tk, int k, int dense,
-                             int use_lm, float scale, uint16_t* O, float* lse, cudaStream_t st) {
+                             int use_lm, float scale, void* O, int out_fp32, float* lse,
+                             cudaStream_t st) {
     using namespace attn;
     DeviceInfo dev;
     zb_status e = current_device(&dev);
@@ -567,6 +577,7 @@ static zb_status launch_attn(const uint16_t* Q, const uint16_t* K, const uint16_
     p.n_items = static_cast<long long>(heads) * Tq;
     p.idx = idx;
     p.O = O;
+    p.out_fp32 = out_fp32;
     p.lse = lse;
     p.status = dev.status;
     p.timeout_ns = wait_timeout_ns();
@@ -603,14 +614,14 @@ extern "C" zb_status zb_tile_sparse_attn(const uint16_t* Q, const uint16_t* K, c
         !aligned16(lse) || (lm && (!aligned16(Kbar_bf16) || !aligned16(Vbar_bf16))))
         return ZB_ERR_ALIGN;
     return launch_attn(Q, K, V, Kbar_bf16, Vbar_bf16, idx, s.heads, s.n_tokens, s.n_tokens, s.tile,
-                       s.tile, k, 0, use_landmarks ? 1 : 0, scale, O, lse,
+                       s.tile, k, 0, use_landmarks ? 1 : 0, scale, O, 0, lse,
                        static_cast<cudaStream_t>(stream));
 }
 
 extern "C" zb_status zb_dense_attn(const uint16_t* Q, int64_t n_q, const uint16_t* K,
                                    const uint16_t* V, int64_t n_kv, int32_t heads,
-                                   int32_t head_dim, float scale, uint16_t* O, float* lse,
-                                   void* stream) {
+                                   int32_t head_dim, float scale, void* O, int32_t out_fp32,
+                                   float* lse, void* stream) {
     if (heads < 1 || n_q < 1 || n_kv < 1) return ZB_ERR_SHAPE;
     if (head_dim != 64) return ZB_ERR_UNSUPPORTED;
     if (!Q || !K || !V || !O) return ZB_ERR_NULL;
@@ -620,5 +631,5 @@ extern "C" zb_status zb_dense_attn(const uint16_t* Q, int64_t n_q, const uint16_
         return ZB_ERR_ALIGN;
     const int Tk = static_cast<int>((n_kv + 127) / 128);
     return launch_attn(Q, K, V, nullptr, nullptr, nullptr, heads, n_q, n_kv, 128, 128, Tk, 1, 0,
-                       scale, O, lse, static_cast<cudaStream_t>(stream));
+                       scale, O, out_fp32 ? 1 : 0, lse, static_cast<cudaStream_t>(stream));
 }
