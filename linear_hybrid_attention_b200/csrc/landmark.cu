@@ -19,7 +19,8 @@
 namespace zb {
 namespace lmk {
 
-constexpr int THREADS = 256;
+constexpr int THREADS = 256;      // gather kernel
+constexpr int LM_THREADS = 512;   // landmark kernel: 16 warps, 8 rows each
 constexpr int HD = 64;
 
 __device__ __forceinline__ void add8(double (&acc)[8], const uint4& v) {
@@ -48,20 +49,21 @@ __device__ __forceinline__ uint16_t f64_to_bf16_rne(double x) {
 // Persistent landmark kernel: one CTA per SM walks (head, tile) items
 // round-robin.  Thread 0 copies the Q, K, V runs of an item (n_j rows x 128 B
 // each, contiguous) into a LM_STAGES-deep shared-memory ring with bulk copies;
-// warp w sums rows [16 w, 16 w + 16) of each tensor, lane l columns 2l, 2l+1,
-// in fp64 (exact for bf16 inputs unless a tile spans > ~38 binades); the 8
+// warp w sums rows [8 w, 8 w + 8) of each tensor, lane l columns 2l, 2l+1,
+// in fp64 (exact for bf16 inputs unless a tile spans > ~38 binades); the 16
 // warp partials are added in a fixed order by 192 threads, one output each.
-constexpr int LM_STAGES = 4;
+// 16 warps per SM hide the latency of the fp32 -> fp64 conversions.
+constexpr int LM_STAGES = 3;
 constexpr uint32_t RUN_BYTES = 128 * HD * 2;  // one full tile of one tensor
 
 struct LmSmem {
     uint8_t buf[LM_STAGES][3][RUN_BYTES];
-    double part[2][THREADS / 32][3][HD];
+    double part[2][LM_THREADS / 32][3][HD];
     uint64_t full[LM_STAGES];
     int abort_flag;
 };
 
-__global__ void __launch_bounds__(THREADS, 1)
+__global__ void __launch_bounds__(LM_THREADS, 1)
 landmark_kernel(const uint16_t* __restrict__ Q, const uint16_t* __restrict__ K,
                 const uint16_t* __restrict__ V, int heads, long long N, int tile, int T,
                 double* __restrict__ Qbar, double* __restrict__ Kbar, uint16_t* __restrict__ Kb16,
@@ -112,33 +114,26 @@ landmark_kernel(const uint16_t* __restrict__ Q, const uint16_t* __restrict__ K,
         item_of(it, h, j, n);
         const bool good = mbar_wait(smem_addr(&sm.full[s]), (it / LM_STAGES) & 1, wc);
         if (good) consumed = it + 1;
-        const int r0 = warp * 16;
-        const int rows = good ? max(0, min(16, n - r0)) : 0;
+        const int r0 = warp * 8;
+        const int rows = good ? max(0, min(8, n - r0)) : 0;
 #pragma unroll
         for (int t = 0; t < 3; ++t) {
             double a0 = 0.0, a1 = 0.0;
             if (t >= t0) {
                 const uint32_t* src = reinterpret_cast<const uint32_t*>(sm.buf[s][t]) + r0 * (HD / 2) + lane;
-                if (rows == 16) {
+                if (rows == 8) {
                     // all loads first, then a tree of adds (sums are exact, order-free)
-                    uint32_t wv[16];
+                    uint32_t wv[8];
 #pragma unroll
-                    for (int r = 0; r < 16; ++r) wv[r] = src[r * (HD / 2)];
-                    double l[8], h[8];
+                    for (int r = 0; r < 8; ++r) wv[r] = src[r * (HD / 2)];
+                    double l[4], h[4];
 #pragma unroll
-                    for (int r = 0; r < 8; ++r) {
+                    for (int r = 0; r < 4; ++r) {
                         l[r] = static_cast<double>(bf16_lo(wv[2 * r])) + static_cast<double>(bf16_lo(wv[2 * r + 1]));
                         h[r] = static_cast<double>(bf16_hi(wv[2 * r])) + static_cast<double>(bf16_hi(wv[2 * r + 1]));
                     }
-#pragma unroll
-                    for (int w = 4; w >= 1; w >>= 1)
-#pragma unroll
-                        for (int r = 0; r < w; ++r) {
-                            l[r] += l[r + w];
-                            h[r] += h[r + w];
-                        }
-                    a0 = l[0];
-                    a1 = h[0];
+                    a0 = (l[0] + l[1]) + (l[2] + l[3]);
+                    a1 = (h[0] + h[1]) + (h[2] + h[3]);
                 } else {
                     for (int r = 0; r < rows; ++r) {
                         const uint32_t wv = src[r * (HD / 2)];
@@ -158,7 +153,7 @@ landmark_kernel(const uint16_t* __restrict__ Q, const uint16_t* __restrict__ K,
             if (t >= t0) {
                 double acc = 0.0;
 #pragma unroll
-                for (int wp = 0; wp < THREADS / 32; ++wp) acc += sm.part[it & 1][wp][t][col];
+                for (int wp = 0; wp < LM_THREADS / 32; ++wp) acc += sm.part[it & 1][wp][t][col];
                 const double mean = acc / static_cast<double>(n);
                 const long long o = (static_cast<long long>(h) * T + j) * HD + col;
                 if (t == 0) {
@@ -228,7 +223,7 @@ extern "C" zb_status zb_landmark_build(const uint16_t* Q, const uint16_t* K, con
     if (cudaFuncSetAttribute(lmk::landmark_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              static_cast<int>(smem)) != cudaSuccess)
         return ZB_ERR_CUDA;
-    lmk::landmark_kernel<<<static_cast<unsigned>(grid), lmk::THREADS, smem, static_cast<cudaStream_t>(stream)>>>(
+    lmk::landmark_kernel<<<static_cast<unsigned>(grid), lmk::LM_THREADS, smem, static_cast<cudaStream_t>(stream)>>>(
         Q, K, V, s.heads, s.n_tokens, s.tile, T, Qbar, Kbar, Kbar_bf16, Vbar_bf16, dev.status,
         wait_timeout_ns());
     return cudaGetLastError() == cudaSuccess ? ZB_OK : ZB_ERR_CUDA;

@@ -61,16 +61,18 @@ inline size_t state_ws_bytes(int heads, long long n) {
     return static_cast<size_t>(g.pairs) * g.chunks * PARTIAL_FLOATS * sizeof(float);
 }
 
-// phi(x) = elu(x) + 1
-__device__ __forceinline__ float phi(float x) { return x > 0.f ? x + 1.f : __expf(x); }
+// phi(x) = elu(x) + 1 = max(x, 0) + exp(min(x, 0))  (x + 1 for x > 0, e^x otherwise)
+__device__ __forceinline__ float phi(float x) {
+    return fmaxf(x, 0.f) + ex2(fminf(x, 0.f) * 1.4426950408889634f);
+}
 
 // ============================================================== state ====
 constexpr int ST_STAGES = 3;
-constexpr int ST_THREADS = 128;
+constexpr int ST_THREADS = 512;  // 16 warps share the phi pass; warps 0..3 read TMEM
 
 struct StateSmem {
     uint8_t buf[ST_STAGES][4][TILE_BYTES];  // [stage][K0, K1, V0, V1]
-    float zred[4][2][HD];
+    float zred[ST_THREADS / 32][2][HD];
     uint64_t full[ST_STAGES], empty[ST_STAGES], done;
     uint32_t tmem_base;
     int abort_flag;
@@ -126,7 +128,7 @@ linear_state_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
 
     constexpr uint32_t IDESC = idesc_bf16(128, 128, 1, 1);
     const int cg = tid & 7;        // logical 16-byte feature group
-    const int rbase = tid >> 3;    // rows rbase + 16 m
+    const int rbase = tid >> 3;    // rows rbase + 64 m
     float z0[8], z1[8];
 #pragma unroll
     for (int e = 0; e < 8; ++e) z0[e] = z1[e] = 0.f;
@@ -145,8 +147,8 @@ linear_state_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
             for (int hh = 0; hh < 2; ++hh) {
                 uint8_t* kt = sm.buf[s][hh];
 #pragma unroll
-                for (int m = 0; m < 8; ++m) {
-                    const int r = rbase + 16 * m;
+                for (int m = 0; m < TILE / (ST_THREADS / 8); ++m) {
+                    const int r = rbase + (ST_THREADS / 8) * m;
                     uint4* p = reinterpret_cast<uint4*>(kt + r * 128 + ((cg ^ (r & 7)) << 4));
                     uint4 v = *p;
                     uint32_t w[4] = {v.x, v.y, v.z, v.w};
@@ -204,7 +206,7 @@ linear_state_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
     }
     tc_fence_after();
     float* part = partial + static_cast<size_t>(blockIdx.x) * PARTIAL_FLOATS;
-    if (steps > 0 && ok) {
+    if (steps > 0 && ok && tid < 128) {
         const int hs = tid >> 6;   // head slot of this TMEM lane
         const int f = tid & 63;    // feature row
         uint32_t r[64];
@@ -218,7 +220,7 @@ linear_state_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
         for (int c = 0; c < 16; ++c)
             dst[c] = make_float4(__uint_as_float(r[4 * c]), __uint_as_float(r[4 * c + 1]),
                                  __uint_as_float(r[4 * c + 2]), __uint_as_float(r[4 * c + 3]));
-    } else {
+    } else if (!(steps > 0 && ok)) {
         for (int e = tid; e < 2 * HD * HD; e += ST_THREADS) part[e] = 0.f;
     }
     // z: lanes cg, cg+8, cg+16, cg+24 of a warp share a feature group
@@ -238,11 +240,11 @@ linear_state_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
         }
     }
     __syncthreads();
-    {
+    if (tid < 128) {
         const int hs = tid >> 6, f = tid & 63;
         float zz = 0.f;
 #pragma unroll
-        for (int w = 0; w < 4; ++w) zz += sm.zred[w][hs][f];
+        for (int w = 0; w < ST_THREADS / 32; ++w) zz += sm.zred[w][hs][f];
         part[2 * HD * HD + hs * HD + f] = (steps > 0 && ok) ? zz : 0.f;
     }
     tc_fence_before();
@@ -271,7 +273,7 @@ __global__ void linear_state_reduce_kernel(const float* __restrict__ partial, in
 
 // ============================================================== apply ====
 constexpr int AP_STAGES = 4;
-constexpr int AP_THREADS = 128;
+constexpr int AP_THREADS = 256;  // 8 warps: the phi pass spreads over all; two threads per output row
 constexpr int BN_ROWS = 80;  // 64 columns of S A, one of z, 15 of zeros
 constexpr uint32_t B_BYTES = BN_ROWS * 128;
 
@@ -329,7 +331,7 @@ linear_apply_kernel(const __grid_constant__ CUtensorMap tm_q, int heads, long lo
 
     constexpr uint32_t IDESC = idesc_bf16(128, BN_ROWS, 0, 0);
     const int cg = tid & 7, rbase = tid >> 3;
-    const uint32_t lane_addr = static_cast<uint32_t>(warp * 32) << 16;
+    const uint32_t lane_addr = static_cast<uint32_t>((warp & 3) * 32) << 16;  // warps w and w + 4 share lanes
     int h_prev = -1;
     int consumed = 0;
     bool ok = true;
@@ -339,24 +341,24 @@ linear_apply_kernel(const __grid_constant__ CUtensorMap tm_q, int heads, long lo
         const int buf = it & 1;
         if (!mbar_wait(smem_addr(&sm.mma_done[buf]), (it >> 1) & 1, wc)) return false;
         tc_fence_after();
-        uint32_t r[96];
+        // this thread: row (warp & 3) * 32 + lane, output columns [32 half, 32 half + 32)
+        const int half = warp >> 2;
+        uint32_t r[32], den;
         const uint32_t ta = tmem + lane_addr + buf * 128;
-        tmem_ld32(ta, sub32(r, 0));
-        tmem_ld32(ta + 32, sub32(r, 32));
-        tmem_ld32(ta + 64, sub32(r, 64));
-        tmem_wait_ld_dep(sub32(r, 0));
-        tmem_wait_ld_dep(sub32(r, 32));
-        tmem_wait_ld_dep(sub32(r, 64));
+        tmem_ld32(ta + half * 32, r);
+        asm volatile("tcgen05.ld.sync.aligned.32x32b.x1.b32 {%0}, [%1];" : "=r"(den) : "r"(ta + 64));
+        tmem_wait_ld_dep(r);
+        asm volatile("tcgen05.wait::ld.sync.aligned;" : "+r"(den)::"memory");
         tc_fence_before();
         const long long item = first + it;
         const int h = static_cast<int>(item / Tn), t = static_cast<int>(item % Tn);
-        const long long row = static_cast<long long>(t) * TILE + tid;
+        const long long row = static_cast<long long>(t) * TILE + (warp & 3) * 32 + lane;
         if (row < n_q) {
-            const float inv = 1.f / __uint_as_float(r[64]);
-            uint4* dst = reinterpret_cast<uint4*>(O + (static_cast<long long>(h) * n_q + row) * HD);
-            const float* bb = sm.bvec[h & 1];
+            const float inv = 1.f / __uint_as_float(den);
+            uint4* dst = reinterpret_cast<uint4*>(O + (static_cast<long long>(h) * n_q + row) * HD + half * 32);
+            const float* bb = sm.bvec[h & 1] + half * 32;
 #pragma unroll
-            for (int c = 0; c < HD / 8; ++c) {
+            for (int c = 0; c < 4; ++c) {
                 float o[8];
 #pragma unroll
                 for (int e = 0; e < 8; ++e) o[e] = fmaf(__uint_as_float(r[c * 8 + e]), inv, bb[c * 8 + e]);
@@ -397,15 +399,15 @@ linear_apply_kernel(const __grid_constant__ CUtensorMap tm_q, int heads, long lo
             }
             {
                 const int ncol = tid & 63;       // output column n
-                const int khalf = tid >> 6;      // rows k in [32 khalf, 32 khalf + 32)
+                const int kpart = tid >> 6;      // rows k in [16 kpart, 16 kpart + 16)
                 float acol[HD];
 #pragma unroll
                 for (int m = 0; m < HD; ++m) acol[m] = Ah ? __ldg(Ah + m * HD + ncol) : (m == ncol ? 1.f : 0.f);
-                for (int kq = 0; kq < 32; kq += 2) {
+                for (int kq = 0; kq < 16; kq += 2) {
                     float v2[2];
 #pragma unroll
                     for (int u = 0; u < 2; ++u) {
-                        const int k = khalf * 32 + kq + u;
+                        const int k = kpart * 16 + kq + u;
                         const float* srow = Sh + k * HD;
                         const float zk = __ldg(zh + k);
                         float acc = 0.f;
@@ -413,7 +415,7 @@ linear_apply_kernel(const __grid_constant__ CUtensorMap tm_q, int heads, long lo
                         for (int m = 0; m < HD; ++m) acc = fmaf(fmaf(-zk, sm.cvec[m], __ldg(srow + m)), acol[m], acc);
                         v2[u] = acc;
                     }
-                    const int k = khalf * 32 + kq;  // even: both land in one 32-bit word
+                    const int k = kpart * 16 + kq;  // even: both land in one 32-bit word
                     const int off = ncol * 128 + ((((k >> 3) ^ (ncol & 7))) << 4) + (k & 7) * 2;
                     *reinterpret_cast<uint32_t*>(bo + off) = pack_bf16x2(v2[0], v2[1]);
                 }
@@ -435,8 +437,8 @@ linear_apply_kernel(const __grid_constant__ CUtensorMap tm_q, int heads, long lo
         if (ok) {
             uint8_t* qt = sm.q[s];
 #pragma unroll
-            for (int m = 0; m < 8; ++m) {
-                const int r = rbase + 16 * m;
+            for (int m = 0; m < TILE / (AP_THREADS / 8); ++m) {
+                const int r = rbase + (AP_THREADS / 8) * m;
                 uint4* p = reinterpret_cast<uint4*>(qt + r * 128 + ((cg ^ (r & 7)) << 4));
                 uint4 v = *p;
                 uint32_t w[4] = {v.x, v.y, v.z, v.w};
