@@ -10,20 +10,32 @@
 // computed.  A landmark's logit carries + ln(n_j) so that it weighs as much as
 // the n_j keys it stands for.
 //
-// Kernel design (one persistent CTA per SM, 192 threads):
-//   warp 0      TMA producer: Q tile of the work item, then for each step the
-//               K and V tile of a selected key tile or a 128-landmark chunk,
-//               into a KV_STAGES-deep ring; also the selected-tile bitmap.
-//   warp 1      MMA issuer (one lane): S = Q K^T into a double-buffered TMEM S,
-//               then O += P V with P read from TMEM (tcgen05 "TS" form).
-//   warps 2..5  softmax warpgroup: one thread per query row; loads its S row
-//               from TMEM, masks, online softmax in the log2 domain with lazy
-//               rescaling of O, writes P (bf16) to TMEM; epilogue O / l.
-// A work item is one (head, query tile); items are dealt round-robin so that
-// CTAs running at the same time work on neighbouring query tiles of the same
-// head and sweep that head's K/V in ascending order together (L2 reuse).
+// Kernel design: one persistent CTA per SM, 384 threads, two work items in
+// flight ("slots").  A work item is one (head, query tile); the CTA's items
+// alternate between the slots.  With d = 64 the softmax (16,384 exponentials
+// per 128 x 128 tile) costs more than the tile's two MMAs, so both slots'
+// softmax warpgroups run at the same time while one warp keeps the tensor core
+// fed for both.
+//   warp 0      Q and K producer (TMA): Q of each slot's item, then K tiles of
+//               the selected key tiles / landmark chunks into a K ring.
+//   warp 2      V producer (TMA): the matching V tiles into a separate V ring
+//               (K is released after Q K^T, V only after P V).
+//   warp 1      MMA issuer (one lane): per slot S = Q K^T into the slot's TMEM
+//               S, then O += P V with P read from TMEM (tcgen05 "TS" form).
+//   warp 3      checks every index list (range, strictly ascending).
+//   warps 4..7  softmax of slot 0, warps 8..11 softmax of slot 1: one thread
+//               per query row; log2-domain online softmax with lazy
+//               rescaling of O, P (bf16) to TMEM, epilogue O / l.
+// A softmax thread reads its S row from TMEM twice in 32-column chunks (once
+// for the row max, once for the exponentials): compact code (the instruction
+// cache is shared by 12 warps running different roles) and few registers.
+// Items are dealt round-robin over CTAs, so CTAs running at the same time work
+// on neighbouring query tiles of one head and sweep its K/V in ascending order
+// together (L2 reuse).
 #include <cuda.h>
 #include <cuda_runtime.h>
+
+#include <mutex>
 
 #include "zb_common.cuh"
 #include "zb_host.h"
@@ -34,32 +46,28 @@ namespace attn {
 constexpr int BM = 128;          // query rows per work item (MMA M)
 constexpr int BN = 128;          // keys per step (QK MMA N, PV MMA K)
 constexpr int HD = 64;           // head dim
-constexpr int KV_STAGES = 4;
-constexpr int NUM_THREADS = 192;
-constexpr int MAX_TILES = 32768;  // bitmap capacity (key tiles)
+constexpr int SLOTS = 2;
+constexpr int K_STAGES = 6;
+constexpr int V_STAGES = 4;
+constexpr int NUM_THREADS = 384;
+constexpr int MAX_TILES = 32768;
 constexpr uint32_t TILE_BYTES = BN * HD * 2;  // 16 KB, one 128 x 64 bf16 tile
 constexpr uint32_t TMEM_COLS = 512;
-// TMEM column map
-constexpr uint32_t TM_S0 = 0;     // S buffer 0: 128 fp32 columns
-constexpr uint32_t TM_S1 = 128;   // S buffer 1
-constexpr uint32_t TM_O = 256;    // O accumulator: 64 fp32 columns
-constexpr uint32_t TM_P0 = 320;   // P buffer 0: 128 bf16 packed in 64 columns
-constexpr uint32_t TM_P1 = 384;   // P buffer 1
+// TMEM columns of slot s start at 256 s: S (128 fp32), P (64 = 128 bf16), O (64 fp32)
+constexpr uint32_t SLOT_COLS = 256, TM_S = 0, TM_P = 128, TM_O = 192;
 
+constexpr uint32_t SLEEP_NS = 20000;
 constexpr float LOG2E = 1.4426950408889634f;
 constexpr float RESCALE_THRESHOLD = 8.0f;  // log2 units: p <= 2^8 before a rescale
 
 struct Smem {
-    uint8_t q[2][TILE_BYTES];
-    uint8_t k[KV_STAGES][TILE_BYTES];
-    uint8_t v[KV_STAGES][TILE_BYTES];
-    uint32_t bitmap[2][MAX_TILES / 32];
-    uint64_t q_full[2], q_empty[2];
-    uint64_t kv_full[KV_STAGES], kv_empty[KV_STAGES];
-    uint64_t s_full[2], s_free[2];
-    uint64_t p_full[2], p_free[2];
-    uint64_t o_free;
-    uint64_t bm_full[2], bm_empty[2];
+    uint8_t q[SLOTS][TILE_BYTES];
+    uint8_t k[K_STAGES][TILE_BYTES];
+    uint8_t v[V_STAGES][TILE_BYTES];
+    uint64_t q_full[SLOTS], q_empty[SLOTS];
+    uint64_t k_full[K_STAGES], k_empty[K_STAGES];
+    uint64_t v_full[V_STAGES], v_empty[V_STAGES];
+    uint64_t s_full[SLOTS], s_free[SLOTS], p_full[SLOTS], p_free[SLOTS], o_free[SLOTS];
     uint64_t drain;
     uint32_t tmem_base;
     int abort_flag;
@@ -73,7 +81,6 @@ struct Params {
     int n_last;        // keys in the last key tile
     int k;             // selected key tiles per query tile (dense: Tk)
     int dense;         // 1: keep every key tile, no index list
-    int use_lm;        // landmarks for unselected tiles
     int lm_chunks;     // ceil(Tk / 128) when landmarks are used, else 0
     float scale_log2;  // softmax scale * log2(e)
     float log2_tk, log2_last;
@@ -86,8 +93,66 @@ struct Params {
     unsigned long long timeout_ns;
 };
 
-__device__ __forceinline__ int steps_of(const Params& p) {
-    return p.k + p.lm_chunks;
+// 32 lanes x 16 consecutive 32-bit columns
+ZB_DEVINL void tmem_st16(uint32_t taddr, const uint32_t* r) {
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
+        "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(taddr),
+        "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),
+        "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15])
+        : "memory");
+}
+
+// 2^x of one value on the FMA pipes (see f2_exp2_poly for the method).
+ZB_DEVINL float exp2_poly(float x) {
+    constexpr float kShift = 12582912.0f;  // 1.5 * 2^23
+    constexpr float kC1 = 0.695116758f, kC2 = 0.227644995f, kC3 = 0.0770670399f;
+    x = fmaxf(x, -127.f);
+    const float t = __fadd_rd(x, kShift);
+    const float f = x - (t - kShift);
+    float p = fmaf(kC3, f, kC2);
+    p = fmaf(p, f, kC1);
+    p = fmaf(p, f, 1.f);
+    return __uint_as_float(__float_as_uint(p) + (__float_as_uint(t) << 23));
+}
+
+// Shared-memory descriptors of the 128-byte-swizzle operand tiles, split in
+// 32-bit halves: the low word holds the start address (>> 4) and LBO, the high
+// word SBO = 1024, the tcgen05 version bit and the swizzle mode, which are the
+// same for every tile here.  Stepping along a tile only adds to the low word
+// (the address field never overflows into LBO: shared memory is < 256 KB).
+constexpr uint32_t DESC_HI = (1024u >> 4) | (1u << 14) | (2u << 29);
+ZB_DEVINL uint32_t desc_lo(uint32_t saddr, uint32_t lbo) { return ((saddr >> 4) & 0x3FFFu) | ((lbo >> 4) << 16); }
+
+// D[tmem] (+)= A[smem] * B[smem], descriptors given by their low words
+ZB_DEVINL void mma_ss(uint32_t d_tmem, uint32_t a_lo, uint32_t b_lo, uint32_t idesc, uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t.reg .b64 da, db;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "mov.b64 da, {%1, %5};\n\t"
+        "mov.b64 db, {%2, %5};\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], da, db, %3, p;\n\t}" ::"r"(d_tmem),
+        "r"(a_lo), "r"(b_lo), "r"(idesc), "r"(accumulate), "r"(DESC_HI)
+        : "memory");
+}
+
+// D[tmem] (+)= A[tmem] * B[smem], B's descriptor given by its low word
+ZB_DEVINL void mma_ts(uint32_t d_tmem, uint32_t a_tmem, uint32_t b_lo, uint32_t idesc, uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t.reg .b64 db;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "mov.b64 db, {%2, %5};\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], db, %3, p;\n\t}" ::"r"(d_tmem),
+        "r"(a_tmem), "r"(b_lo), "r"(idesc), "r"(accumulate), "r"(DESC_HI)
+        : "memory");
+}
+
+// The key tile of step j of an item: selected tile idx[j] (clamped), or -1 for a landmark chunk.
+ZB_DEVINL int step_tile(const Params& p, const int32_t* list, int j) {
+    if (j >= p.k) return -1;
+    if (p.dense) return j;
+    int t = __ldg(list + j);
+    return t < 0 ? 0 : (t >= p.Tk ? p.Tk - 1 : t);
 }
 
 __global__ void __launch_bounds__(NUM_THREADS, 1)
@@ -98,34 +163,40 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
     Smem& sm = *reinterpret_cast<Smem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const int warp = warp_id();
     const int lane = lane_id();
+    const int wg = warp >> 2;
     const WaitCtx wc{p.status, &sm.abort_flag, p.timeout_ns};
-    const int n_steps = steps_of(p);
+    const int n = p.k + p.lm_chunks;  // steps per item
+    const long long first = blockIdx.x, G = gridDim.x;
+    const int cnt = first < p.n_items ? static_cast<int>((p.n_items - 1 - first) / G + 1) : 0;
+    const int rounds = (cnt + 1) / 2;
 
     // ---------------------------------------------------------- set-up ----
     // Zero the operand buffers once: a 64-row TMA box leaves rows 64..127 of
     // a buffer untouched, and those rows must hold finite values.
     {
         uint4* z = reinterpret_cast<uint4*>(&sm.q[0][0]);
-        const int n16 = (2 + 2 * KV_STAGES) * TILE_BYTES / 16;
+        const int n16 = (SLOTS + K_STAGES + V_STAGES) * TILE_BYTES / 16;
         for (int i = threadIdx.x; i < n16; i += NUM_THREADS) z[i] = make_uint4(0, 0, 0, 0);
     }
     if (threadIdx.x == 0) {
         sm.abort_flag = 0;
-        for (int i = 0; i < 2; ++i) {
-            mbar_init(smem_addr(&sm.q_full[i]), 1);
-            mbar_init(smem_addr(&sm.q_empty[i]), 1);
-            mbar_init(smem_addr(&sm.s_full[i]), 1);
-            mbar_init(smem_addr(&sm.s_free[i]), 128);
-            mbar_init(smem_addr(&sm.p_full[i]), 128);
-            mbar_init(smem_addr(&sm.p_free[i]), 1);
-            mbar_init(smem_addr(&sm.bm_full[i]), 1);
-            mbar_init(smem_addr(&sm.bm_empty[i]), 128);
+        for (int s = 0; s < SLOTS; ++s) {
+            mbar_init(smem_addr(&sm.q_full[s]), 1);
+            mbar_init(smem_addr(&sm.q_empty[s]), 1);
+            mbar_init(smem_addr(&sm.s_full[s]), 1);
+            mbar_init(smem_addr(&sm.s_free[s]), 128);
+            mbar_init(smem_addr(&sm.p_full[s]), 128);
+            mbar_init(smem_addr(&sm.p_free[s]), 1);
+            mbar_init(smem_addr(&sm.o_free[s]), 128);
         }
-        for (int i = 0; i < KV_STAGES; ++i) {
-            mbar_init(smem_addr(&sm.kv_full[i]), 1);
-            mbar_init(smem_addr(&sm.kv_empty[i]), 1);
+        for (int i = 0; i < K_STAGES; ++i) {
+            mbar_init(smem_addr(&sm.k_full[i]), 1);
+            mbar_init(smem_addr(&sm.k_empty[i]), 1);
         }
-        mbar_init(smem_addr(&sm.o_free), 128);
+        for (int i = 0; i < V_STAGES; ++i) {
+            mbar_init(smem_addr(&sm.v_full[i]), 1);
+            mbar_init(smem_addr(&sm.v_empty[i]), 1);
+        }
         mbar_init(smem_addr(&sm.drain), 1);
         fence_mbar_init();
     }
@@ -145,106 +216,68 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
     tc_fence_after();
     const uint32_t tmem = sm.tmem_base;
 
-    if (warp == 0) {
-        // ============================================== TMA producer ====
-        // Lane 0 does every wait and issues every copy; the warp helps read
-        // the index list and build the bitmap.  Each wait's outcome is
-        // broadcast so that all lanes leave the loops together.
-        const uint32_t FULL = 0xffffffffu;
-        long long g = 0;
-        int it = 0;
-        // per-buffer bit: a load was issued / parity of the last one issued
-        uint32_t kv_issued = 0, kv_parity = 0, q_issued = 0, q_parity = 0;
-        bool ok = true;
-        for (long long item = blockIdx.x; item < p.n_items && ok; item += gridDim.x, ++it) {
-            const int h = static_cast<int>(item / p.Tq);
-            const int i = static_cast<int>(item % p.Tq);
-            const int32_t* list = p.dense ? nullptr : p.idx + item * static_cast<long long>(p.k);
-            // selected-tile bitmap for the landmark steps of this item
-            if (p.lm_chunks) {
-                const int b = it & 1;
-                int w_ok = 1;
-                if (lane == 0) w_ok = mbar_wait(smem_addr(&sm.bm_empty[b]), ((it >> 1) & 1) ^ 1, wc);
-                if (!__shfl_sync(FULL, w_ok, 0)) { ok = false; break; }
-                uint32_t* bm = sm.bitmap[b];
-                const int words = (p.Tk + 31) >> 5;
-                for (int w = lane; w < words; w += 32) bm[w] = 0u;
-                __syncwarp();
-                int bad = 0;
-                for (int q0 = 0; q0 < p.k; q0 += 32) {
-                    const int qq = q0 + lane;
-                    const int j = qq < p.k ? list[qq] : 0;
-                    int jprev = __shfl_up_sync(FULL, j, 1);
-                    if (lane == 0) jprev = (q0 == 0) ? -1 : list[q0 - 1];
-                    if (qq < p.k) {
-                        if (j < 0 || j >= p.Tk || j <= jprev) bad = 1;
-                        else atomicOr(&bm[j >> 5], 1u << (j & 31));
-                    }
-                }
-                if (__any_sync(FULL, bad) && lane == 0) flag_status(p.status, ZB_ERR_INDEX);
-                __syncwarp();
-                if (lane == 0) mbar_arrive(smem_addr(&sm.bm_full[b]));
-            }
-            // Q tile
-            const int qs = it & 1;
-            {
-                int w_ok = 1;
-                if (lane == 0) {
-                    w_ok = mbar_wait(smem_addr(&sm.q_empty[qs]), ((it >> 1) & 1) ^ 1, wc);
-                    if (w_ok) {
-                        const uint32_t bar = smem_addr(&sm.q_full[qs]);
-                        mbar_arrive_expect_tx(bar, p.tq * HD * 2);
-                        tma_load_3d(smem_addr(sm.q[qs]), &tm_q, bar, 0, i * p.tq, h);
-                        q_issued |= 1u << qs;
-                        q_parity = (q_parity & ~(1u << qs)) | (((it >> 1) & 1u) << qs);
-                    }
-                }
-                if (!__shfl_sync(FULL, w_ok, 0)) { ok = false; break; }
-            }
-            // K/V steps
-            int jcache = 0;
-            for (int st = 0; st < n_steps; ++st) {
-                const long long gg = g + st;
-                const int s = static_cast<int>(gg % KV_STAGES);
-                const uint32_t use = static_cast<uint32_t>(gg / KV_STAGES);
-                if (!p.dense && st < p.k && (st & 31) == 0) {
-                    const int qq = st + lane;
-                    jcache = qq < p.k ? list[qq] : 0;
-                }
-                int j = st;
-                if (!p.dense && st < p.k) j = __shfl_sync(FULL, jcache, st & 31);
-                int w_ok = 1;
-                if (lane == 0) {
-                    w_ok = mbar_wait(smem_addr(&sm.kv_empty[s]), (use & 1) ^ 1, wc);
-                    if (w_ok) {
-                        const uint32_t bar = smem_addr(&sm.kv_full[s]);
-                        if (st < p.k) {
-                            j = j < 0 ? 0 : (j >= p.Tk ? p.Tk - 1 : j);
-                            mbar_arrive_expect_tx(bar, 2u * p.tk * HD * 2);
-                            tma_load_3d(smem_addr(sm.k[s]), &tm_k, bar, 0, j * p.tk, h);
-                            tma_load_3d(smem_addr(sm.v[s]), &tm_v, bar, 0, j * p.tk, h);
-                        } else {
-                            const int c = st - p.k;
-                            mbar_arrive_expect_tx(bar, 2u * TILE_BYTES);
-                            tma_load_3d(smem_addr(sm.k[s]), &tm_kb, bar, 0, c * BN, h);
-                            tma_load_3d(smem_addr(sm.v[s]), &tm_vb, bar, 0, c * BN, h);
-                        }
-                        kv_issued |= 1u << s;
-                        kv_parity = (kv_parity & ~(1u << s)) | ((use & 1u) << s);
-                    }
-                }
-                if (!__shfl_sync(FULL, w_ok, 0)) { ok = false; break; }
-            }
-            g += n_steps;
-        }
-        // Leave no TMA write in flight: wait (bounded, even after an abort) for
-        // the last load issued into every buffer.
+    if (warp == 0 || warp == 2) {
         if (lane == 0) {
+            // =========================== producers: warp 0 Q + K, warp 2 V ====
+            const bool is_k = warp == 0;
+            const int STAGES = is_k ? K_STAGES : V_STAGES;
+            uint64_t* full = is_k ? sm.k_full : sm.v_full;
+            uint64_t* empty = is_k ? sm.k_empty : sm.v_empty;
+            uint8_t(*buf)[TILE_BYTES] = is_k ? sm.k : sm.v;
+            const CUtensorMap* map = is_k ? &tm_k : &tm_v;
+            const CUtensorMap* lmap = is_k ? &tm_kb : &tm_vb;
+            uint32_t seq = 0;                    // loads issued into the ring
+            uint32_t issued_mask = 0, parity_mask = 0, q_issued = 0, q_parity = 0;
+            bool ok = true;
+            for (int r = 0; r < rounds && ok; ++r) {
+                const int A = (2 * r + 1 < cnt) ? 2 : 1;
+                int hs[SLOTS], is_[SLOTS];
+                const int32_t* lists[SLOTS];
+#pragma unroll
+                for (int s = 0; s < SLOTS; ++s) {
+                    if (s >= A) break;
+                    const long long item = first + static_cast<long long>(2 * r + s) * G;
+                    hs[s] = static_cast<int>(item / p.Tq);
+                    is_[s] = static_cast<int>(item % p.Tq);
+                    lists[s] = p.dense ? nullptr : p.idx + item * static_cast<long long>(p.k);
+                    if (is_k) {
+                        if (!mbar_wait(smem_addr(&sm.q_empty[s]), (r & 1) ^ 1, wc)) { ok = false; break; }
+                        const uint32_t bar = smem_addr(&sm.q_full[s]);
+                        mbar_arrive_expect_tx(bar, p.tq * HD * 2);
+                        tma_load_3d(smem_addr(sm.q[s]), &tm_q, bar, 0, is_[s] * p.tq, hs[s]);
+                        q_issued |= 1u << s;
+                        q_parity = (q_parity & ~(1u << s)) | ((r & 1u) << s);
+                    }
+                }
+                if (!ok) break;
+                for (int j = 0; j < n && ok; ++j) {
+#pragma unroll
+                    for (int s = 0; s < SLOTS; ++s) {
+                        if (s >= A) break;
+                        const int st = static_cast<int>(seq % STAGES);
+                        const uint32_t use = seq / STAGES;
+                        if (!mbar_wait(smem_addr(&empty[st]), (use & 1) ^ 1, wc)) { ok = false; break; }
+                        const uint32_t bar = smem_addr(&full[st]);
+                        const int t = step_tile(p, lists[s], j);
+                        if (t >= 0) {
+                            mbar_arrive_expect_tx(bar, p.tk * HD * 2);
+                            tma_load_3d(smem_addr(buf[st]), map, bar, 0, t * p.tk, hs[s]);
+                        } else {
+                            mbar_arrive_expect_tx(bar, TILE_BYTES);
+                            tma_load_3d(smem_addr(buf[st]), lmap, bar, 0, (j - p.k) * BN, hs[s]);
+                        }
+                        issued_mask |= 1u << st;
+                        parity_mask = (parity_mask & ~(1u << st)) | ((use & 1u) << st);
+                        ++seq;
+                    }
+                }
+            }
+            // leave no TMA write in flight (bounded, even after an abort)
             volatile int no_abort = 0;
             const WaitCtx w2{p.status, &no_abort, p.timeout_ns};
-            for (int s = 0; s < KV_STAGES; ++s)
-                if ((kv_issued >> s) & 1u) mbar_wait(smem_addr(&sm.kv_full[s]), (kv_parity >> s) & 1u, w2);
-            for (int s = 0; s < 2; ++s)
+            for (int st = 0; st < STAGES; ++st)
+                if ((issued_mask >> st) & 1u) mbar_wait(smem_addr(&full[st]), (parity_mask >> st) & 1u, w2);
+            for (int s = 0; s < SLOTS; ++s)
                 if ((q_issued >> s) & 1u) mbar_wait(smem_addr(&sm.q_full[s]), (q_parity >> s) & 1u, w2);
         }
         __syncwarp();
@@ -253,158 +286,207 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
         constexpr uint32_t IDESC_QK = idesc_bf16(BM, BN, 0, 0);  // Q K-major, K K-major
         constexpr uint32_t IDESC_PV = idesc_bf16(BM, HD, 0, 1);  // P (TMEM), V MN-major
         if (lane == 0) {
-            long long g = 0;
-            int it = 0;
+            const uint32_t q_lo0 = desc_lo(smem_addr(sm.q[0]), 16);
+            const uint32_t k_lo0 = desc_lo(smem_addr(sm.k[0]), 16);
+            const uint32_t v_lo0 = desc_lo(smem_addr(sm.v[0]), 0);
+            constexpr uint32_t TILE_LO = TILE_BYTES >> 4;
+            int k_next = 0, v_next = 0;
+            uint32_t k_ph = 0, v_ph = 0;
             bool ok = true;
-            for (long long item = blockIdx.x; item < p.n_items && ok; item += gridDim.x, ++it) {
-                const int qs = it & 1;
-                if (!mbar_wait(smem_addr(&sm.q_full[qs]), (it >> 1) & 1, wc)) { ok = false; break; }
+            auto issue_qk = [&](int s, long long g) -> bool {
+                const int ks = k_next;
+                if (!mbar_wait_sleep(smem_addr(&sm.k_full[ks]), k_ph, wc, SLEEP_NS)) return false;
+                if (++k_next == K_STAGES) { k_next = 0; k_ph ^= 1u; }
+                if (!mbar_wait_sleep(smem_addr(&sm.s_free[s]), static_cast<uint32_t>((g & 1) ^ 1), wc, SLEEP_NS)) return false;
                 tc_fence_after();
-                const uint32_t q_base = smem_addr(sm.q[qs]);
-                // S[b] = Q K_s^T for step gg
-                auto issue_qk = [&](long long gg) -> bool {
-                    const int s = static_cast<int>(gg % KV_STAGES);
-                    const uint32_t use = static_cast<uint32_t>(gg / KV_STAGES);
-                    const int b = static_cast<int>(gg & 1);
-                    const uint32_t buse = static_cast<uint32_t>(gg >> 1);
-                    if (!mbar_wait(smem_addr(&sm.kv_full[s]), use & 1, wc)) return false;
-                    if (!mbar_wait(smem_addr(&sm.s_free[b]), (buse & 1) ^ 1, wc)) return false;
-                    tc_fence_after();
-                    const uint32_t k_base = smem_addr(sm.k[s]);
-                    const uint32_t d_tmem = tmem + (b ? TM_S1 : TM_S0);
+                const uint32_t qa = q_lo0 + s * TILE_LO, kb = k_lo0 + ks * TILE_LO;
+                const uint32_t d_tmem = tmem + s * SLOT_COLS + TM_S;
 #pragma unroll
-                    for (int kk = 0; kk < HD / 16; ++kk) {
-                        const uint64_t ad = sdesc_sw128(q_base + kk * 32, 16, 1024);
-                        const uint64_t bd = sdesc_sw128(k_base + kk * 32, 16, 1024);
-                        umma_ss(d_tmem, ad, bd, IDESC_QK, kk > 0 ? 1u : 0u);
-                    }
-                    umma_commit(smem_addr(&sm.s_full[b]));
-                    return true;
-                };
-                if (!issue_qk(g)) { ok = false; break; }
-                for (int st = 0; st < n_steps; ++st) {
-                    const long long gg = g + st;
-                    if (st + 1 < n_steps) {
-                        if (!issue_qk(gg + 1)) { ok = false; break; }
-                    }
-                    if (st + 1 == n_steps) umma_commit(smem_addr(&sm.q_empty[qs]));
-                    const int b = static_cast<int>(gg & 1);
-                    const uint32_t buse = static_cast<uint32_t>(gg >> 1);
-                    if (!mbar_wait(smem_addr(&sm.p_full[b]), buse & 1, wc)) { ok = false; break; }
-                    if (st == 0) {
-                        if (!mbar_wait(smem_addr(&sm.o_free), (it & 1) ^ 1, wc)) { ok = false; break; }
-                    }
-                    tc_fence_after();
-                    const int s = static_cast<int>(gg % KV_STAGES);
-                    const uint32_t v_base = smem_addr(sm.v[s]);
-                    const uint32_t p_tmem = tmem + (b ? TM_P1 : TM_P0);
+                for (int kk = 0; kk < HD / 16; ++kk) mma_ss(d_tmem, qa + kk * 2, kb + kk * 2, IDESC_QK, kk > 0 ? 1u : 0u);
+                umma_commit(smem_addr(&sm.s_full[s]));
+                umma_commit(smem_addr(&sm.k_empty[ks]));
+                return true;
+            };
+            for (int r = 0; r < rounds && ok; ++r) {
+                const int A = (2 * r + 1 < cnt) ? 2 : 1;
+                for (int s = 0; s < A && ok; ++s)
+                    if (!mbar_wait_sleep(smem_addr(&sm.q_full[s]), r & 1, wc, SLEEP_NS)) ok = false;
+                if (!ok) break;
+                tc_fence_after();
+                for (int s = 0; s < A && ok; ++s)
+                    if (!issue_qk(s, static_cast<long long>(r) * n)) ok = false;
+                for (int j = 0; j < n && ok; ++j) {
+                    for (int s = 0; s < A; ++s) {
+                        const long long g = static_cast<long long>(r) * n + j;
+                        if (j + 1 < n) {
+                            if (!issue_qk(s, g + 1)) { ok = false; break; }
+                        } else {
+                            umma_commit(smem_addr(&sm.q_empty[s]));
+                        }
+                        if (!mbar_wait_sleep(smem_addr(&sm.p_full[s]), static_cast<uint32_t>(g & 1), wc, SLEEP_NS)) { ok = false; break; }
+                        if (j == 0) {
+                            if (!mbar_wait_sleep(smem_addr(&sm.o_free[s]), (r & 1) ^ 1, wc, SLEEP_NS)) { ok = false; break; }
+                        }
+                        const int vs = v_next;
+                        if (!mbar_wait_sleep(smem_addr(&sm.v_full[vs]), v_ph, wc, SLEEP_NS)) { ok = false; break; }
+                        if (++v_next == V_STAGES) { v_next = 0; v_ph ^= 1u; }
+                        tc_fence_after();
+                        const uint32_t vb = v_lo0 + vs * TILE_LO;
+                        const uint32_t p_tmem = tmem + s * SLOT_COLS + TM_P;
+                        const uint32_t o_tmem = tmem + s * SLOT_COLS + TM_O;
 #pragma unroll
-                    for (int kk = 0; kk < BN / 16; ++kk) {
-                        const uint64_t bd = sdesc_sw128(v_base + kk * 2048, 0, 1024);
-                        umma_ts(tmem + TM_O, p_tmem + kk * 8, bd, IDESC_PV, (st > 0 || kk > 0) ? 1u : 0u);
+                        for (int kk = 0; kk < BN / 16; ++kk)
+                            mma_ts(o_tmem, p_tmem + kk * 8, vb + kk * 128, IDESC_PV, (j > 0 || kk > 0) ? 1u : 0u);
+                        umma_commit(smem_addr(&sm.v_empty[vs]));
+                        umma_commit(smem_addr(&sm.p_free[s]));
                     }
-                    umma_commit(smem_addr(&sm.kv_empty[s]));
-                    umma_commit(smem_addr(&sm.p_free[b]));
                 }
-                g += n_steps;
             }
-            // No tcgen05.mma may still run when TMEM is released.
+            // no tcgen05.mma may still run when TMEM is released
             umma_commit(smem_addr(&sm.drain));
             volatile int no_abort = 0;
             const WaitCtx w2{p.status, &no_abort, p.timeout_ns};
             mbar_wait(smem_addr(&sm.drain), 0, w2);
         }
         __syncwarp();
-    } else {
-        // ============================================ softmax warpgroup ====
+    } else if (warp == 3) {
+        // ============================ index-list check (off the critical path) ====
+        // Every list must be in range and strictly ascending; a bad one sets
+        // ZB_ERR_INDEX (the kernel itself clamps indices and never reads out of
+        // bounds).  32 entries per step, one per lane.
+        if (!p.dense) {
+            for (int it = 0; it < cnt; ++it) {
+                const long long item = first + static_cast<long long>(it) * G;
+                const int32_t* list = p.idx + item * static_cast<long long>(p.k);
+                int bad = 0;
+                for (int q0 = 0; q0 < p.k; q0 += 32) {
+                    const int q = q0 + lane;
+                    const int t = q < p.k ? __ldg(list + q) : 0;
+                    int prev = __shfl_up_sync(0xffffffffu, t, 1);
+                    if (lane == 0) prev = q0 == 0 ? -1 : __ldg(list + q0 - 1);
+                    if (q < p.k && (t < 0 || t >= p.Tk || t <= prev)) bad = 1;
+                }
+                if (__any_sync(0xffffffffu, bad)) {
+                    if (lane == 0) flag_status(p.status, ZB_ERR_INDEX);
+                    break;
+                }
+            }
+        }
+    } else if (wg >= 1) {
+        // ===================================== softmax warpgroup of a slot ====
+        const int s = wg - 1;
         const int quarter = warp & 3;            // TMEM lane quarter this warp may access
         const int row = quarter * 32 + lane;     // query row within the tile
         const uint32_t lane_addr = static_cast<uint32_t>(quarter * 32) << 16;
-        long long g = 0;
-        int it = 0;
+        const uint32_t tm_s = tmem + lane_addr + s * SLOT_COLS + TM_S;
+        const uint32_t tm_p = tmem + lane_addr + s * SLOT_COLS + TM_P;
+        const uint32_t tm_o = tmem + lane_addr + s * SLOT_COLS + TM_O;
         bool ok = true;
-        for (long long item = blockIdx.x; item < p.n_items && ok; item += gridDim.x, ++it) {
+        for (int r = 0; r < rounds && ok; ++r) {
+            const int it = 2 * r + s;
+            if (it >= cnt) break;
+            const long long item = first + static_cast<long long>(it) * G;
             const int h = static_cast<int>(item / p.Tq);
             const int i = static_cast<int>(item % p.Tq);
+            const int32_t* list = p.dense ? nullptr : p.idx + item * static_cast<long long>(p.k);
             // valid columns of the last selected tile (only the last key tile is ragged)
             int last_valid = p.tk;
             if (p.k > 0) {
-                const int jl = p.dense ? p.Tk - 1 : p.idx[item * static_cast<long long>(p.k) + p.k - 1];
+                const int jl = p.dense ? p.Tk - 1 : __ldg(list + p.k - 1);
                 if (jl == p.Tk - 1) last_valid = p.n_last;
             }
-            const uint32_t* bm = sm.bitmap[it & 1];
-            if (p.lm_chunks) {
-                if (!mbar_wait(smem_addr(&sm.bm_full[it & 1]), (it >> 1) & 1, wc)) { ok = false; break; }
-            }
+            int ip = 0;           // walk over the sorted index list for landmark masks
             float m = -INFINITY;  // running max of the log2-domain logits (lazy)
             float l = 0.f;        // running sum of 2^(x - m)
-            for (int st = 0; st < n_steps; ++st) {
-                const long long gg = g + st;
-                const int b = static_cast<int>(gg & 1);
-                const uint32_t buse = static_cast<uint32_t>(gg >> 1);
-                if (!mbar_wait(smem_addr(&sm.s_full[b]), buse & 1, wc)) { ok = false; break; }
+            long long g = static_cast<long long>(r) * n;
+            for (int j = 0; j < n; ++j, ++g) {
+                if (!mbar_wait(smem_addr(&sm.s_full[s]), static_cast<uint32_t>(g & 1), wc)) { ok = false; break; }
                 tc_fence_after();
-                float x[BN];
-                {
-                    uint32_t raw[BN];
-                    const uint32_t sa = tmem + lane_addr + (b ? TM_S1 : TM_S0);
-#pragma unroll
-                    for (int c = 0; c < BN / 32; ++c) tmem_ld32(sa + c * 32, sub32(raw, c * 32));
-#pragma unroll
-                    for (int c = 0; c < BN / 32; ++c) tmem_wait_ld_dep(sub32(raw, c * 32));
-#pragma unroll
-                    for (int e = 0; e < BN; ++e) x[e] = __uint_as_float(raw[e]);
-                }
-                tc_fence_before();
-                mbar_arrive(smem_addr(&sm.s_free[b]));
-                // ---- row max (tree of 3-input max; no long dependency chain)
-                // Selected tiles: max of the raw scores, scaled afterwards
-                // (scale > 0).  Landmark chunks: x = s * scale + bias first,
-                // bias = log2(n_j), or -inf for selected / out-of-range tiles.
-                const bool is_lm = st >= p.k;
-                const uint64_t c2 = f2_pack(p.scale_log2, p.scale_log2);
-                if (!is_lm) {
-                    const int valid = (st == p.k - 1) ? last_valid : p.tk;
-                    if (valid < BN) {
-#pragma unroll
-                        for (int e = 0; e < BN; ++e)
-                            if (e >= valid) x[e] = -INFINITY;
-                    }
-                } else {
-                    const int j0 = (st - p.k) * BN;
-#pragma unroll
-                    for (int w = 0; w < BN / 32; ++w) {
-                        const int jw = j0 + w * 32;
-                        uint32_t bits = (jw < p.Tk) ? bm[jw >> 5] : 0xFFFFFFFFu;
-                        if (jw + 32 > p.Tk) {  // the chunk runs past the last tile
-                            const int keep = p.Tk - jw;
-                            bits |= keep <= 0 ? 0xFFFFFFFFu : (0xFFFFFFFFu << keep);
+                const bool is_lm = j >= p.k;
+                // Per-column treatment of S: selected tiles mask columns past the
+                // tile's length; landmark chunks become s * scale + log2(n_j), or
+                // -inf for selected / out-of-range tiles (the selected ones come
+                // from a walk over the sorted index list, kept in 4 mask words).
+                const int valid = is_lm ? BN : ((j == p.k - 1) ? last_valid : p.tk);
+                const int j0 = (j - p.k) * BN;
+                uint32_t s0 = 0u, s1 = 0u, s2 = 0u, s3 = 0u;
+                if (is_lm) {
+                    while (ip < p.k) {
+                        const int t = __ldg(list + ip);
+                        if (t >= j0 + BN) break;
+                        if (t >= j0) {
+                            const int c = t - j0;
+                            const uint32_t bit = 1u << (c & 31);
+                            s0 |= (c >> 5) == 0 ? bit : 0u;
+                            s1 |= (c >> 5) == 1 ? bit : 0u;
+                            s2 |= (c >> 5) == 2 ? bit : 0u;
+                            s3 |= (c >> 5) == 3 ? bit : 0u;
                         }
+                        ++ip;
+                    }
+                    const int past = p.Tk - j0;  // columns >= past are beyond the last tile
+                    if (past < 32) s0 |= past <= 0 ? 0xFFFFFFFFu : (0xFFFFFFFFu << past);
+                    if (past < 64) s1 |= past <= 32 ? 0xFFFFFFFFu : (0xFFFFFFFFu << (past - 32));
+                    if (past < 96) s2 |= past <= 64 ? 0xFFFFFFFFu : (0xFFFFFFFFu << (past - 64));
+                    if (past < 128) s3 |= past <= 96 ? 0xFFFFFFFFu : (0xFFFFFFFFu << (past - 96));
+                }
+                // Per-column treatment of chunk c of S (raw words r): selected tiles
+                // mask columns past the tile's length; landmark chunks become
+                // s * scale + log2(n_j), or -inf for selected / out-of-range tiles.
+                auto treat = [&](float (&y)[32], const uint32_t (&r)[32], int c) {
+                    if (is_lm) {
+                        const uint32_t bits = c == 0 ? s0 : (c == 1 ? s1 : (c == 2 ? s2 : s3));
+                        const int lastc = p.Tk - 1 - j0 - c * 32;  // column of the ragged last tile
 #pragma unroll
-                        for (int e = 0; e < 32; e += 2) {
-                            const int j = jw + e;
-                            float b0 = (j == p.Tk - 1) ? p.log2_last : p.log2_tk;
-                            float b1 = (j + 1 == p.Tk - 1) ? p.log2_last : p.log2_tk;
-                            if ((bits >> e) & 1u) b0 = -INFINITY;
-                            if ((bits >> (e + 1)) & 1u) b1 = -INFINITY;
-                            float v0, v1;
-                            f2_unpack(f2_fma(f2_pack(x[w * 32 + e], x[w * 32 + e + 1]), c2, f2_pack(b0, b1)), v0, v1);
-                            x[w * 32 + e] = v0;
-                            x[w * 32 + e + 1] = v1;
+                        for (int e = 0; e < 32; ++e) {
+                            float bias = (e == lastc) ? p.log2_last : p.log2_tk;
+                            if ((bits >> e) & 1u) bias = -INFINITY;
+                            y[e] = fmaf(__uint_as_float(r[e]), p.scale_log2, bias);
+                        }
+                    } else {
+                        const int vc = valid - c * 32;  // valid columns in this chunk
+#pragma unroll
+                        for (int e = 0; e < 32; ++e) y[e] = __uint_as_float(r[e]);
+                        if (vc < 32) {  // only a ragged last tile (or a 64-row tile) needs the mask
+#pragma unroll
+                            for (int e = 0; e < 32; ++e)
+                                if (e >= vc) y[e] = -INFINITY;
                         }
                     }
-                }
-                float mx;
-                {
-                    float g[8];
+                };
+                // one 32-column chunk c of S into y[] (treated)
+                auto load_chunk = [&](float (&y)[32], int c) {
+                    uint32_t r[32];
+                    tmem_ld32(tm_s + c * 32, r);
+                    tmem_wait_ld_dep(r);
+                    treat(y, r, c);
+                };
+                // chunks c and c + 1 with one TMEM wait
+                auto load_chunk2 = [&](float (&y)[32], float (&z)[32], int c) {
+                    uint32_t r[32], r2[32];
+                    tmem_ld32(tm_s + c * 32, r);
+                    tmem_ld32(tm_s + c * 32 + 32, r2);
+                    tmem_wait_ld_dep(r);
+                    tmem_wait_ld_dep(r2);
+                    treat(y, r, c);
+                    treat(z, r2, c + 1);
+                };
+                // ---- pass 1: row max (two chunks per TMEM wait)
+                float mx = -INFINITY;
+#pragma unroll 1
+                for (int c = 0; c < BN / 32; c += 2) {
+                    float y[32], z[32];
+                    load_chunk2(y, z, c);
+                    float g0 = fmax3(y[0], y[1], y[2]), g1 = fmax3(z[0], z[1], z[2]);
+                    float g2 = fmax3(y[3], y[4], y[5]), g3 = fmax3(z[3], z[4], z[5]);
 #pragma unroll
-                    for (int q = 0; q < 8; ++q) {
-                        float t = fmax3(x[16 * q], x[16 * q + 1], x[16 * q + 2]);
-#pragma unroll
-                        for (int e = 3; e < 15; e += 2) t = fmax3(t, x[16 * q + e], x[16 * q + e + 1]);
-                        g[q] = fmaxf(t, x[16 * q + 15]);
+                    for (int e = 6; e < 30; e += 2) {
+                        g0 = fmax3(g0, y[e], y[e + 1]);
+                        g1 = fmax3(g1, z[e], z[e + 1]);
                     }
-                    mx = fmax3(fmax3(g[0], g[1], g[2]), fmax3(g[3], g[4], g[5]), fmaxf(g[6], g[7]));
+                    g2 = fmax3(g2, y[30], y[31]);
+                    g3 = fmax3(g3, z[30], z[31]);
+                    mx = fmaxf(mx, fmaxf(fmax3(g0, g1, g2), g3));
                 }
                 if (!is_lm) mx *= p.scale_log2;
                 // ---- lazy rescale: keep the old max unless the new one exceeds it by > 8
@@ -416,85 +498,79 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                     m = m_new;
                     l *= alpha;
                 }
-                const float msub = (m == -INFINITY) ? 0.f : m;
-                // ---- p = 2^(x - m): 3 of every 8 pairs on the FMA pipes, the
-                // rest on MUFU; packed fp32x2 arithmetic; 4 independent sums
-                uint32_t pk[BN / 2];
-                const uint64_t nm2 = f2_pack(-msub, -msub);
-                uint64_t acc[4] = {0ull, 0ull, 0ull, 0ull};
+                const float nm = (m == -INFINITY) ? 0.f : -m;
+                const float cm = is_lm ? 1.f : p.scale_log2;  // landmark logits are already scaled
+                // P of this slot is free once P V of the previous step is done;
+                // O then holds every earlier step and can be rescaled
+                if (!mbar_wait(smem_addr(&sm.p_free[s]), static_cast<uint32_t>((g & 1) ^ 1), wc)) { ok = false; break; }
+                tc_fence_after();
+                if (rescale && j > 0) {
+#pragma unroll 1
+                    for (int c = 0; c < HD / 32; ++c) {
+                        uint32_t ro[32];
+                        tmem_ld32(tm_o + c * 32, ro);
+                        tmem_wait_ld_dep(ro);
 #pragma unroll
-                for (int q = 0; q < BN / 2; ++q) {
-                    const uint64_t xin = f2_pack(x[2 * q], x[2 * q + 1]);
-                    const uint64_t xs = is_lm ? f2_add(xin, nm2) : f2_fma(xin, c2, nm2);
-                    uint64_t pv;
-                    if ((q & 7) < 3) {
-                        pv = f2_exp2_poly(xs);
-                    } else {
-                        float a0, a1;
-                        f2_unpack(xs, a0, a1);
-                        pv = f2_pack(ex2(a0), ex2(a1));
+                        for (int e = 0; e < 32; ++e) ro[e] = __float_as_uint(__uint_as_float(ro[e]) * alpha);
+                        tmem_st32(tm_o + c * 32, ro);
+                        tmem_wait_st();
                     }
-                    acc[q & 3] = f2_add(acc[q & 3], pv);
-                    float p0, p1;
-                    f2_unpack(pv, p0, p1);
-                    pk[q] = pack_bf16x2(p0, p1);
                 }
-                {
-                    float s0, s1, s2, s3;
-                    f2_unpack(f2_add(f2_add(acc[0], acc[1]), f2_add(acc[2], acc[3])), s0, s1);
-                    (void)s2;
-                    (void)s3;
-                    l += s0 + s1;
-                }
-                // P buffer b is free once PV of step gg-2 is done
-                if (!mbar_wait(smem_addr(&sm.p_free[b]), (buse & 1) ^ 1, wc)) { ok = false; break; }
-                if (rescale && st > 0) {
-                    // O must hold every PV up to step gg-1 before it is rescaled
-                    const long long gp = gg - 1;
-                    if (!mbar_wait(smem_addr(&sm.p_free[gp & 1]), static_cast<uint32_t>(gp >> 1) & 1, wc)) {
-                        ok = false;
-                        break;
+                // ---- pass 2: p = 2^(x * cm - m) per chunk (1 of 4 pairs on the FMA
+                // pipes, the rest on MUFU), packed fp32x2, bf16 pairs straight to TMEM
+                const uint64_t cm2 = f2_pack(cm, cm), nm2 = f2_pack(nm, nm);
+                uint64_t acc0 = 0ull, acc1 = 0ull;
+#pragma unroll 1
+                for (int c = 0; c < BN / 32; ++c) {
+                    float y[32];
+                    load_chunk(y, c);
+                    if (c == BN / 32 - 1) {
+                        tc_fence_before();
+                        mbar_arrive(smem_addr(&sm.s_free[s]));  // S fully read: the next Q K^T may overwrite it
                     }
-                    tc_fence_after();
-                    uint32_t ro[HD];
-                    const uint32_t oa = tmem + lane_addr + TM_O;
+                    uint32_t pk[16];
 #pragma unroll
-                    for (int c = 0; c < HD / 32; ++c) tmem_ld32(oa + c * 32, sub32(ro, c * 32));
-#pragma unroll
-                    for (int c = 0; c < HD / 32; ++c) tmem_wait_ld_dep(sub32(ro, c * 32));
-#pragma unroll
-                    for (int e = 0; e < HD; ++e) ro[e] = __float_as_uint(__uint_as_float(ro[e]) * alpha);
-#pragma unroll
-                    for (int c = 0; c < HD / 32; ++c) tmem_st32(oa + c * 32, sub32(ro, c * 32));
-                    tmem_wait_st();
+                    for (int q = 0; q < 16; ++q) {
+                        const uint64_t xs = f2_fma(f2_pack(y[2 * q], y[2 * q + 1]), cm2, nm2);
+                        uint64_t pv;
+                        if ((q & 3) == 1) {
+                            pv = f2_exp2_poly(xs);
+                        } else {
+                            float a0, a1;
+                            f2_unpack(xs, a0, a1);
+                            pv = f2_pack(ex2(a0), ex2(a1));
+                        }
+                        if (q & 1) acc1 = f2_add(acc1, pv); else acc0 = f2_add(acc0, pv);
+                        float p0, p1;
+                        f2_unpack(pv, p0, p1);
+                        pk[q] = pack_bf16x2(p0, p1);
+                    }
+                    tmem_st16(tm_p + c * 16, pk);
                 }
-                {
-                    const uint32_t pa = tmem + lane_addr + (b ? TM_P1 : TM_P0);
-#pragma unroll
-                    for (int c = 0; c < BN / 64; ++c) tmem_st32(pa + c * 32, sub32(pk, c * 32));
-                }
+                float rs0, rs1;
+                f2_unpack(f2_add(acc0, acc1), rs0, rs1);
+                l += rs0 + rs1;
                 tmem_wait_st();
                 tc_fence_before();
-                mbar_arrive(smem_addr(&sm.p_full[b]));
+                mbar_arrive(smem_addr(&sm.p_full[s]));
             }
             if (!ok) break;
-            if (p.lm_chunks) mbar_arrive(smem_addr(&sm.bm_empty[it & 1]));
             // ------------------------------------------------ epilogue ----
-            const long long gl = g + n_steps - 1;
-            if (!mbar_wait(smem_addr(&sm.p_free[gl & 1]), static_cast<uint32_t>(gl >> 1) & 1, wc)) { ok = false; break; }
+            const long long gl = g - 1;
+            if (!mbar_wait(smem_addr(&sm.p_free[s]), static_cast<uint32_t>(gl & 1), wc)) { ok = false; break; }
             tc_fence_after();
             float o[HD];
             {
                 uint32_t ro[HD];
 #pragma unroll
-                for (int c = 0; c < HD / 32; ++c) tmem_ld32(tmem + lane_addr + TM_O + c * 32, sub32(ro, c * 32));
+                for (int c = 0; c < HD / 32; ++c) tmem_ld32(tm_o + c * 32, sub32(ro, c * 32));
 #pragma unroll
                 for (int c = 0; c < HD / 32; ++c) tmem_wait_ld_dep(sub32(ro, c * 32));
 #pragma unroll
                 for (int e = 0; e < HD; ++e) o[e] = __uint_as_float(ro[e]);
             }
             tc_fence_before();
-            mbar_arrive(smem_addr(&sm.o_free));
+            mbar_arrive(smem_addr(&sm.o_free[s]));
             const long long qrow = static_cast<long long>(i) * p.tq + row;
             if (row < p.tq && qrow < p.n_q) {
                 const float inv = 1.f / l;
@@ -518,7 +594,6 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                 }
                 if (p.lse) p.lse[static_cast<long long>(h) * p.n_q + qrow] = (m + __log2f(l)) * 0.6931471805599453f;
             }
-            g += n_steps;
         }
     }
 
@@ -569,7 +644,6 @@ static zb_status launch_attn(const uint16_t* Q, const uint16_t* K, const uint16_
     p.n_last = static_cast<int>(n_kv - static_cast<long long>(Tk - 1) * tk);
     p.k = k;
     p.dense = dense;
-    p.use_lm = use_lm;
     p.lm_chunks = lm_chunks;
     p.scale_log2 = scale * LOG2E;
     p.log2_tk = log2f(static_cast<float>(tk));

@@ -58,6 +58,21 @@ ZB_DEVINL bool mbar_try_wait(uint32_t bar, uint32_t parity) {
     return ok != 0;
 }
 
+// As mbar_try_wait, but the thread may sleep up to `hint_ns` inside the call
+// (it wakes as soon as the phase completes): a waiting warp then takes no
+// issue slots from the warps doing work.
+ZB_DEVINL bool mbar_try_wait_sleep(uint32_t bar, uint32_t parity, uint32_t hint_ns) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.acquire.cta.shared::cta.b64 p, [%1], %2, %3;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(bar), "r"(parity), "r"(hint_ns)
+        : "memory");
+    return ok != 0;
+}
+
 // Everything a bounded wait needs: the device status word, a CTA-wide abort
 // flag in shared memory and the time limit.
 struct WaitCtx {
@@ -74,6 +89,24 @@ ZB_DEVINL bool mbar_wait(uint32_t bar, uint32_t parity, const WaitCtx& w) {
     const uint64_t t0 = globaltimer_ns();
     for (uint32_t it = 1;; ++it) {
         if (mbar_try_wait(bar, parity)) return true;
+        if ((it & 15u) == 0) {
+            if (*w.abort_flag) return false;
+            if (globaltimer_ns() - t0 > w.timeout_ns) {
+                flag_status(w.status, ZB_ERR_TIMEOUT);
+                *w.abort_flag = 1;
+                return false;
+            }
+        }
+    }
+}
+
+// mbar_wait with sleeping polls (at most `hint_ns` per poll; the time limit
+// and the abort flag are checked every 16 polls).
+ZB_DEVINL bool mbar_wait_sleep(uint32_t bar, uint32_t parity, const WaitCtx& w, uint32_t hint_ns) {
+    if (mbar_try_wait(bar, parity)) return true;
+    const uint64_t t0 = globaltimer_ns();
+    for (uint32_t it = 1;; ++it) {
+        if (mbar_try_wait_sleep(bar, parity, hint_ns)) return true;
         if ((it & 15u) == 0) {
             if (*w.abort_flag) return false;
             if (globaltimer_ns() - t0 > w.timeout_ns) {
