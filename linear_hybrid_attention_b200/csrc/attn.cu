@@ -47,28 +47,38 @@ constexpr int BM = 128;          // query rows per work item (MMA M)
 constexpr int BN = 128;          // keys per step (QK MMA N, PV MMA K)
 constexpr int HD = 64;           // head dim
 constexpr int SLOTS = 2;
-constexpr int K_STAGES = 6;
-constexpr int V_STAGES = 4;
+constexpr int K_STAGES = 3;      // per slot
+constexpr int V_STAGES = 2;      // per slot
 constexpr int NUM_THREADS = 384;
 constexpr int MAX_TILES = 32768;
 constexpr uint32_t TILE_BYTES = BN * HD * 2;  // 16 KB, one 128 x 64 bf16 tile
 constexpr uint32_t TMEM_COLS = 512;
 // TMEM columns of slot s start at 256 s: S (128 fp32), P (64 = 128 bf16), O (64 fp32)
 constexpr uint32_t SLOT_COLS = 256, TM_S = 0, TM_P = 128, TM_O = 192;
+constexpr uint32_t SLEEP_NS = 20000;  // longest sleep inside one barrier poll of a role thread
 
-constexpr uint32_t SLEEP_NS = 20000;
 constexpr float LOG2E = 1.4426950408889634f;
 constexpr float RESCALE_THRESHOLD = 8.0f;  // log2 units: p <= 2^8 before a rescale
 
-struct Smem {
-    uint8_t q[SLOTS][TILE_BYTES];
+// Everything of one slot's pipeline: its operand tiles (1024-byte aligned, as
+// the 128-byte swizzle needs) and barriers.
+struct __align__(1024) SlotSmem {
+    uint8_t q[TILE_BYTES];
     uint8_t k[K_STAGES][TILE_BYTES];
     uint8_t v[V_STAGES][TILE_BYTES];
-    uint64_t q_full[SLOTS], q_empty[SLOTS];
+    uint64_t q_full, q_empty;
     uint64_t k_full[K_STAGES], k_empty[K_STAGES];
     uint64_t v_full[V_STAGES], v_empty[V_STAGES];
-    uint64_t s_full[SLOTS], s_free[SLOTS], p_full[SLOTS], p_free[SLOTS], o_free[SLOTS];
+    uint64_t s_full, s_free, p_full, p_free, o_free;
     uint64_t drain;
+};
+
+struct Smem {
+    SlotSmem slot[SLOTS];
+    // Selected key tiles of each slot's current and next item as bitmaps (for
+    // the landmark masks); built at the item's start, cleared after its last P V.
+    uint32_t bm[SLOTS][2][MAX_TILES / 32];
+    uint64_t bm_ready[SLOTS][2];
     uint32_t tmem_base;
     int abort_flag;
 };
@@ -101,19 +111,6 @@ ZB_DEVINL void tmem_st16(uint32_t taddr, const uint32_t* r) {
         "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),
         "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15])
         : "memory");
-}
-
-// 2^x of one value on the FMA pipes (see f2_exp2_poly for the method).
-ZB_DEVINL float exp2_poly(float x) {
-    constexpr float kShift = 12582912.0f;  // 1.5 * 2^23
-    constexpr float kC1 = 0.695116758f, kC2 = 0.227644995f, kC3 = 0.0770670399f;
-    x = fmaxf(x, -127.f);
-    const float t = __fadd_rd(x, kShift);
-    const float f = x - (t - kShift);
-    float p = fmaf(kC3, f, kC2);
-    p = fmaf(p, f, kC1);
-    p = fmaf(p, f, 1.f);
-    return __uint_as_float(__float_as_uint(p) + (__float_as_uint(t) << 23));
 }
 
 // Shared-memory descriptors of the 128-byte-swizzle operand tiles, split in
@@ -163,41 +160,48 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
     Smem& sm = *reinterpret_cast<Smem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const int warp = warp_id();
     const int lane = lane_id();
-    const int wg = warp >> 2;
     const WaitCtx wc{p.status, &sm.abort_flag, p.timeout_ns};
     const int n = p.k + p.lm_chunks;  // steps per item
     const long long first = blockIdx.x, G = gridDim.x;
     const int cnt = first < p.n_items ? static_cast<int>((p.n_items - 1 - first) / G + 1) : 0;
-    const int rounds = (cnt + 1) / 2;
 
     // ---------------------------------------------------------- set-up ----
-    // Zero the operand buffers once: a 64-row TMA box leaves rows 64..127 of
-    // a buffer untouched, and those rows must hold finite values.
-    {
-        uint4* z = reinterpret_cast<uint4*>(&sm.q[0][0]);
-        const int n16 = (SLOTS + K_STAGES + V_STAGES) * TILE_BYTES / 16;
+    // Zero the operand tiles once: a 64-row TMA box leaves rows 64..127 of a
+    // tile untouched, and those rows must hold finite values.
+    for (int s = 0; s < SLOTS; ++s) {
+        uint4* z = reinterpret_cast<uint4*>(sm.slot[s].q);
+        const int n16 = (1 + K_STAGES + V_STAGES) * TILE_BYTES / 16;
         for (int i = threadIdx.x; i < n16; i += NUM_THREADS) z[i] = make_uint4(0, 0, 0, 0);
+    }
+    if (p.lm_chunks) {
+        uint32_t* z = &sm.bm[0][0][0];
+        for (int i = threadIdx.x; i < SLOTS * 2 * (MAX_TILES / 32); i += NUM_THREADS) z[i] = 0u;
     }
     if (threadIdx.x == 0) {
         sm.abort_flag = 0;
         for (int s = 0; s < SLOTS; ++s) {
-            mbar_init(smem_addr(&sm.q_full[s]), 1);
-            mbar_init(smem_addr(&sm.q_empty[s]), 1);
-            mbar_init(smem_addr(&sm.s_full[s]), 1);
-            mbar_init(smem_addr(&sm.s_free[s]), 128);
-            mbar_init(smem_addr(&sm.p_full[s]), 128);
-            mbar_init(smem_addr(&sm.p_free[s]), 1);
-            mbar_init(smem_addr(&sm.o_free[s]), 128);
+            mbar_init(smem_addr(&sm.bm_ready[s][0]), 128);
+            mbar_init(smem_addr(&sm.bm_ready[s][1]), 128);
         }
-        for (int i = 0; i < K_STAGES; ++i) {
-            mbar_init(smem_addr(&sm.k_full[i]), 1);
-            mbar_init(smem_addr(&sm.k_empty[i]), 1);
+        for (int s = 0; s < SLOTS; ++s) {
+            SlotSmem& b = sm.slot[s];
+            mbar_init(smem_addr(&b.q_full), 1);
+            mbar_init(smem_addr(&b.q_empty), 1);
+            for (int i = 0; i < K_STAGES; ++i) {
+                mbar_init(smem_addr(&b.k_full[i]), 1);
+                mbar_init(smem_addr(&b.k_empty[i]), 1);
+            }
+            for (int i = 0; i < V_STAGES; ++i) {
+                mbar_init(smem_addr(&b.v_full[i]), 1);
+                mbar_init(smem_addr(&b.v_empty[i]), 1);
+            }
+            mbar_init(smem_addr(&b.s_full), 1);
+            mbar_init(smem_addr(&b.s_free), 128);
+            mbar_init(smem_addr(&b.p_full), 128);
+            mbar_init(smem_addr(&b.p_free), 1);
+            mbar_init(smem_addr(&b.o_free), 128);
+            mbar_init(smem_addr(&b.drain), 1);
         }
-        for (int i = 0; i < V_STAGES; ++i) {
-            mbar_init(smem_addr(&sm.v_full[i]), 1);
-            mbar_init(smem_addr(&sm.v_empty[i]), 1);
-        }
-        mbar_init(smem_addr(&sm.drain), 1);
         fence_mbar_init();
     }
     fence_proxy_async_smem();
@@ -216,277 +220,254 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
     tc_fence_after();
     const uint32_t tmem = sm.tmem_base;
 
-    if (warp == 0 || warp == 2) {
-        if (lane == 0) {
-            // =========================== producers: warp 0 Q + K, warp 2 V ====
-            const bool is_k = warp == 0;
-            const int STAGES = is_k ? K_STAGES : V_STAGES;
-            uint64_t* full = is_k ? sm.k_full : sm.v_full;
-            uint64_t* empty = is_k ? sm.k_empty : sm.v_empty;
-            uint8_t(*buf)[TILE_BYTES] = is_k ? sm.k : sm.v;
-            const CUtensorMap* map = is_k ? &tm_k : &tm_v;
-            const CUtensorMap* lmap = is_k ? &tm_kb : &tm_vb;
-            uint32_t seq = 0;                    // loads issued into the ring
-            uint32_t issued_mask = 0, parity_mask = 0, q_issued = 0, q_parity = 0;
+    if (warp < 4) {
+        // Role warps: warp 0 / 2 produce for slot 0 / 1, warp 1 / 3 issue its
+        // MMAs.  The two slots' pipelines share nothing but the SM.
+        const int s = warp >> 1;
+        SlotSmem& b = sm.slot[s];
+        const int items = (cnt + 1 - s) / 2;  // this slot's items: it = 2 r + s
+        if ((warp & 1) == 0 && lane == 0) {
+            // ================================================ producer ====
+            // Q of each item, then per step the K and V tile of the selected
+            // key tile or landmark chunk, each into its own ring.
+            int kst = 0, vst = 0;
+            uint32_t kph = 0, vph = 0;
+            uint32_t k_issued = 0, v_issued = 0, k_par = 0, v_par = 0;
+            bool q_issued = false;
+            uint32_t q_par = 0;
             bool ok = true;
-            for (int r = 0; r < rounds && ok; ++r) {
-                const int A = (2 * r + 1 < cnt) ? 2 : 1;
-                int hs[SLOTS], is_[SLOTS];
-                const int32_t* lists[SLOTS];
-#pragma unroll
-                for (int s = 0; s < SLOTS; ++s) {
-                    if (s >= A) break;
-                    const long long item = first + static_cast<long long>(2 * r + s) * G;
-                    hs[s] = static_cast<int>(item / p.Tq);
-                    is_[s] = static_cast<int>(item % p.Tq);
-                    lists[s] = p.dense ? nullptr : p.idx + item * static_cast<long long>(p.k);
-                    if (is_k) {
-                        if (!mbar_wait(smem_addr(&sm.q_empty[s]), (r & 1) ^ 1, wc)) { ok = false; break; }
-                        const uint32_t bar = smem_addr(&sm.q_full[s]);
-                        mbar_arrive_expect_tx(bar, p.tq * HD * 2);
-                        tma_load_3d(smem_addr(sm.q[s]), &tm_q, bar, 0, is_[s] * p.tq, hs[s]);
-                        q_issued |= 1u << s;
-                        q_parity = (q_parity & ~(1u << s)) | ((r & 1u) << s);
+            for (int r = 0; r < items && ok; ++r) {
+                const long long item = first + static_cast<long long>(2 * r + s) * G;
+                const int h = static_cast<int>(item / p.Tq);
+                const int i = static_cast<int>(item % p.Tq);
+                const int32_t* list = p.dense ? nullptr : p.idx + item * static_cast<long long>(p.k);
+                if (!mbar_wait_sleep(smem_addr(&b.q_empty), (r & 1) ^ 1, wc, SLEEP_NS)) break;
+                mbar_arrive_expect_tx(smem_addr(&b.q_full), p.tq * HD * 2);
+                tma_load_3d(smem_addr(b.q), &tm_q, smem_addr(&b.q_full), 0, i * p.tq, h);
+                q_issued = true;
+                q_par = r & 1u;
+                for (int j = 0; j < n; ++j) {
+                    const int t = step_tile(p, list, j);
+                    if (!mbar_wait_sleep(smem_addr(&b.k_empty[kst]), kph ^ 1u, wc, SLEEP_NS)) { ok = false; break; }
+                    if (t >= 0) {
+                        mbar_arrive_expect_tx(smem_addr(&b.k_full[kst]), p.tk * HD * 2);
+                        tma_load_3d(smem_addr(b.k[kst]), &tm_k, smem_addr(&b.k_full[kst]), 0, t * p.tk, h);
+                    } else {
+                        mbar_arrive_expect_tx(smem_addr(&b.k_full[kst]), TILE_BYTES);
+                        tma_load_3d(smem_addr(b.k[kst]), &tm_kb, smem_addr(&b.k_full[kst]), 0, (j - p.k) * BN, h);
                     }
-                }
-                if (!ok) break;
-                for (int j = 0; j < n && ok; ++j) {
-#pragma unroll
-                    for (int s = 0; s < SLOTS; ++s) {
-                        if (s >= A) break;
-                        const int st = static_cast<int>(seq % STAGES);
-                        const uint32_t use = seq / STAGES;
-                        if (!mbar_wait(smem_addr(&empty[st]), (use & 1) ^ 1, wc)) { ok = false; break; }
-                        const uint32_t bar = smem_addr(&full[st]);
-                        const int t = step_tile(p, lists[s], j);
-                        if (t >= 0) {
-                            mbar_arrive_expect_tx(bar, p.tk * HD * 2);
-                            tma_load_3d(smem_addr(buf[st]), map, bar, 0, t * p.tk, hs[s]);
-                        } else {
-                            mbar_arrive_expect_tx(bar, TILE_BYTES);
-                            tma_load_3d(smem_addr(buf[st]), lmap, bar, 0, (j - p.k) * BN, hs[s]);
-                        }
-                        issued_mask |= 1u << st;
-                        parity_mask = (parity_mask & ~(1u << st)) | ((use & 1u) << st);
-                        ++seq;
+                    k_issued |= 1u << kst;
+                    k_par = (k_par & ~(1u << kst)) | (kph << kst);
+                    if (++kst == K_STAGES) { kst = 0; kph ^= 1u; }
+                    if (!mbar_wait_sleep(smem_addr(&b.v_empty[vst]), vph ^ 1u, wc, SLEEP_NS)) { ok = false; break; }
+                    if (t >= 0) {
+                        mbar_arrive_expect_tx(smem_addr(&b.v_full[vst]), p.tk * HD * 2);
+                        tma_load_3d(smem_addr(b.v[vst]), &tm_v, smem_addr(&b.v_full[vst]), 0, t * p.tk, h);
+                    } else {
+                        mbar_arrive_expect_tx(smem_addr(&b.v_full[vst]), TILE_BYTES);
+                        tma_load_3d(smem_addr(b.v[vst]), &tm_vb, smem_addr(&b.v_full[vst]), 0, (j - p.k) * BN, h);
                     }
+                    v_issued |= 1u << vst;
+                    v_par = (v_par & ~(1u << vst)) | (vph << vst);
+                    if (++vst == V_STAGES) { vst = 0; vph ^= 1u; }
                 }
             }
             // leave no TMA write in flight (bounded, even after an abort)
             volatile int no_abort = 0;
             const WaitCtx w2{p.status, &no_abort, p.timeout_ns};
-            for (int st = 0; st < STAGES; ++st)
-                if ((issued_mask >> st) & 1u) mbar_wait(smem_addr(&full[st]), (parity_mask >> st) & 1u, w2);
-            for (int s = 0; s < SLOTS; ++s)
-                if ((q_issued >> s) & 1u) mbar_wait(smem_addr(&sm.q_full[s]), (q_parity >> s) & 1u, w2);
-        }
-        __syncwarp();
-    } else if (warp == 1) {
-        // ================================================= MMA issuer ====
-        constexpr uint32_t IDESC_QK = idesc_bf16(BM, BN, 0, 0);  // Q K-major, K K-major
-        constexpr uint32_t IDESC_PV = idesc_bf16(BM, HD, 0, 1);  // P (TMEM), V MN-major
-        if (lane == 0) {
-            const uint32_t q_lo0 = desc_lo(smem_addr(sm.q[0]), 16);
-            const uint32_t k_lo0 = desc_lo(smem_addr(sm.k[0]), 16);
-            const uint32_t v_lo0 = desc_lo(smem_addr(sm.v[0]), 0);
+            for (int st = 0; st < K_STAGES; ++st)
+                if ((k_issued >> st) & 1u) mbar_wait(smem_addr(&b.k_full[st]), (k_par >> st) & 1u, w2);
+            for (int st = 0; st < V_STAGES; ++st)
+                if ((v_issued >> st) & 1u) mbar_wait(smem_addr(&b.v_full[st]), (v_par >> st) & 1u, w2);
+            if (q_issued) mbar_wait(smem_addr(&b.q_full), q_par, w2);
+        } else if ((warp & 1) == 1 && lane == 0) {
+            // ============================================== MMA issuer ====
+            // Per step: S = Q K^T (as soon as the softmax has read the previous
+            // S), then O += P V with P read from TMEM (tcgen05 "TS" form).
+            constexpr uint32_t IDESC_QK = idesc_bf16(BM, BN, 0, 0);  // Q K-major, K K-major
+            constexpr uint32_t IDESC_PV = idesc_bf16(BM, HD, 0, 1);  // P (TMEM), V MN-major
+            const uint32_t q_lo = desc_lo(smem_addr(b.q), 16);
+            const uint32_t k_lo0 = desc_lo(smem_addr(b.k[0]), 16);
+            const uint32_t v_lo0 = desc_lo(smem_addr(b.v[0]), 0);
             constexpr uint32_t TILE_LO = TILE_BYTES >> 4;
-            int k_next = 0, v_next = 0;
-            uint32_t k_ph = 0, v_ph = 0;
+            const uint32_t s_tmem = tmem + s * SLOT_COLS + TM_S;
+            const uint32_t p_tmem = tmem + s * SLOT_COLS + TM_P;
+            const uint32_t o_tmem = tmem + s * SLOT_COLS + TM_O;
+            int kst = 0, vst = 0;
+            uint32_t kph = 0, vph = 0;
+            long long g = 0;  // steps of this slot so far
             bool ok = true;
-            auto issue_qk = [&](int s, long long g) -> bool {
-                const int ks = k_next;
-                if (!mbar_wait_sleep(smem_addr(&sm.k_full[ks]), k_ph, wc, SLEEP_NS)) return false;
-                if (++k_next == K_STAGES) { k_next = 0; k_ph ^= 1u; }
-                if (!mbar_wait_sleep(smem_addr(&sm.s_free[s]), static_cast<uint32_t>((g & 1) ^ 1), wc, SLEEP_NS)) return false;
+            auto issue_qk = [&]() -> bool {
+                if (!mbar_wait_sleep(smem_addr(&b.k_full[kst]), kph, wc, SLEEP_NS)) return false;
+                if (!mbar_wait_sleep(smem_addr(&b.s_free), static_cast<uint32_t>((g & 1) ^ 1), wc, SLEEP_NS)) return false;
                 tc_fence_after();
-                const uint32_t qa = q_lo0 + s * TILE_LO, kb = k_lo0 + ks * TILE_LO;
-                const uint32_t d_tmem = tmem + s * SLOT_COLS + TM_S;
+                const uint32_t kb = k_lo0 + kst * TILE_LO;
 #pragma unroll
-                for (int kk = 0; kk < HD / 16; ++kk) mma_ss(d_tmem, qa + kk * 2, kb + kk * 2, IDESC_QK, kk > 0 ? 1u : 0u);
-                umma_commit(smem_addr(&sm.s_full[s]));
-                umma_commit(smem_addr(&sm.k_empty[ks]));
+                for (int kk = 0; kk < HD / 16; ++kk) mma_ss(s_tmem, q_lo + kk * 2, kb + kk * 2, IDESC_QK, kk > 0 ? 1u : 0u);
+                umma_commit(smem_addr(&b.s_full));
+                umma_commit(smem_addr(&b.k_empty[kst]));
+                if (++kst == K_STAGES) { kst = 0; kph ^= 1u; }
                 return true;
             };
-            for (int r = 0; r < rounds && ok; ++r) {
-                const int A = (2 * r + 1 < cnt) ? 2 : 1;
-                for (int s = 0; s < A && ok; ++s)
-                    if (!mbar_wait_sleep(smem_addr(&sm.q_full[s]), r & 1, wc, SLEEP_NS)) ok = false;
-                if (!ok) break;
+            for (int r = 0; r < items && ok; ++r) {
+                if (!mbar_wait_sleep(smem_addr(&b.q_full), r & 1, wc, SLEEP_NS)) break;
                 tc_fence_after();
-                for (int s = 0; s < A && ok; ++s)
-                    if (!issue_qk(s, static_cast<long long>(r) * n)) ok = false;
-                for (int j = 0; j < n && ok; ++j) {
-                    for (int s = 0; s < A; ++s) {
-                        const long long g = static_cast<long long>(r) * n + j;
-                        if (j + 1 < n) {
-                            if (!issue_qk(s, g + 1)) { ok = false; break; }
-                        } else {
-                            umma_commit(smem_addr(&sm.q_empty[s]));
-                        }
-                        if (!mbar_wait_sleep(smem_addr(&sm.p_full[s]), static_cast<uint32_t>(g & 1), wc, SLEEP_NS)) { ok = false; break; }
-                        if (j == 0) {
-                            if (!mbar_wait_sleep(smem_addr(&sm.o_free[s]), (r & 1) ^ 1, wc, SLEEP_NS)) { ok = false; break; }
-                        }
-                        const int vs = v_next;
-                        if (!mbar_wait_sleep(smem_addr(&sm.v_full[vs]), v_ph, wc, SLEEP_NS)) { ok = false; break; }
-                        if (++v_next == V_STAGES) { v_next = 0; v_ph ^= 1u; }
-                        tc_fence_after();
-                        const uint32_t vb = v_lo0 + vs * TILE_LO;
-                        const uint32_t p_tmem = tmem + s * SLOT_COLS + TM_P;
-                        const uint32_t o_tmem = tmem + s * SLOT_COLS + TM_O;
-#pragma unroll
-                        for (int kk = 0; kk < BN / 16; ++kk)
-                            mma_ts(o_tmem, p_tmem + kk * 8, vb + kk * 128, IDESC_PV, (j > 0 || kk > 0) ? 1u : 0u);
-                        umma_commit(smem_addr(&sm.v_empty[vs]));
-                        umma_commit(smem_addr(&sm.p_free[s]));
+                if (!issue_qk()) break;  // S of step 0 (g is its step number)
+                for (int j = 0; j < n; ++j, ++g) {
+                    if (j + 1 < n) {
+                        ++g;
+                        const bool q_ok = issue_qk();
+                        --g;
+                        if (!q_ok) { ok = false; break; }
+                    } else {
+                        umma_commit(smem_addr(&b.q_empty));
                     }
+                    if (!mbar_wait_sleep(smem_addr(&b.p_full), static_cast<uint32_t>(g & 1), wc, SLEEP_NS)) { ok = false; break; }
+                    if (j == 0) {
+                        if (!mbar_wait_sleep(smem_addr(&b.o_free), (r & 1) ^ 1, wc, SLEEP_NS)) { ok = false; break; }
+                    }
+                    if (!mbar_wait_sleep(smem_addr(&b.v_full[vst]), vph, wc, SLEEP_NS)) { ok = false; break; }
+                    tc_fence_after();
+                    const uint32_t vb = v_lo0 + vst * TILE_LO;
+#pragma unroll
+                    for (int kk = 0; kk < BN / 16; ++kk)
+                        mma_ts(o_tmem, p_tmem + kk * 8, vb + kk * 128, IDESC_PV, (j > 0 || kk > 0) ? 1u : 0u);
+                    umma_commit(smem_addr(&b.v_empty[vst]));
+                    umma_commit(smem_addr(&b.p_free));
+                    if (++vst == V_STAGES) { vst = 0; vph ^= 1u; }
                 }
             }
-            // no tcgen05.mma may still run when TMEM is released
-            umma_commit(smem_addr(&sm.drain));
+            // no tcgen05.mma of this thread may still run when TMEM is released
+            umma_commit(smem_addr(&b.drain));
             volatile int no_abort = 0;
             const WaitCtx w2{p.status, &no_abort, p.timeout_ns};
-            mbar_wait(smem_addr(&sm.drain), 0, w2);
+            mbar_wait(smem_addr(&b.drain), 0, w2);
         }
         __syncwarp();
-    } else if (warp == 3) {
-        // ============================ index-list check (off the critical path) ====
-        // Every list must be in range and strictly ascending; a bad one sets
-        // ZB_ERR_INDEX (the kernel itself clamps indices and never reads out of
-        // bounds).  32 entries per step, one per lane.
-        if (!p.dense) {
-            for (int it = 0; it < cnt; ++it) {
-                const long long item = first + static_cast<long long>(it) * G;
-                const int32_t* list = p.idx + item * static_cast<long long>(p.k);
-                int bad = 0;
-                for (int q0 = 0; q0 < p.k; q0 += 32) {
-                    const int q = q0 + lane;
-                    const int t = q < p.k ? __ldg(list + q) : 0;
-                    int prev = __shfl_up_sync(0xffffffffu, t, 1);
-                    if (lane == 0) prev = q0 == 0 ? -1 : __ldg(list + q0 - 1);
-                    if (q < p.k && (t < 0 || t >= p.Tk || t <= prev)) bad = 1;
-                }
-                if (__any_sync(0xffffffffu, bad)) {
-                    if (lane == 0) flag_status(p.status, ZB_ERR_INDEX);
-                    break;
-                }
-            }
-        }
-    } else if (wg >= 1) {
+    } else {
         // ===================================== softmax warpgroup of a slot ====
-        const int s = wg - 1;
+        const int s = (warp >> 2) - 1;
+        SlotSmem& b = sm.slot[s];
         const int quarter = warp & 3;            // TMEM lane quarter this warp may access
         const int row = quarter * 32 + lane;     // query row within the tile
         const uint32_t lane_addr = static_cast<uint32_t>(quarter * 32) << 16;
         const uint32_t tm_s = tmem + lane_addr + s * SLOT_COLS + TM_S;
         const uint32_t tm_p = tmem + lane_addr + s * SLOT_COLS + TM_P;
         const uint32_t tm_o = tmem + lane_addr + s * SLOT_COLS + TM_O;
+        const uint64_t c2 = f2_pack(p.scale_log2, p.scale_log2);
+        const int items = (cnt + 1 - s) / 2;
+        uint32_t ph = 0;  // parity of this slot's step counter
         bool ok = true;
-        for (int r = 0; r < rounds && ok; ++r) {
-            const int it = 2 * r + s;
-            if (it >= cnt) break;
-            const long long item = first + static_cast<long long>(it) * G;
+        for (int r = 0; r < items && ok; ++r) {
+            const long long item = first + static_cast<long long>(2 * r + s) * G;
             const int h = static_cast<int>(item / p.Tq);
             const int i = static_cast<int>(item % p.Tq);
             const int32_t* list = p.dense ? nullptr : p.idx + item * static_cast<long long>(p.k);
+            // Index-list check, 1/128 of the list per thread: in range and
+            // strictly ascending, else ZB_ERR_INDEX (the producers clamp, so a
+            // bad list never leads to an out-of-bounds read).
+            // With landmarks, the same pass marks the selected tiles in this
+            // item's bitmap (indices clamped into range).
+            uint32_t* bm = sm.bm[s][r & 1];
+            if (list) {
+                int bad = 0;
+                for (int q = row; q < p.k; q += BM) {
+                    const int t = __ldg(list + q);
+                    const int prev = q > 0 ? __ldg(list + q - 1) : -1;
+                    bad |= (t < 0) | (t >= p.Tk) | (t <= prev);
+                    if (p.lm_chunks) {
+                        const int tc = t < 0 ? 0 : (t >= p.Tk ? p.Tk - 1 : t);
+                        atomicOr(&bm[tc >> 5], 1u << (tc & 31));
+                    }
+                }
+                if (bad) flag_status(p.status, ZB_ERR_INDEX);
+            }
+            if (p.lm_chunks) mbar_arrive(smem_addr(&sm.bm_ready[s][r & 1]));
             // valid columns of the last selected tile (only the last key tile is ragged)
             int last_valid = p.tk;
             if (p.k > 0) {
                 const int jl = p.dense ? p.Tk - 1 : __ldg(list + p.k - 1);
                 if (jl == p.Tk - 1) last_valid = p.n_last;
             }
-            int ip = 0;           // walk over the sorted index list for landmark masks
             float m = -INFINITY;  // running max of the log2-domain logits (lazy)
             float l = 0.f;        // running sum of 2^(x - m)
-            long long g = static_cast<long long>(r) * n;
-            for (int j = 0; j < n; ++j, ++g) {
-                if (!mbar_wait(smem_addr(&sm.s_full[s]), static_cast<uint32_t>(g & 1), wc)) { ok = false; break; }
+            for (int j = 0; j < n; ++j, ph ^= 1u) {
+                if (!mbar_wait(smem_addr(&b.s_full), ph, wc)) { ok = false; break; }
                 tc_fence_after();
-                const bool is_lm = j >= p.k;
-                // Per-column treatment of S: selected tiles mask columns past the
-                // tile's length; landmark chunks become s * scale + log2(n_j), or
-                // -inf for selected / out-of-range tiles (the selected ones come
-                // from a walk over the sorted index list, kept in 4 mask words).
-                const int valid = is_lm ? BN : ((j == p.k - 1) ? last_valid : p.tk);
-                const int j0 = (j - p.k) * BN;
-                uint32_t s0 = 0u, s1 = 0u, s2 = 0u, s3 = 0u;
-                if (is_lm) {
-                    while (ip < p.k) {
-                        const int t = __ldg(list + ip);
-                        if (t >= j0 + BN) break;
-                        if (t >= j0) {
-                            const int c = t - j0;
-                            const uint32_t bit = 1u << (c & 31);
-                            s0 |= (c >> 5) == 0 ? bit : 0u;
-                            s1 |= (c >> 5) == 1 ? bit : 0u;
-                            s2 |= (c >> 5) == 2 ? bit : 0u;
-                            s3 |= (c >> 5) == 3 ? bit : 0u;
-                        }
-                        ++ip;
-                    }
-                    const int past = p.Tk - j0;  // columns >= past are beyond the last tile
-                    if (past < 32) s0 |= past <= 0 ? 0xFFFFFFFFu : (0xFFFFFFFFu << past);
-                    if (past < 64) s1 |= past <= 32 ? 0xFFFFFFFFu : (0xFFFFFFFFu << (past - 32));
-                    if (past < 96) s2 |= past <= 64 ? 0xFFFFFFFFu : (0xFFFFFFFFu << (past - 64));
-                    if (past < 128) s3 |= past <= 96 ? 0xFFFFFFFFu : (0xFFFFFFFFu << (past - 96));
+                float x[BN];
+                {
+                    uint32_t raw[BN];
+#pragma unroll
+                    for (int c = 0; c < BN / 32; ++c) tmem_ld32(tm_s + c * 32, sub32(raw, c * 32));
+#pragma unroll
+                    for (int c = 0; c < BN / 32; ++c) tmem_wait_ld_dep(sub32(raw, c * 32));
+#pragma unroll
+                    for (int e = 0; e < BN; ++e) x[e] = __uint_as_float(raw[e]);
                 }
-                // Per-column treatment of chunk c of S (raw words r): selected tiles
-                // mask columns past the tile's length; landmark chunks become
-                // s * scale + log2(n_j), or -inf for selected / out-of-range tiles.
-                auto treat = [&](float (&y)[32], const uint32_t (&r)[32], int c) {
-                    if (is_lm) {
-                        const uint32_t bits = c == 0 ? s0 : (c == 1 ? s1 : (c == 2 ? s2 : s3));
-                        const int lastc = p.Tk - 1 - j0 - c * 32;  // column of the ragged last tile
+                tc_fence_before();
+                mbar_arrive(smem_addr(&b.s_free));  // S is in registers: the next Q K^T may overwrite it
+                const bool is_lm = j >= p.k;
+                if (!is_lm) {
+                    // selected tile: mask the columns past the tile's length
+                    const int valid = (j == p.k - 1) ? last_valid : p.tk;
+                    if (valid < BN) {
 #pragma unroll
-                        for (int e = 0; e < 32; ++e) {
-                            float bias = (e == lastc) ? p.log2_last : p.log2_tk;
-                            if ((bits >> e) & 1u) bias = -INFINITY;
-                            y[e] = fmaf(__uint_as_float(r[e]), p.scale_log2, bias);
-                        }
-                    } else {
-                        const int vc = valid - c * 32;  // valid columns in this chunk
-#pragma unroll
-                        for (int e = 0; e < 32; ++e) y[e] = __uint_as_float(r[e]);
-                        if (vc < 32) {  // only a ragged last tile (or a 64-row tile) needs the mask
-#pragma unroll
-                            for (int e = 0; e < 32; ++e)
-                                if (e >= vc) y[e] = -INFINITY;
-                        }
+                        for (int e = 0; e < BN; ++e)
+                            if (e >= valid) x[e] = -INFINITY;
                     }
-                };
-                // one 32-column chunk c of S into y[] (treated)
-                auto load_chunk = [&](float (&y)[32], int c) {
-                    uint32_t r[32];
-                    tmem_ld32(tm_s + c * 32, r);
-                    tmem_wait_ld_dep(r);
-                    treat(y, r, c);
-                };
-                // chunks c and c + 1 with one TMEM wait
-                auto load_chunk2 = [&](float (&y)[32], float (&z)[32], int c) {
-                    uint32_t r[32], r2[32];
-                    tmem_ld32(tm_s + c * 32, r);
-                    tmem_ld32(tm_s + c * 32 + 32, r2);
-                    tmem_wait_ld_dep(r);
-                    tmem_wait_ld_dep(r2);
-                    treat(y, r, c);
-                    treat(z, r2, c + 1);
-                };
-                // ---- pass 1: row max (two chunks per TMEM wait)
-                float mx = -INFINITY;
+                } else {
+                    // landmark chunk: x = s * scale + log2(n_j), or -inf for
+                    // selected tiles (from the item's bitmap) and for columns
+                    // past the last tile
+                    const int j0 = (j - p.k) * BN;
+                    if (j == p.k) {  // first landmark step: every thread's bits are in
+                        if (!mbar_wait(smem_addr(&sm.bm_ready[s][r & 1]), (r >> 1) & 1, wc)) { ok = false; break; }
+                    }
 #pragma unroll 1
-                for (int c = 0; c < BN / 32; c += 2) {
-                    float y[32], z[32];
-                    load_chunk2(y, z, c);
-                    float g0 = fmax3(y[0], y[1], y[2]), g1 = fmax3(z[0], z[1], z[2]);
-                    float g2 = fmax3(y[3], y[4], y[5]), g3 = fmax3(z[3], z[4], z[5]);
-#pragma unroll
-                    for (int e = 6; e < 30; e += 2) {
-                        g0 = fmax3(g0, y[e], y[e + 1]);
-                        g1 = fmax3(g1, z[e], z[e + 1]);
+                    for (int w = 0; w < BN / 32; ++w) {
+                        const int jw = j0 + w * 32;
+                        uint32_t bits = jw < p.Tk ? bm[jw >> 5] : 0u;
+                        const int keep = p.Tk - jw;  // columns >= keep are beyond the last tile
+                        if (keep < 32) bits |= keep <= 0 ? 0xFFFFFFFFu : (0xFFFFFFFFu << keep);
+                        const int lastc = p.Tk - 1 - jw;  // column of the ragged last tile
+                        // bias of this 32-column word, applied under a switch on w so
+                        // that x stays in registers
+                        switch (w) {
+#define ZB_LM_WORD(W)                                                                      \
+    case W:                                                                                \
+        _Pragma("unroll") for (int e = 0; e < 32; e += 2) {                                \
+            const float b0 = ((bits >> e) & 1u) ? -INFINITY                                \
+                                                : (e == lastc ? p.log2_last : p.log2_tk);  \
+            const float b1 = ((bits >> (e + 1)) & 1u) ? -INFINITY                          \
+                                                      : (e + 1 == lastc ? p.log2_last : p.log2_tk); \
+            float v0, v1;                                                                  \
+            f2_unpack(f2_fma(f2_pack(x[W * 32 + e], x[W * 32 + e + 1]), c2,                \
+                             f2_pack(b0, b1)), v0, v1);                                    \
+            x[W * 32 + e] = v0;                                                            \
+            x[W * 32 + e + 1] = v1;                                                        \
+        }                                                                                  \
+        break;
+                            ZB_LM_WORD(0)
+                            ZB_LM_WORD(1)
+                            ZB_LM_WORD(2)
+                            ZB_LM_WORD(3)
+#undef ZB_LM_WORD
+                        }
                     }
-                    g2 = fmax3(g2, y[30], y[31]);
-                    g3 = fmax3(g3, z[30], z[31]);
-                    mx = fmaxf(mx, fmaxf(fmax3(g0, g1, g2), g3));
+                }
+                // ---- row max: a tree of 3-input max (selected tiles: of the
+                // raw scores, scaled afterwards, as scale > 0)
+                float mx;
+                {
+                    float gq[8];
+#pragma unroll
+                    for (int q = 0; q < 8; ++q) {
+                        float t = fmax3(x[16 * q], x[16 * q + 1], x[16 * q + 2]);
+#pragma unroll
+                        for (int e = 3; e < 15; e += 2) t = fmax3(t, x[16 * q + e], x[16 * q + e + 1]);
+                        gq[q] = fmaxf(t, x[16 * q + 15]);
+                    }
+                    mx = fmax3(fmax3(gq[0], gq[1], gq[2]), fmax3(gq[3], gq[4], gq[5]), fmaxf(gq[6], gq[7]));
                 }
                 if (!is_lm) mx *= p.scale_log2;
                 // ---- lazy rescale: keep the old max unless the new one exceeds it by > 8
@@ -499,10 +480,11 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                     l *= alpha;
                 }
                 const float nm = (m == -INFINITY) ? 0.f : -m;
-                const float cm = is_lm ? 1.f : p.scale_log2;  // landmark logits are already scaled
-                // P of this slot is free once P V of the previous step is done;
-                // O then holds every earlier step and can be rescaled
-                if (!mbar_wait(smem_addr(&sm.p_free[s]), static_cast<uint32_t>((g & 1) ^ 1), wc)) { ok = false; break; }
+                const uint64_t nm2 = f2_pack(nm, nm);
+                const uint64_t cm2 = is_lm ? f2_pack(1.f, 1.f) : c2;  // landmark logits are already scaled
+                // P is free once P V of the previous step is done; O then holds
+                // every earlier step and can be rescaled
+                if (!mbar_wait(smem_addr(&b.p_free), ph ^ 1u, wc)) { ok = false; break; }
                 tc_fence_after();
                 if (rescale && j > 0) {
 #pragma unroll 1
@@ -516,30 +498,18 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                         tmem_wait_st();
                     }
                 }
-                // ---- pass 2: p = 2^(x * cm - m) per chunk (1 of 4 pairs on the FMA
-                // pipes, the rest on MUFU), packed fp32x2, bf16 pairs straight to TMEM
-                const uint64_t cm2 = f2_pack(cm, cm), nm2 = f2_pack(nm, nm);
+                // ---- p = 2^(x * scale - m): packed fp32x2 arithmetic, exponentials
+                // on MUFU, two partial sums, bf16 pairs to TMEM per 32 columns
                 uint64_t acc0 = 0ull, acc1 = 0ull;
-#pragma unroll 1
+#pragma unroll
                 for (int c = 0; c < BN / 32; ++c) {
-                    float y[32];
-                    load_chunk(y, c);
-                    if (c == BN / 32 - 1) {
-                        tc_fence_before();
-                        mbar_arrive(smem_addr(&sm.s_free[s]));  // S fully read: the next Q K^T may overwrite it
-                    }
                     uint32_t pk[16];
 #pragma unroll
                     for (int q = 0; q < 16; ++q) {
-                        const uint64_t xs = f2_fma(f2_pack(y[2 * q], y[2 * q + 1]), cm2, nm2);
-                        uint64_t pv;
-                        if ((q & 3) == 1) {
-                            pv = f2_exp2_poly(xs);
-                        } else {
-                            float a0, a1;
-                            f2_unpack(xs, a0, a1);
-                            pv = f2_pack(ex2(a0), ex2(a1));
-                        }
+                        const uint64_t xs = f2_fma(f2_pack(x[c * 32 + 2 * q], x[c * 32 + 2 * q + 1]), cm2, nm2);
+                        float a0, a1;
+                        f2_unpack(xs, a0, a1);
+                        const uint64_t pv = f2_pack(ex2(a0), ex2(a1));
                         if (q & 1) acc1 = f2_add(acc1, pv); else acc0 = f2_add(acc0, pv);
                         float p0, p1;
                         f2_unpack(pv, p0, p1);
@@ -547,18 +517,28 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                     }
                     tmem_st16(tm_p + c * 16, pk);
                 }
-                float rs0, rs1;
-                f2_unpack(f2_add(acc0, acc1), rs0, rs1);
-                l += rs0 + rs1;
+                {
+                    float s0, s1;
+                    f2_unpack(f2_add(acc0, acc1), s0, s1);
+                    l += s0 + s1;
+                }
                 tmem_wait_st();
                 tc_fence_before();
-                mbar_arrive(smem_addr(&sm.p_full[s]));
+                mbar_arrive(smem_addr(&b.p_full));
             }
             if (!ok) break;
             // ------------------------------------------------ epilogue ----
-            const long long gl = g - 1;
-            if (!mbar_wait(smem_addr(&sm.p_free[s]), static_cast<uint32_t>(gl & 1), wc)) { ok = false; break; }
+            // P V of the item's last step (parity ph ^ 1) has completed, so every
+            // thread of the slot is past its landmark steps: clear this item's bits
+            if (!mbar_wait(smem_addr(&b.p_free), ph ^ 1u, wc)) { ok = false; break; }
             tc_fence_after();
+            if (list && p.lm_chunks) {
+                for (int q = row; q < p.k; q += BM) {
+                    const int t = __ldg(list + q);
+                    const int tc = t < 0 ? 0 : (t >= p.Tk ? p.Tk - 1 : t);
+                    atomicAnd(&bm[tc >> 5], ~(1u << (tc & 31)));
+                }
+            }
             float o[HD];
             {
                 uint32_t ro[HD];
@@ -570,7 +550,7 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                 for (int e = 0; e < HD; ++e) o[e] = __uint_as_float(ro[e]);
             }
             tc_fence_before();
-            mbar_arrive(smem_addr(&sm.o_free[s]));
+            mbar_arrive(smem_addr(&b.o_free));
             const long long qrow = static_cast<long long>(i) * p.tq + row;
             if (row < p.tq && qrow < p.n_q) {
                 const float inv = 1.f / l;
