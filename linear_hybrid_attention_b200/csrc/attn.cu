@@ -13,22 +13,22 @@
 // Kernel design: one persistent CTA per SM, 384 threads, two work items in
 // flight ("slots").  A work item is one (head, query tile); the CTA's items
 // alternate between the slots.  With d = 64 the softmax (16,384 exponentials
-// per 128 x 128 tile) costs more than the tile's two MMAs, so both slots'
-// softmax warpgroups run at the same time while one warp keeps the tensor core
-// fed for both.
-//   warp 0      Q and K producer (TMA): Q of each slot's item, then K tiles of
-//               the selected key tiles / landmark chunks into a K ring.
-//   warp 2      V producer (TMA): the matching V tiles into a separate V ring
-//               (K is released after Q K^T, V only after P V).
-//   warp 1      MMA issuer (one lane): per slot S = Q K^T into the slot's TMEM
-//               S, then O += P V with P read from TMEM (tcgen05 "TS" form).
-//   warp 3      checks every index list (range, strictly ascending).
-//   warps 4..7  softmax of slot 0, warps 8..11 softmax of slot 1: one thread
-//               per query row; log2-domain online softmax with lazy
-//               rescaling of O, P (bf16) to TMEM, epilogue O / l.
-// A softmax thread reads its S row from TMEM twice in 32-column chunks (once
-// for the row max, once for the exponentials): compact code (the instruction
-// cache is shared by 12 warps running different roles) and few registers.
+// per 128 x 128 tile) costs more than the tile's two MMAs, so two softmax
+// warpgroups run at the same time, and each slot is a pipeline of its own
+// (producer, MMA issuer, softmax) that shares nothing with the other slot but
+// the SM.
+//   warps 0 / 2  producer of slot 0 / 1 (one lane, TMA): Q of each item, then
+//                per step the K and V tile of the selected key tile or
+//                landmark chunk, K and V each in a ring of their own.
+//   warps 1 / 3  MMA issuer of slot 0 / 1 (one lane): S = Q K^T into the
+//                slot's TMEM S as soon as the softmax has read the previous S,
+//                then O += P V with P read from TMEM (tcgen05 "TS" form).
+//   warps 4..7   softmax of slot 0, warps 8..11 softmax of slot 1: one thread
+//                per query row reads its whole S row into registers (S is then
+//                free for the next Q K^T), log2-domain online softmax with
+//                lazy rescaling of O, P (bf16) to TMEM, epilogue O / l.  They
+//                also check the index lists and keep the slot's bitmap of
+//                selected tiles from which the landmark masks are read.
 // Items are dealt round-robin over CTAs, so CTAs running at the same time work
 // on neighbouring query tiles of one head and sweep its K/V in ascending order
 // together (L2 reuse).
