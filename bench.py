@@ -50,6 +50,31 @@ def measured_peaks():
     return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
 
 
+# ---------------------------------------------------------------- traffic ----
+def recorded_traffic(workload: str):
+    """DRAM bytes per launch of the sparse kernel from the committed ncu summary
+    (profiles/sparse_attn_<workload>_dram.md), or None when there is none or the
+    kernel source changed since it was taken (its sha256 is recorded there)."""
+    import hashlib
+    path = os.path.join(ROOT, "profiles", f"sparse_attn_{workload}_dram.md")
+    src = os.path.join(ROOT, "linear_hybrid_attention_b200", "csrc", "attn.cu")
+    if not os.path.exists(path) or not os.path.exists(src):
+        return None, "no ncu DRAM capture recorded for this workload"
+    fields = {}
+    with open(path) as f:
+        for line in f:
+            if ":" in line and line.startswith("- "):
+                k, v = line[2:].split(":", 1)
+                fields[k.strip()] = v.strip().strip("`")
+    sha = hashlib.sha256(open(src, "rb").read()).hexdigest()
+    if fields.get("attn.cu sha256") != sha:
+        return None, "kernel changed since the recorded ncu DRAM capture"
+    try:
+        return float(fields["dram bytes per launch"]), path
+    except (KeyError, ValueError):
+        return None, "ncu DRAM summary unreadable"
+
+
 # ----------------------------------------------------------------- clocks ----
 class ClockSampler:
     """nvidia-smi sampling of SM clock and throttle reasons during the timed region."""
@@ -223,6 +248,7 @@ def main():
     ap.add_argument("--keep-frac", type=float, default=None, help="override the kept fraction of key tiles")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
+    ap.add_argument("--no-dense-ref", action="store_true", help="skip the dense-attention comparator")
     ap.add_argument("--profile", action="store_true", help="short run for profilers: no JSON extras")
     args = ap.parse_args()
 
@@ -329,9 +355,12 @@ def main():
     lin_state_bytes = 2 * tensor_bytes               # reads K, V
     lin_apply_bytes = 2 * tensor_bytes               # reads Q, writes O
     hbm = peaks["hbm_gbs"]
+    traffic, traffic_src = recorded_traffic(w.name)
     roofline = {"kernel": "zb_tile_sparse_attn", "bound": "tensor", "achieved": sparse_tf,
                 "peak": peaks["bf16_tflops_sustained"], "unit": "TFLOP/s",
-                "frac": sparse_tf / peaks["bf16_tflops_sustained"], "traffic": None,
+                "frac": sparse_tf / peaks["bf16_tflops_sustained"], "traffic": traffic,
+                "traffic_unit": "bytes per launch (dram__bytes_read.sum + dram__bytes_write.sum)",
+                "traffic_source": traffic_src,
                 "peak_kind": f"bf16 sustained ({peaks['source']}); kernel runs inside a long step",
                 "frac_of_burst": sparse_tf / peaks["bf16_tflops"],
                 "algorithmic": f"{flops:.4e} FLOP per launch = 4*d*sum n_i*n_j over kept (query tile, key tile) pairs"}
@@ -354,6 +383,35 @@ def main():
     stage_ms = {"sparse_stage": (kt["landmark"] + kt["topk"] + kt["sparse_attn"]) * 1e3,
                 "linear_stage": (kt["linear_state"] + kt["calib_dense"] + kt["calib_rest"] + kt["linear_apply"]) * 1e3,
                 "linear_stage_without_fit": (kt["linear_state"] + kt["linear_apply"]) * 1e3}
+    # the pages' headline allocation 0.7L: tokens / (0.7 t_linear + 0.3 t_sparse)
+    t_lin = stage_ms["linear_stage"] / 1e3
+    t_sp = stage_ms["sparse_stage"] / 1e3
+    hybrid_07 = w.n_tokens / (0.7 * t_lin + 0.3 * t_sp) / 1e6 * world
+
+    # --------------------------------------------------- dense comparator ----
+    # Dense softmax attention at the same shape, timed on one head (the heads
+    # are independent launches of identical cost) and scaled to all heads.
+    dense_ref = None
+    if not args.no_dense_ref:
+        Od = torch.empty((1, w.n_tokens, w.head_dim), dtype=torch.bfloat16, device=dev)
+        q1, k1, v1 = Q[:1], K[:1], V[:1]
+        zb.zb_dense_attn(q1, k1, v1, layer.scale, out=Od)
+        torch.cuda.synchronize()
+        a = torch.cuda.Event(enable_timing=True)
+        bb = torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        zb.zb_dense_attn(q1, k1, v1, layer.scale, out=Od)
+        bb.record(stream)
+        torch.cuda.synchronize()
+        zb.zb_last_device_status()
+        t_head = a.elapsed_time(bb) / 1e3
+        dense_flops = 4.0 * w.n_tokens * w.n_tokens * w.head_dim
+        dense_ref = {"ms_all_heads": t_head * w.heads * 1e3, "ms_one_head": t_head * 1e3,
+                     "tflops": dense_flops / t_head / 1e12,
+                     "frac_of_sustained": dense_flops / t_head / 1e12 / peaks["bf16_tflops_sustained"],
+                     "sparse_stage_speedup": t_head * w.heads / t_sp,
+                     "note": "zb_dense_attn on head 0 at full length, scaled by the head count"}
+        del Od
 
     # ------------------------------------------------------------ e2e ----
     e2e = None
@@ -403,6 +461,7 @@ def main():
                 "config": config_dict(w), "e2e": e2e, "gpu_launches": layer.launches_per_step * args.steps,
                 "roofline": roofline, "kernel_roofline": kernel_rooflines, "stage_ms": stage_ms,
                 "kernel_ms": {n: v * 1e3 for n, v in kt.items()}, "clocks": clk, "cpu_baseline": cpu,
+                "hybrid_0.7L_mtokens_s": hybrid_07, "dense_reference": dense_ref,
                 "peaks": peaks}
         print(json.dumps(line), flush=True)
     if world > 1:

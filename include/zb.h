@@ -185,6 +185,24 @@ zb_status zb_linear_apply(const uint16_t* Q, int32_t heads, int64_t n_q,
                           void* stream);
 
 /*
+ * The whole linear-attention stage in one call: zb_linear_state followed by
+ * zb_linear_apply (bf16 output) on the same tokens, the state S, z kept in the
+ * workspace (Abstract: linear attention for the tolerant stages; section "How
+ * Zebra3D works": its output corrected by the per-head affine map).
+ *   in : Q, K, V bf16 [H][N][d];  A fp32 [H][d][d] or NULL (identity);
+ *        b fp32 [H][d] or NULL (zero);  ws of >= zb_linear_attn_workspace_bytes()
+ *        bytes, 16-byte aligned, owned by the caller
+ *   out: O bf16 [H][N][d]
+ * Two kernel launches for the state, one for the output, all on `stream`.
+ * Errors: ZB_ERR_NULL, ZB_ERR_SHAPE, ZB_ERR_ALIGN, ZB_ERR_UNSUPPORTED,
+ * ZB_ERR_WORKSPACE, ZB_ERR_CUDA.
+ */
+size_t zb_linear_attn_workspace_bytes(int32_t heads, int64_t n_tokens, int32_t head_dim);
+zb_status zb_linear_attn(const uint16_t* Q, const uint16_t* K, const uint16_t* V, int32_t heads,
+                         int64_t n_tokens, int32_t head_dim, const float* A, const float* b,
+                         uint16_t* O, void* ws, size_t ws_bytes, void* stream);
+
+/*
  * Closed-form affine fit (Abstract: closed-form affine fitting makes the
  * conversion training-free; Table 3 (a) of "Zebra3D: Efficient Hybrid
  * Foundation Models ..." compares no fit with fitted variants): per head, the

@@ -26,7 +26,7 @@ from . import _lib
 
 __all__ = [
     "ZbError", "Landmarks", "zb_abi_version", "zb_landmark_build", "zb_tile_score_topk",
-    "zb_tile_sparse_attn", "zb_dense_attn", "zb_linear_state", "zb_linear_apply",
+    "zb_tile_sparse_attn", "zb_dense_attn", "zb_linear_state", "zb_linear_apply", "zb_linear_attn",
     "zb_affine_fit", "zb_gather_tiles", "zb_last_device_status", "HybridLayer",
     "LAUNCHES_PER_CALL",
 ]
@@ -36,7 +36,7 @@ HEAD_DIM = 64
 # kernels each entry point launches (for counting launches in a timed region)
 LAUNCHES_PER_CALL = {
     "zb_landmark_build": 1, "zb_tile_score_topk": 2, "zb_tile_sparse_attn": 1, "zb_dense_attn": 1,
-    "zb_linear_state": 2, "zb_linear_apply": 1, "zb_affine_fit": 3, "zb_gather_tiles": 1,
+    "zb_linear_state": 2, "zb_linear_apply": 1, "zb_linear_attn": 3, "zb_affine_fit": 3, "zb_gather_tiles": 1,
 }
 
 
@@ -234,6 +234,28 @@ def zb_linear_apply(Q, S, z, A: Optional[torch.Tensor] = None, b: Optional[torch
     st = _lib_handle().zb_linear_apply(_ptr(Q), H, N, d, _ptr(S), _ptr(z), _ptr(A), _ptr(b), _ptr(O),
                                        1 if out_fp32 else 0, _stream())
     _check(st, "zb_linear_apply")
+    return O
+
+
+def linear_attn_workspace_bytes(heads: int, n_tokens: int, head_dim: int = HEAD_DIM) -> int:
+    return int(_lib_handle().zb_linear_attn_workspace_bytes(heads, n_tokens, head_dim))
+
+
+def zb_linear_attn(Q, K, V, A: Optional[torch.Tensor] = None, b: Optional[torch.Tensor] = None,
+                   out: Optional[torch.Tensor] = None, ws: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """The whole linear stage in one C call: O = (phi(Q) S / (phi(Q) . z)) A + b, bf16."""
+    for t, n in ((Q, "Q"), (K, "K"), (V, "V")):
+        _need(t, torch.bfloat16, n, 3)
+    if A is not None:
+        _need(A, torch.float32, "A", 3)
+    if b is not None:
+        _need(b, torch.float32, "b", 2)
+    H, N, d = Q.shape
+    O = _out((H, N, d), torch.bfloat16, Q.device, out, "O")
+    ws = _ws(linear_attn_workspace_bytes(H, N, d), Q.device, ws)
+    st = _lib_handle().zb_linear_attn(_ptr(Q), _ptr(K), _ptr(V), H, N, d, _ptr(A), _ptr(b), _ptr(O), _ptr(ws),
+                                      ws.numel() * ws.element_size(), _stream())
+    _check(st, "zb_linear_attn")
     return O
 
 

@@ -639,6 +639,42 @@ extern "C" zb_status zb_linear_apply(const uint16_t* Q, int32_t heads, int64_t n
     return cudaGetLastError() == cudaSuccess ? ZB_OK : ZB_ERR_CUDA;
 }
 
+// ==================================================== the whole stage ====
+// zb_linear_attn = zb_linear_state + zb_linear_apply in one call; the state S,
+// z and the state partials live in the caller's workspace:
+//   [S: H d d fp32][z: H d fp32][partials], each part 256-byte aligned.
+namespace zb {
+namespace lin {
+static size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+static size_t attn_s_bytes(int heads) { return align256(size_t(heads) * 64 * 64 * sizeof(float)); }
+static size_t attn_z_bytes(int heads) { return align256(size_t(heads) * 64 * sizeof(float)); }
+}  // namespace lin
+}  // namespace zb
+
+extern "C" size_t zb_linear_attn_workspace_bytes(int32_t heads, int64_t n_tokens, int32_t head_dim) {
+    if (heads < 1 || n_tokens < 1 || head_dim != 64) return 0;
+    return lin::attn_s_bytes(heads) + lin::attn_z_bytes(heads) + lin::align256(lin::state_ws_bytes(heads, n_tokens));
+}
+
+extern "C" zb_status zb_linear_attn(const uint16_t* Q, const uint16_t* K, const uint16_t* V, int32_t heads,
+                                    int64_t n_tokens, int32_t head_dim, const float* A, const float* b,
+                                    uint16_t* O, void* ws, size_t ws_bytes, void* stream) {
+    if (heads < 1 || n_tokens < 1) return ZB_ERR_SHAPE;
+    if (head_dim != 64) return ZB_ERR_UNSUPPORTED;
+    if (!Q || !O) return ZB_ERR_NULL;
+    if (!aligned16(Q) || !aligned16(O) || !aligned16(A) || !aligned16(b) || !aligned16(ws)) return ZB_ERR_ALIGN;
+    const size_t need = zb_linear_attn_workspace_bytes(heads, n_tokens, head_dim);
+    if (!ws || ws_bytes < need) return ZB_ERR_WORKSPACE;
+    unsigned char* w = static_cast<unsigned char*>(ws);
+    float* S = reinterpret_cast<float*>(w);
+    float* z = reinterpret_cast<float*>(w + lin::attn_s_bytes(heads));
+    void* part = w + lin::attn_s_bytes(heads) + lin::attn_z_bytes(heads);
+    zb_status e = zb_linear_state(K, V, heads, n_tokens, head_dim, S, z, part,
+                                  ws_bytes - lin::attn_s_bytes(heads) - lin::attn_z_bytes(heads), stream);
+    if (e != ZB_OK) return e;
+    return zb_linear_apply(Q, heads, n_tokens, head_dim, S, z, A, b, O, 0, stream);
+}
+
 // ======================================= linear state without a workspace ====
 // zb_linear_state needs a caller-allocated workspace for the per-CTA partial
 // states.  Some callers cannot allocate device memory when they call the

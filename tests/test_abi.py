@@ -27,7 +27,7 @@ def _declared():
 def test_header_declares_the_calls():
     names = _declared()
     for n in ["zb_landmark_build", "zb_tile_score_topk", "zb_tile_sparse_attn", "zb_dense_attn",
-              "zb_linear_state", "zb_linear_apply", "zb_affine_fit", "zb_gather_tiles",
+              "zb_linear_state", "zb_linear_apply", "zb_linear_attn", "zb_affine_fit", "zb_gather_tiles",
               "zb_last_device_status", "zb_status_string", "zb_abi_version"]:
         assert n in names
 
@@ -52,6 +52,10 @@ def test_workspace_sizes(lib):
     assert lib.zb_linear_state_workspace_bytes(16, 1000, 32) == 0
     assert lib.zb_affine_fit_workspace_bytes(16, 4096, 64) == 16 * (128 + 16 * 2 * 4096) * 8
     assert lib.zb_affine_fit_workspace_bytes(0, 4096, 64) == 0
+    # the one-call linear stage holds S, z and the state partials, each 256-byte aligned
+    lin = lib.zb_linear_attn_workspace_bytes(16, 1024 * 1374, 64)
+    assert lin >= n + 16 * 64 * 65 * 4 and lin % 256 == 0
+    assert lib.zb_linear_attn_workspace_bytes(16, 1000, 32) == 0
     assert lib.zb_tile_score_topk_workspace_bytes(_shape(H=16, N=1024 * 1374, t=128)) == 4 * 10992 ** 2 * 8
     assert lib.zb_tile_score_topk_workspace_bytes(_shape(H=2, N=256, t=64)) == 2 * 16 * 8
 
@@ -100,6 +104,13 @@ def test_validation_errors_before_launch(lib):
     assert lib.zb_linear_apply(FAKE, 2, 256, 64, FAKE, None, None, None, FAKE, 0, None) == 1
     assert lib.zb_linear_apply(FAKE, 2, 256, 64, FAKE, FAKE, FAKE + 2, None, FAKE, 1, None) == 3
     # affine fit: too few rows, workspace
+    lin = lib.zb_linear_attn_workspace_bytes(2, 256, 64)
+    assert lib.zb_linear_attn(FAKE, FAKE, FAKE, 2, 0, 64, None, None, FAKE, FAKE, lin, None) == 2
+    assert lib.zb_linear_attn(FAKE, FAKE, FAKE, 2, 256, 32, None, None, FAKE, FAKE, lin, None) == 4
+    assert lib.zb_linear_attn(None, FAKE, FAKE, 2, 256, 64, None, None, FAKE, FAKE, lin, None) == 1
+    assert lib.zb_linear_attn(FAKE, FAKE, FAKE, 2, 256, 64, FAKE + 4, None, FAKE, FAKE, lin, None) == 3
+    assert lib.zb_linear_attn(FAKE, FAKE, FAKE, 2, 256, 64, None, None, FAKE, FAKE, lin - 1, None) == 5
+    assert lib.zb_linear_attn(FAKE, FAKE, FAKE, 2, 256, 64, None, None, FAKE, None, lin, None) == 5
     assert lib.zb_affine_fit(FAKE, FAKE, 2, 64, 64, FAKE, FAKE, FAKE, 1 << 30, None) == 2
     wsn = lib.zb_affine_fit_workspace_bytes(2, 300, 64)
     assert lib.zb_affine_fit(FAKE, FAKE, 2, 300, 64, FAKE, FAKE, FAKE, wsn - 8, None) == 5

@@ -52,6 +52,29 @@ def test_linear_attention_matches_oracle(heads, n, affine):
     assert rel_err_per_head(host(O), ref) <= REL_TOL
 
 
+@pytest.mark.parametrize("heads,n,affine", [(2, 300, False), (3, 5000, True)])
+def test_linear_attn_one_call_matches_oracle(heads, n, affine):
+    """zb_linear_attn (state + output in one C call) against the fp64 oracle, and
+    bit-identical to the two separate calls it is made of."""
+    zb = _zb()
+    w = workload("linear256", heads=heads, n_tokens=n)
+    Q, K, V = synth.make_qkv(w, device="cuda")
+    A = b = None
+    if affine:
+        g = torch.Generator(device="cuda").manual_seed(5)
+        A = (torch.eye(64, device="cuda") + 0.1 * torch.randn(heads, 64, 64, generator=g, device="cuda")).contiguous()
+        b = (0.01 * torch.randn(heads, 64, generator=g, device="cuda")).contiguous()
+    O = zb.zb_linear_attn(Q, K, V, A, b)
+    S, z = zb.zb_linear_state(K, V)
+    O2 = zb.zb_linear_apply(Q, S, z, A, b)
+    sync_ok()
+    assert torch.equal(O, O2)
+    ref = oracle.linear_attention(host(Q), host(K), host(V),
+                                  None if A is None else A.double().cpu().numpy(),
+                                  None if b is None else b.double().cpu().numpy())
+    assert rel_err_per_head(host(O), ref) <= REL_TOL
+
+
 def test_affine_fit_matches_oracle_on_same_inputs():
     zb = _zb()
     g = torch.Generator(device="cuda").manual_seed(11)
