@@ -294,7 +294,7 @@ def main():
                               ws=layer.ws_topk)
         mark(2)
         zb.zb_tile_sparse_attn(Q, K, V, layer.lm.Kbar_bf16, layer.lm.Vbar_bf16, layer.idx, w.k, w.tile, True,
-                               layer.scale, out=layer.O_sparse)
+                               layer.scale, out=layer.O_sparse, ws=layer.ws_attn)
         mark(3)
         zb.zb_linear_state(K, V, layer.S, layer.z, layer.ws_lin)
         mark(4)

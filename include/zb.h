@@ -120,16 +120,24 @@ zb_status zb_tile_score_topk(const double* Qbar, const double* Kbar, zb_shape s,
  *        NULL when use_landmarks == 0);  idx int32 [H][T][k], each row strictly
  *        ascending in [0, T) (checked on the device: ZB_ERR_INDEX);  0 <= k <= T
  *        (k == 0 needs use_landmarks);  scale > 0 (usually 1/sqrt(d)).
+ *   ws : NULL, or zb_tile_sparse_attn_workspace_bytes() bytes, 16-byte aligned,
+ *        owned by the caller and not shared with a call running at the same
+ *        time.  With a workspace the call zeroes two counters in it (in stream
+ *        order) and launches cooperatively; the work items in flight on all SMs
+ *        then start each round together, so their ascending sweeps over a
+ *        head's selected K/V tiles stay close and share L2 (far less DRAM
+ *        traffic at long sequences).  The result is bit-identical either way.
  *   out: O bf16 [H][N][d];  lse fp32 [H][N] natural-log log-sum-exp of each
  *        row's logits (may be NULL).
  * Errors: ZB_ERR_NULL, ZB_ERR_SHAPE, ZB_ERR_ALIGN, ZB_ERR_UNSUPPORTED (T > 32768),
- * ZB_ERR_CUDA.
+ * ZB_ERR_WORKSPACE, ZB_ERR_CUDA.
  */
+size_t zb_tile_sparse_attn_workspace_bytes(void);
 zb_status zb_tile_sparse_attn(const uint16_t* Q, const uint16_t* K, const uint16_t* V,
                               const uint16_t* Kbar_bf16, const uint16_t* Vbar_bf16,
                               const int32_t* idx, int32_t k, int32_t use_landmarks,
                               float scale, zb_shape s, uint16_t* O, float* lse,
-                              void* stream);
+                              void* ws, size_t ws_bytes, void* stream);
 
 /*
  * Dense softmax attention softmax(scale * Q K^T) V: the unconverted layer the

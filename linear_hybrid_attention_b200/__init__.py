@@ -146,8 +146,13 @@ def zb_tile_score_topk(Qbar: torch.Tensor, Kbar: torch.Tensor, n_tokens: int, ti
 def zb_tile_sparse_attn(Q, K, V, Kbar_bf16, Vbar_bf16, idx, k: int, tile: int,
                         use_landmarks: bool = True, scale: Optional[float] = None,
                         out: Optional[torch.Tensor] = None, lse: Optional[torch.Tensor] = None,
-                        want_lse: bool = False):
-    """Tile-sparse softmax attention with landmarks; returns O (and lse if asked)."""
+                        want_lse: bool = False, ws: Optional[torch.Tensor] = None,
+                        wave_sync: bool = True):
+    """Tile-sparse softmax attention with landmarks; returns O (and lse if asked).
+
+    wave_sync passes the call a small workspace (``ws``, or a fresh one) so that
+    the work items in flight sweep K/V in step (more L2 reuse); the result is
+    the same bit for bit without it."""
     for t, n in ((Q, "Q"), (K, "K"), (V, "V")):
         _need(t, torch.bfloat16, n, 3)
     H, N, d = Q.shape
@@ -163,10 +168,15 @@ def zb_tile_sparse_attn(Q, K, V, Kbar_bf16, Vbar_bf16, idx, k: int, tile: int,
     O = _out((H, N, d), torch.bfloat16, Q.device, out, "O")
     if want_lse or lse is not None:
         lse = _out((H, N), torch.float32, Q.device, lse, "lse")
+    if wave_sync:
+        ws = _ws(int(_lib_handle().zb_tile_sparse_attn_workspace_bytes()), Q.device, ws)
+    else:
+        ws = None
     st = _lib_handle().zb_tile_sparse_attn(
         _ptr(Q), _ptr(K), _ptr(V), _ptr(Kbar_bf16 if use_landmarks else None),
         _ptr(Vbar_bf16 if use_landmarks else None), _ptr(idx), int(k), 1 if use_landmarks else 0,
-        float(scale), _lib.ZbShape(H, N, d, tile), _ptr(O), _ptr(lse), _stream())
+        float(scale), _lib.ZbShape(H, N, d, tile), _ptr(O), _ptr(lse), _ptr(ws),
+        0 if ws is None else ws.numel() * ws.element_size(), _stream())
     _check(st, "zb_tile_sparse_attn")
     return (O, lse) if lse is not None else O
 
@@ -317,6 +327,8 @@ class HybridLayer:
                             torch.empty(H, T, d, dtype=torch.bfloat16, device=dev))
         self.idx = torch.empty(H, T, k, dtype=torch.int32, device=dev)
         self.ws_topk = torch.empty(max(topk_workspace_bytes(H, N, tile, d), 16), dtype=torch.uint8, device=dev)
+        self.ws_attn = torch.empty(int(_lib_handle().zb_tile_sparse_attn_workspace_bytes()), dtype=torch.uint8,
+                                   device=dev)
         self.O_sparse = torch.empty(H, N, d, dtype=torch.bfloat16, device=dev)
         self.O_linear = torch.empty(H, N, d, dtype=torch.bfloat16, device=dev)
         self.S = torch.empty(H, d, d, dtype=torch.float32, device=dev)
@@ -348,7 +360,7 @@ class HybridLayer:
         zb_tile_score_topk(self.lm.Qbar, self.lm.Kbar, self.n_tokens, self.tile, self.k, out=self.idx,
                            ws=self.ws_topk)
         return zb_tile_sparse_attn(Q, K, V, self.lm.Kbar_bf16, self.lm.Vbar_bf16, self.idx, self.k,
-                                   self.tile, True, self.scale, out=self.O_sparse)
+                                   self.tile, True, self.scale, out=self.O_sparse, ws=self.ws_attn)
 
     def calibrate(self, Q, K, V):
         zb_linear_state(K, V, self.S, self.z, self.ws_lin)

@@ -27,8 +27,9 @@ PROTOTYPES = {
     "zb_landmark_build": (c_i32, [c_vp, c_vp, c_vp, ZbShape, c_vp, c_vp, c_vp, c_vp, c_vp]),
     "zb_tile_score_topk_workspace_bytes": (c_sz, [ZbShape]),
     "zb_tile_score_topk": (c_i32, [c_vp, c_vp, ZbShape, c_i32, c_vp, c_vp, c_sz, c_vp]),
+    "zb_tile_sparse_attn_workspace_bytes": (c_sz, []),
     "zb_tile_sparse_attn": (c_i32, [c_vp, c_vp, c_vp, c_vp, c_vp, c_vp, c_i32, c_i32, c_f32, ZbShape,
-                                    c_vp, c_vp, c_vp]),
+                                    c_vp, c_vp, c_vp, c_sz, c_vp]),
     "zb_dense_attn": (c_i32, [c_vp, c_i64, c_vp, c_vp, c_i64, c_i32, c_i32, c_f32, c_vp, c_i32, c_vp, c_vp]),
     "zb_linear_state_workspace_bytes": (c_sz, [c_i32, c_i64, c_i32]),
     "zb_linear_state": (c_i32, [c_vp, c_vp, c_i32, c_i64, c_i32, c_vp, c_vp, c_vp, c_sz, c_vp]),

@@ -99,6 +99,7 @@ struct Params {
     void* O;
     int out_fp32;      // 1: O is fp32, else bf16
     float* lse;
+    unsigned* wave;    // 2 zeroed counters for the wave synchronisation, or NULL
     int* status;
     unsigned long long timeout_ns;
 };
@@ -142,6 +143,25 @@ ZB_DEVINL void mma_ts(uint32_t d_tmem, uint32_t a_tmem, uint32_t b_lo, uint32_t 
         "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], db, %3, p;\n\t}" ::"r"(d_tmem),
         "r"(a_tmem), "r"(b_lo), "r"(idesc), "r"(accumulate), "r"(DESC_HI)
         : "memory");
+}
+
+// Wave synchronisation across the grid: spin (bounded) until *ctr >= target.
+ZB_DEVINL bool wave_wait(const unsigned* ctr, unsigned target, const WaitCtx& w) {
+    const uint64_t t0 = globaltimer_ns();
+    for (uint32_t it = 0;; ++it) {
+        unsigned v;
+        asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(ctr) : "memory");
+        if (v >= target) return true;
+        if ((it & 15u) == 15u) {
+            if (*w.abort_flag) return false;
+            if (globaltimer_ns() - t0 > w.timeout_ns) {
+                flag_status(w.status, ZB_ERR_TIMEOUT);
+                *w.abort_flag = 1;
+                return false;
+            }
+        }
+        __nanosleep(128);
+    }
 }
 
 // The key tile of step j of an item: selected tile idx[j] (clamped), or -1 for a landmark chunk.
@@ -236,7 +256,19 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
             bool q_issued = false;
             uint32_t q_par = 0;
             bool ok = true;
+            // Wave synchronisation (when the caller passed counters): round r
+            // of this slot starts on every CTA together, so the items in flight
+            // sweep the head's K/V in step and share it through L2.  Barrier
+            // r >= 1 is passed when all G producers of the slot have arrived;
+            // R_s rounds in all (the most any CTA has).
+            const int R = ((static_cast<int>((p.n_items - 1) / G) + 1) + 1 - s) / 2;
+            int arrived = 0;  // barriers arrived at so far
             for (int r = 0; r < items && ok; ++r) {
+                if (p.wave && r >= 1) {
+                    atomicAdd(p.wave + s, 1u);
+                    arrived = r;
+                    if (!wave_wait(p.wave + s, static_cast<unsigned>(r) * static_cast<unsigned>(G), wc)) break;
+                }
                 const long long item = first + static_cast<long long>(2 * r + s) * G;
                 const int h = static_cast<int>(item / p.Tq);
                 const int i = static_cast<int>(item % p.Tq);
@@ -272,7 +304,11 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                     if (++vst == V_STAGES) { vst = 0; vph ^= 1u; }
                 }
             }
-            // leave no TMA write in flight (bounded, even after an abort)
+            // arrive at the barriers of the rounds this CTA does not run (so the
+            // others pass them), then leave no TMA write in flight (bounded,
+            // even after an abort)
+            if (p.wave)
+                for (int r = arrived + 1; r < R; ++r) atomicAdd(p.wave + s, 1u);
             volatile int no_abort = 0;
             const WaitCtx w2{p.status, &no_abort, p.timeout_ns};
             for (int st = 0; st < K_STAGES; ++st)
@@ -594,7 +630,7 @@ static zb_status launch_attn(const uint16_t* Q, const uint16_t* K, const uint16_
                              const uint16_t* Kb, const uint16_t* Vb, const int32_t* idx, int heads,
                              long long n_q, long long n_kv, int tq, int tk, int k, int dense,
                              int use_lm, float scale, void* O, int out_fp32, float* lse,
-                             cudaStream_t st) {
+                             unsigned* wave, cudaStream_t st) {
     using namespace attn;
     DeviceInfo dev;
     zb_status e = current_device(&dev);
@@ -633,6 +669,7 @@ static zb_status launch_attn(const uint16_t* Q, const uint16_t* K, const uint16_
     p.O = O;
     p.out_fp32 = out_fp32;
     p.lse = lse;
+    p.wave = wave;
     p.status = dev.status;
     p.timeout_ns = wait_timeout_ns();
     const size_t smem = attn_smem_bytes();
@@ -640,19 +677,30 @@ static zb_status launch_attn(const uint16_t* Q, const uint16_t* K, const uint16_
                                           static_cast<int>(smem));
     if (ce != cudaSuccess) return ZB_ERR_CUDA;
     const long long grid = p.n_items < dev.sm_count ? p.n_items : dev.sm_count;
-    sparse_attn_kernel<<<static_cast<unsigned>(grid), NUM_THREADS, smem, st>>>(mq, mk, mv, mkb, mvb, p);
-    return cudaGetLastError() == cudaSuccess ? ZB_OK : ZB_ERR_CUDA;
+    if (!wave) {
+        sparse_attn_kernel<<<static_cast<unsigned>(grid), NUM_THREADS, smem, st>>>(mq, mk, mv, mkb, mvb, p);
+        return cudaGetLastError() == cudaSuccess ? ZB_OK : ZB_ERR_CUDA;
+    }
+    // The wave barriers need every CTA resident at once: zero the counters in
+    // stream order, then a cooperative launch (which guarantees co-residency).
+    if (cudaMemsetAsync(wave, 0, 2 * sizeof(unsigned), st) != cudaSuccess) return ZB_ERR_CUDA;
+    void* args[] = {&mq, &mk, &mv, &mkb, &mvb, &p};
+    ce = cudaLaunchCooperativeKernel(reinterpret_cast<const void*>(sparse_attn_kernel),
+                                     dim3(static_cast<unsigned>(grid)), dim3(NUM_THREADS), args, smem, st);
+    return ce == cudaSuccess ? ZB_OK : ZB_ERR_CUDA;
 }
 
 }  // namespace zb
 
 using namespace zb;
 
+extern "C" size_t zb_tile_sparse_attn_workspace_bytes(void) { return 256; }
+
 extern "C" zb_status zb_tile_sparse_attn(const uint16_t* Q, const uint16_t* K, const uint16_t* V,
                                          const uint16_t* Kbar_bf16, const uint16_t* Vbar_bf16,
                                          const int32_t* idx, int32_t k, int32_t use_landmarks,
                                          float scale, zb_shape s, uint16_t* O, float* lse,
-                                         void* stream) {
+                                         void* ws, size_t ws_bytes, void* stream) {
     zb_status e = check_shape(s);
     if (e != ZB_OK) return e;
     if (!Q || !K || !V || !O) return ZB_ERR_NULL;
@@ -665,10 +713,11 @@ extern "C" zb_status zb_tile_sparse_attn(const uint16_t* Q, const uint16_t* K, c
     if (lm && (!Kbar_bf16 || !Vbar_bf16)) return ZB_ERR_NULL;
     if (!(scale > 0.f) || !isfinite(scale)) return ZB_ERR_SHAPE;
     if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(O) || !aligned16(idx) ||
-        !aligned16(lse) || (lm && (!aligned16(Kbar_bf16) || !aligned16(Vbar_bf16))))
+        !aligned16(lse) || !aligned16(ws) || (lm && (!aligned16(Kbar_bf16) || !aligned16(Vbar_bf16))))
         return ZB_ERR_ALIGN;
+    if (ws && ws_bytes < zb_tile_sparse_attn_workspace_bytes()) return ZB_ERR_WORKSPACE;
     return launch_attn(Q, K, V, Kbar_bf16, Vbar_bf16, idx, s.heads, s.n_tokens, s.n_tokens, s.tile,
-                       s.tile, k, 0, use_landmarks ? 1 : 0, scale, O, 0, lse,
+                       s.tile, k, 0, use_landmarks ? 1 : 0, scale, O, 0, lse, static_cast<unsigned*>(ws),
                        static_cast<cudaStream_t>(stream));
 }
 
@@ -685,5 +734,5 @@ extern "C" zb_status zb_dense_attn(const uint16_t* Q, int64_t n_q, const uint16_
         return ZB_ERR_ALIGN;
     const int Tk = static_cast<int>((n_kv + 127) / 128);
     return launch_attn(Q, K, V, nullptr, nullptr, nullptr, heads, n_q, n_kv, 128, 128, Tk, 1, 0,
-                       scale, O, out_fp32 ? 1 : 0, lse, static_cast<cudaStream_t>(stream));
+                       scale, O, out_fp32 ? 1 : 0, lse, nullptr, static_cast<cudaStream_t>(stream));
 }

@@ -86,13 +86,17 @@ def test_validation_errors_before_launch(lib):
     assert lib.zb_tile_score_topk(FAKE, FAKE, S, 0, None, None, 0, None) == 0  # nothing to do
     # sparse attention
     a = (FAKE, FAKE, FAKE, FAKE, FAKE, FAKE)
-    assert lib.zb_tile_sparse_attn(*a, 5, 1, 0.125, S, FAKE, None, None) == 2          # k > T
-    assert lib.zb_tile_sparse_attn(*a, 0, 0, 0.125, S, FAKE, None, None) == 2          # no keys
-    assert lib.zb_tile_sparse_attn(*a, 2, 1, -1.0, S, FAKE, None, None) == 2           # scale
-    assert lib.zb_tile_sparse_attn(FAKE, FAKE, FAKE, None, FAKE, FAKE, 2, 1, 0.125, S, FAKE, None, None) == 1
-    assert lib.zb_tile_sparse_attn(FAKE, FAKE, FAKE, FAKE, FAKE, None, 2, 1, 0.125, S, FAKE, None, None) == 1
-    assert lib.zb_tile_sparse_attn(*a, 2, 1, 0.125, S, FAKE + 4, None, None) == 3
-    assert lib.zb_tile_sparse_attn(*a, 2, 1, 0.125, _shape(N=128 * 40000), FAKE, None, None) == 4  # T > 32768
+    assert lib.zb_tile_sparse_attn(*a, 5, 1, 0.125, S, FAKE, None, None, 0, None) == 2          # k > T
+    assert lib.zb_tile_sparse_attn(*a, 0, 0, 0.125, S, FAKE, None, None, 0, None) == 2          # no keys
+    assert lib.zb_tile_sparse_attn(*a, 2, 1, -1.0, S, FAKE, None, None, 0, None) == 2           # scale
+    assert lib.zb_tile_sparse_attn(FAKE, FAKE, FAKE, None, FAKE, FAKE, 2, 1, 0.125, S, FAKE, None, None, 0, None) == 1
+    assert lib.zb_tile_sparse_attn(FAKE, FAKE, FAKE, FAKE, FAKE, None, 2, 1, 0.125, S, FAKE, None, None, 0, None) == 1
+    assert lib.zb_tile_sparse_attn(*a, 2, 1, 0.125, S, FAKE + 4, None, None, 0, None) == 3
+    assert lib.zb_tile_sparse_attn(*a, 2, 1, 0.125, _shape(N=128 * 40000), FAKE, None, None, 0, None) == 4  # T > 32768
+    wsa = lib.zb_tile_sparse_attn_workspace_bytes()
+    assert wsa == 256
+    assert lib.zb_tile_sparse_attn(*a, 2, 1, 0.125, S, FAKE, None, FAKE, wsa - 1, None) == 5   # short workspace
+    assert lib.zb_tile_sparse_attn(*a, 2, 1, 0.125, S, FAKE, None, FAKE + 8, wsa, None) == 3   # misaligned
     # dense
     assert lib.zb_dense_attn(FAKE, 0, FAKE, FAKE, 10, 2, 64, 0.125, FAKE, 0, None, None) == 2
     assert lib.zb_dense_attn(FAKE, 10, FAKE, FAKE, 10, 2, 128, 0.125, FAKE, 1, None, None) == 4

@@ -128,6 +128,22 @@ def test_sparse_full_views32_sampled():
     assert (O.float() >= Vh.amin(1, keepdim=True) - 1e-2).all()
 
 
+def test_wave_sync_is_bit_identical():
+    """The 32-view stage (about 18 rounds per slot on every SM) with and without
+    the wave synchronisation: only the schedule differs, not one bit of O."""
+    zb = _zb()
+    w = workload("views32")
+    Q, K, V = synth.make_qkv(w, device="cuda")
+    lm = zb.zb_landmark_build(Q, K, V, w.tile)
+    idx = zb.zb_tile_score_topk(lm.Qbar, lm.Kbar, w.n_tokens, w.tile, w.k)
+    a, la = zb.zb_tile_sparse_attn(Q, K, V, lm.Kbar_bf16, lm.Vbar_bf16, idx, w.k, w.tile, want_lse=True,
+                                   wave_sync=True)
+    b, lb = zb.zb_tile_sparse_attn(Q, K, V, lm.Kbar_bf16, lm.Vbar_bf16, idx, w.k, w.tile, want_lse=True,
+                                   wave_sync=False)
+    sync_ok()
+    assert torch.equal(a, b) and torch.equal(la, lb)
+
+
 @pytest.mark.parametrize("nq,nk", [(300, 1000), (128, 128), (1, 77), (4096, 6000)])
 def test_dense_matches_oracle(nq, nk):
     zb = _zb()
