@@ -122,7 +122,7 @@ zb_status zb_tile_score_topk(const double* Qbar, const double* Kbar, zb_shape s,
  *        (k == 0 needs use_landmarks);  scale > 0 (usually 1/sqrt(d)).
  *   ws : NULL, or zb_tile_sparse_attn_workspace_bytes() bytes, 16-byte aligned,
  *        owned by the caller and not shared with a call running at the same
- *        time.  With a workspace the call zeroes two counters in it (in stream
+ *        time.  With a workspace the call zeroes a counter in it (in stream
  *        order) and launches cooperatively; the work items in flight on all SMs
  *        then start each round together, so their ascending sweeps over a
  *        head's selected K/V tiles stay close and share L2 (far less DRAM

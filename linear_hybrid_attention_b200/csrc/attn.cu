@@ -99,7 +99,7 @@ struct Params {
     void* O;
     int out_fp32;      // 1: O is fp32, else bf16
     float* lse;
-    unsigned* wave;    // 2 zeroed counters for the wave synchronisation, or NULL
+    unsigned* wave;    // zeroed counter for the wave synchronisation, or NULL
     int* status;
     unsigned long long timeout_ns;
 };
@@ -256,18 +256,18 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
             bool q_issued = false;
             uint32_t q_par = 0;
             bool ok = true;
-            // Wave synchronisation (when the caller passed counters): round r
-            // of this slot starts on every CTA together, so the items in flight
-            // sweep the head's K/V in step and share it through L2.  Barrier
-            // r >= 1 is passed when all G producers of the slot have arrived;
-            // R_s rounds in all (the most any CTA has).
-            const int R = ((static_cast<int>((p.n_items - 1) / G) + 1) + 1 - s) / 2;
+            // Wave synchronisation (when the caller passed a counter): round r
+            // starts on both slots of every CTA together, so the items in
+            // flight sweep the head's K/V in step and share it through L2.
+            // Barrier r >= 1 is passed when all 2 G producers have arrived; R
+            // rounds in all (the most any slot of any CTA has).
+            const int R = (static_cast<int>((p.n_items - 1) / G) + 2) / 2;
             int arrived = 0;  // barriers arrived at so far
             for (int r = 0; r < items && ok; ++r) {
                 if (p.wave && r >= 1) {
-                    atomicAdd(p.wave + s, 1u);
+                    atomicAdd(p.wave, 1u);
                     arrived = r;
-                    if (!wave_wait(p.wave + s, static_cast<unsigned>(r) * static_cast<unsigned>(G), wc)) break;
+                    if (!wave_wait(p.wave, static_cast<unsigned>(r) * 2u * static_cast<unsigned>(G), wc)) break;
                 }
                 const long long item = first + static_cast<long long>(2 * r + s) * G;
                 const int h = static_cast<int>(item / p.Tq);
@@ -308,7 +308,7 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
             // others pass them), then leave no TMA write in flight (bounded,
             // even after an abort)
             if (p.wave)
-                for (int r = arrived + 1; r < R; ++r) atomicAdd(p.wave + s, 1u);
+                for (int r = arrived + 1; r < R; ++r) atomicAdd(p.wave, 1u);
             volatile int no_abort = 0;
             const WaitCtx w2{p.status, &no_abort, p.timeout_ns};
             for (int st = 0; st < K_STAGES; ++st)
@@ -683,7 +683,7 @@ static zb_status launch_attn(const uint16_t* Q, const uint16_t* K, const uint16_
     }
     // The wave barriers need every CTA resident at once: zero the counters in
     // stream order, then a cooperative launch (which guarantees co-residency).
-    if (cudaMemsetAsync(wave, 0, 2 * sizeof(unsigned), st) != cudaSuccess) return ZB_ERR_CUDA;
+    if (cudaMemsetAsync(wave, 0, sizeof(unsigned), st) != cudaSuccess) return ZB_ERR_CUDA;
     void* args[] = {&mq, &mk, &mv, &mkb, &mvb, &p};
     ce = cudaLaunchCooperativeKernel(reinterpret_cast<const void*>(sparse_attn_kernel),
                                      dim3(static_cast<unsigned>(grid)), dim3(NUM_THREADS), args, smem, st);
