@@ -56,6 +56,12 @@ constexpr uint32_t TMEM_COLS = 512;
 // TMEM columns of slot s start at 256 s: S (128 fp32), P (64 = 128 bf16), O (64 fp32)
 constexpr uint32_t SLOT_COLS = 256, TM_S = 0, TM_P = 128, TM_O = 192;
 constexpr uint32_t SLEEP_NS = 20000;  // longest sleep inside one barrier poll of a role thread
+// Registers: the kernel is compiled for LAUNCH_REGS per thread (384 threads,
+// one CTA per SM); the role warpgroup then gives registers back and the two
+// softmax warpgroups take them (setmaxnreg), which adds up exactly:
+// 128 * ROLE_REGS + 256 * SOFTMAX_REGS == 384 * LAUNCH_REGS.
+constexpr int LAUNCH_REGS = 168, ROLE_REGS = 56, SOFTMAX_REGS = 224;
+static_assert(128 * ROLE_REGS + 256 * SOFTMAX_REGS == NUM_THREADS * LAUNCH_REGS, "register split");
 
 constexpr float LOG2E = 1.4426950408889634f;
 constexpr float RESCALE_THRESHOLD = 8.0f;  // log2 units: p <= 2^8 before a rescale
@@ -103,6 +109,11 @@ struct Params {
     int* status;
     unsigned long long timeout_ns;
 };
+
+template <int N>
+ZB_DEVINL void setmaxnreg_inc() { asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N)); }
+template <int N>
+ZB_DEVINL void setmaxnreg_dec() { asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N)); }
 
 // 32 lanes x 16 consecutive 32-bit columns
 ZB_DEVINL void tmem_st16(uint32_t taddr, const uint32_t* r) {
@@ -241,6 +252,7 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
     const uint32_t tmem = sm.tmem_base;
 
     if (warp < 4) {
+        setmaxnreg_dec<ROLE_REGS>();
         // Role warps: warp 0 / 2 produce for slot 0 / 1, warp 1 / 3 issue its
         // MMAs.  The two slots' pipelines share nothing but the SM.
         const int s = warp >> 1;
@@ -381,6 +393,7 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
         }
         __syncwarp();
     } else {
+        setmaxnreg_inc<SOFTMAX_REGS>();
         // ===================================== softmax warpgroup of a slot ====
         const int s = (warp >> 2) - 1;
         SlotSmem& b = sm.slot[s];
@@ -672,6 +685,19 @@ static zb_status launch_attn(const uint16_t* Q, const uint16_t* K, const uint16_
     p.wave = wave;
     p.status = dev.status;
     p.timeout_ns = wait_timeout_ns();
+    // The setmaxnreg split only adds up for a kernel compiled to exactly
+    // LAUNCH_REGS registers per thread; refuse to launch anything else.
+    static int regs_ok = -1;
+    static std::mutex regs_mu;
+    {
+        std::lock_guard<std::mutex> lock(regs_mu);
+        if (regs_ok < 0) {
+            cudaFuncAttributes fa;
+            if (cudaFuncGetAttributes(&fa, sparse_attn_kernel) != cudaSuccess) return ZB_ERR_CUDA;
+            regs_ok = fa.numRegs == LAUNCH_REGS ? 1 : 0;
+        }
+        if (!regs_ok) return ZB_ERR_UNSUPPORTED;
+    }
     const size_t smem = attn_smem_bytes();
     cudaError_t ce = cudaFuncSetAttribute(sparse_attn_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                           static_cast<int>(smem));
