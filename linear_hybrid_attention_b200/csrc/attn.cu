@@ -290,30 +290,58 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                 tma_load_3d(smem_addr(b.q), &tm_q, smem_addr(&b.q_full), 0, i * p.tq, h);
                 q_issued = true;
                 q_par = r & 1u;
-                for (int j = 0; j < n; ++j) {
-                    const int t = step_tile(p, list, j);
-                    if (!mbar_wait_sleep(smem_addr(&b.k_empty[kst]), kph ^ 1u, wc, SLEEP_NS)) { ok = false; break; }
-                    if (t >= 0) {
-                        mbar_arrive_expect_tx(smem_addr(&b.k_full[kst]), p.tk * HD * 2);
-                        tma_load_3d(smem_addr(b.k[kst]), &tm_k, smem_addr(&b.k_full[kst]), 0, t * p.tk, h);
-                    } else {
-                        mbar_arrive_expect_tx(smem_addr(&b.k_full[kst]), TILE_BYTES);
-                        tma_load_3d(smem_addr(b.k[kst]), &tm_kb, smem_addr(&b.k_full[kst]), 0, (j - p.k) * BN, h);
+                // K and V fill their rings independently (K leads: S = Q K^T
+                // of a step is needed before its P V), so a slow V stage never
+                // holds back the K loads.  Non-blocking tests; after a round
+                // without progress a short sleep, and a time limit.
+                int kj = 0, vj = 0;  // next K / V step of the item to load
+                uint64_t idle_since = 0;
+                while (vj < n) {
+                    bool progressed = false;
+                    if (kj < n && mbar_test(smem_addr(&b.k_empty[kst]), kph ^ 1u)) {
+                        const int t = step_tile(p, list, kj);
+                        if (t >= 0) {
+                            mbar_arrive_expect_tx(smem_addr(&b.k_full[kst]), p.tk * HD * 2);
+                            tma_load_3d(smem_addr(b.k[kst]), &tm_k, smem_addr(&b.k_full[kst]), 0, t * p.tk, h);
+                        } else {
+                            mbar_arrive_expect_tx(smem_addr(&b.k_full[kst]), TILE_BYTES);
+                            tma_load_3d(smem_addr(b.k[kst]), &tm_kb, smem_addr(&b.k_full[kst]), 0, (kj - p.k) * BN, h);
+                        }
+                        k_issued |= 1u << kst;
+                        k_par = (k_par & ~(1u << kst)) | (kph << kst);
+                        if (++kst == K_STAGES) { kst = 0; kph ^= 1u; }
+                        ++kj;
+                        progressed = true;
                     }
-                    k_issued |= 1u << kst;
-                    k_par = (k_par & ~(1u << kst)) | (kph << kst);
-                    if (++kst == K_STAGES) { kst = 0; kph ^= 1u; }
-                    if (!mbar_wait_sleep(smem_addr(&b.v_empty[vst]), vph ^ 1u, wc, SLEEP_NS)) { ok = false; break; }
-                    if (t >= 0) {
-                        mbar_arrive_expect_tx(smem_addr(&b.v_full[vst]), p.tk * HD * 2);
-                        tma_load_3d(smem_addr(b.v[vst]), &tm_v, smem_addr(&b.v_full[vst]), 0, t * p.tk, h);
-                    } else {
-                        mbar_arrive_expect_tx(smem_addr(&b.v_full[vst]), TILE_BYTES);
-                        tma_load_3d(smem_addr(b.v[vst]), &tm_vb, smem_addr(&b.v_full[vst]), 0, (j - p.k) * BN, h);
+                    if (vj < kj && mbar_test(smem_addr(&b.v_empty[vst]), vph ^ 1u)) {
+                        const int t = step_tile(p, list, vj);
+                        if (t >= 0) {
+                            mbar_arrive_expect_tx(smem_addr(&b.v_full[vst]), p.tk * HD * 2);
+                            tma_load_3d(smem_addr(b.v[vst]), &tm_v, smem_addr(&b.v_full[vst]), 0, t * p.tk, h);
+                        } else {
+                            mbar_arrive_expect_tx(smem_addr(&b.v_full[vst]), TILE_BYTES);
+                            tma_load_3d(smem_addr(b.v[vst]), &tm_vb, smem_addr(&b.v_full[vst]), 0, (vj - p.k) * BN, h);
+                        }
+                        v_issued |= 1u << vst;
+                        v_par = (v_par & ~(1u << vst)) | (vph << vst);
+                        if (++vst == V_STAGES) { vst = 0; vph ^= 1u; }
+                        ++vj;
+                        progressed = true;
                     }
-                    v_issued |= 1u << vst;
-                    v_par = (v_par & ~(1u << vst)) | (vph << vst);
-                    if (++vst == V_STAGES) { vst = 0; vph ^= 1u; }
+                    if (progressed) {
+                        idle_since = 0;
+                        continue;
+                    }
+                    const uint64_t now = globaltimer_ns();
+                    if (idle_since == 0) idle_since = now;
+                    if (*wc.abort_flag) { ok = false; break; }
+                    if (now - idle_since > p.timeout_ns) {
+                        flag_status(p.status, ZB_ERR_TIMEOUT);
+                        *wc.abort_flag = 1;
+                        ok = false;
+                        break;
+                    }
+                    __nanosleep(64);
                 }
             }
             // arrive at the barriers of the rounds this CTA does not run (so the
@@ -465,43 +493,40 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                             if (e >= valid) x[e] = -INFINITY;
                     }
                 } else {
-                    // landmark chunk: x = s * scale + log2(n_j), or -inf for
-                    // selected tiles (from the item's bitmap) and for columns
-                    // past the last tile
+                    // landmark chunk: x = s * scale + log2(t), or -inf for selected
+                    // tiles (from the item's bitmap) and for columns past the last
+                    // tile; the ragged last tile's landmark (in the item's last
+                    // chunk) then gets log2(n_last) instead
                     const int j0 = (j - p.k) * BN;
                     if (j == p.k) {  // first landmark step: every thread's bits are in
                         if (!mbar_wait(smem_addr(&sm.bm_ready[s][r & 1]), (r >> 1) & 1, wc)) { ok = false; break; }
                     }
-#pragma unroll 1
+                    uint32_t bits[BN / 32];
+#pragma unroll
                     for (int w = 0; w < BN / 32; ++w) {
                         const int jw = j0 + w * 32;
-                        uint32_t bits = jw < p.Tk ? bm[jw >> 5] : 0u;
+                        bits[w] = jw < p.Tk ? bm[jw >> 5] : 0u;
                         const int keep = p.Tk - jw;  // columns >= keep are beyond the last tile
-                        if (keep < 32) bits |= keep <= 0 ? 0xFFFFFFFFu : (0xFFFFFFFFu << keep);
-                        const int lastc = p.Tk - 1 - jw;  // column of the ragged last tile
-                        // bias of this 32-column word, applied under a switch on w so
-                        // that x stays in registers
-                        switch (w) {
-#define ZB_LM_WORD(W)                                                                      \
-    case W:                                                                                \
-        _Pragma("unroll") for (int e = 0; e < 32; e += 2) {                                \
-            const float b0 = ((bits >> e) & 1u) ? -INFINITY                                \
-                                                : (e == lastc ? p.log2_last : p.log2_tk);  \
-            const float b1 = ((bits >> (e + 1)) & 1u) ? -INFINITY                          \
-                                                      : (e + 1 == lastc ? p.log2_last : p.log2_tk); \
-            float v0, v1;                                                                  \
-            f2_unpack(f2_fma(f2_pack(x[W * 32 + e], x[W * 32 + e + 1]), c2,                \
-                             f2_pack(b0, b1)), v0, v1);                                    \
-            x[W * 32 + e] = v0;                                                            \
-            x[W * 32 + e + 1] = v1;                                                        \
-        }                                                                                  \
-        break;
-                            ZB_LM_WORD(0)
-                            ZB_LM_WORD(1)
-                            ZB_LM_WORD(2)
-                            ZB_LM_WORD(3)
-#undef ZB_LM_WORD
+                        if (keep < 32) bits[w] |= keep <= 0 ? 0xFFFFFFFFu : (0xFFFFFFFFu << keep);
+                    }
+                    const float lt = p.log2_tk;
+#pragma unroll
+                    for (int w = 0; w < BN / 32; ++w) {
+#pragma unroll
+                        for (int e = 0; e < 32; e += 2) {
+                            const float b0 = ((bits[w] >> e) & 1u) ? -INFINITY : lt;
+                            const float b1 = ((bits[w] >> (e + 1)) & 1u) ? -INFINITY : lt;
+                            float v0, v1;
+                            f2_unpack(f2_fma(f2_pack(x[w * 32 + e], x[w * 32 + e + 1]), c2, f2_pack(b0, b1)), v0, v1);
+                            x[w * 32 + e] = v0;
+                            x[w * 32 + e + 1] = v1;
                         }
+                    }
+                    if (j == n - 1 && p.n_last != p.tk) {  // once per item
+                        const int lastc = p.Tk - 1 - j0;
+                        const float dl = p.log2_last - p.log2_tk;
+#pragma unroll
+                        for (int e = 0; e < BN; ++e) x[e] += e == lastc ? dl : 0.f;
                     }
                 }
                 // ---- row max: a tree of 3-input max (selected tiles: of the
@@ -547,8 +572,9 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                         tmem_wait_st();
                     }
                 }
-                // ---- p = 2^(x * scale - m): packed fp32x2 arithmetic, exponentials
-                // on MUFU, two partial sums, bf16 pairs to TMEM per 32 columns
+                // ---- p = 2^(x * scale - m): packed fp32x2 arithmetic, 1 of every
+                // 4 pairs on the FMA pipes (polynomial) and the rest on MUFU, two
+                // partial sums, bf16 pairs to TMEM per 32 columns
                 uint64_t acc0 = 0ull, acc1 = 0ull;
 #pragma unroll
                 for (int c = 0; c < BN / 32; ++c) {
@@ -556,9 +582,14 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
 #pragma unroll
                     for (int q = 0; q < 16; ++q) {
                         const uint64_t xs = f2_fma(f2_pack(x[c * 32 + 2 * q], x[c * 32 + 2 * q + 1]), cm2, nm2);
-                        float a0, a1;
-                        f2_unpack(xs, a0, a1);
-                        const uint64_t pv = f2_pack(ex2(a0), ex2(a1));
+                        uint64_t pv;
+                        if ((q & 3) == 1) {
+                            pv = f2_exp2_poly(xs);
+                        } else {
+                            float a0, a1;
+                            f2_unpack(xs, a0, a1);
+                            pv = f2_pack(ex2(a0), ex2(a1));
+                        }
                         if (q & 1) acc1 = f2_add(acc1, pv); else acc0 = f2_add(acc0, pv);
                         float p0, p1;
                         f2_unpack(pv, p0, p1);
