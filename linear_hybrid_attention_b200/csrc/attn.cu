@@ -183,6 +183,10 @@ ZB_DEVINL int step_tile(const Params& p, const int32_t* list, int j) {
     return t < 0 ? 0 : (t >= p.Tk ? p.Tk - 1 : t);
 }
 
+// LM: whether the launch has landmark chunks.  The launches without (dense
+// attention, tile-sparse without landmarks) use an instantiation that holds no
+// landmark code at all, which keeps their step loop short.
+template <bool LM>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
 sparse_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                    const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_kb,
@@ -483,7 +487,7 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                 }
                 tc_fence_before();
                 mbar_arrive(smem_addr(&b.s_free));  // S is in registers: the next Q K^T may overwrite it
-                const bool is_lm = j >= p.k;
+                const bool is_lm = LM && j >= p.k;
                 if (!is_lm) {
                     // selected tile: mask the columns past the tile's length
                     const int valid = (j == p.k - 1) ? last_valid : p.tk;
@@ -492,7 +496,7 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                         for (int e = 0; e < BN; ++e)
                             if (e >= valid) x[e] = -INFINITY;
                     }
-                } else {
+                } else if constexpr (LM) {
                     // landmark chunk: x = s * scale + log2(t), or -inf for selected
                     // tiles (from the item's bitmap) and for columns past the last
                     // tile; the ragged last tile's landmark (in the item's last
@@ -723,27 +727,31 @@ static zb_status launch_attn(const uint16_t* Q, const uint16_t* K, const uint16_
     {
         std::lock_guard<std::mutex> lock(regs_mu);
         if (regs_ok < 0) {
-            cudaFuncAttributes fa;
-            if (cudaFuncGetAttributes(&fa, sparse_attn_kernel) != cudaSuccess) return ZB_ERR_CUDA;
-            regs_ok = fa.numRegs == LAUNCH_REGS ? 1 : 0;
+            cudaFuncAttributes fa, fb;
+            if (cudaFuncGetAttributes(&fa, sparse_attn_kernel<true>) != cudaSuccess) return ZB_ERR_CUDA;
+            if (cudaFuncGetAttributes(&fb, sparse_attn_kernel<false>) != cudaSuccess) return ZB_ERR_CUDA;
+            regs_ok = (fa.numRegs == LAUNCH_REGS && fb.numRegs == LAUNCH_REGS) ? 1 : 0;
         }
         if (!regs_ok) return ZB_ERR_UNSUPPORTED;
     }
+    const void* kern = lm_chunks ? reinterpret_cast<const void*>(sparse_attn_kernel<true>)
+                                 : reinterpret_cast<const void*>(sparse_attn_kernel<false>);
     const size_t smem = attn_smem_bytes();
-    cudaError_t ce = cudaFuncSetAttribute(sparse_attn_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                          static_cast<int>(smem));
+    cudaError_t ce = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
     if (ce != cudaSuccess) return ZB_ERR_CUDA;
     const long long grid = p.n_items < dev.sm_count ? p.n_items : dev.sm_count;
     if (!wave) {
-        sparse_attn_kernel<<<static_cast<unsigned>(grid), NUM_THREADS, smem, st>>>(mq, mk, mv, mkb, mvb, p);
+        if (lm_chunks)
+            sparse_attn_kernel<true><<<static_cast<unsigned>(grid), NUM_THREADS, smem, st>>>(mq, mk, mv, mkb, mvb, p);
+        else
+            sparse_attn_kernel<false><<<static_cast<unsigned>(grid), NUM_THREADS, smem, st>>>(mq, mk, mv, mkb, mvb, p);
         return cudaGetLastError() == cudaSuccess ? ZB_OK : ZB_ERR_CUDA;
     }
     // The wave barriers need every CTA resident at once: zero the counters in
     // stream order, then a cooperative launch (which guarantees co-residency).
     if (cudaMemsetAsync(wave, 0, sizeof(unsigned), st) != cudaSuccess) return ZB_ERR_CUDA;
     void* args[] = {&mq, &mk, &mv, &mkb, &mvb, &p};
-    ce = cudaLaunchCooperativeKernel(reinterpret_cast<const void*>(sparse_attn_kernel),
-                                     dim3(static_cast<unsigned>(grid)), dim3(NUM_THREADS), args, smem, st);
+    ce = cudaLaunchCooperativeKernel(kern, dim3(static_cast<unsigned>(grid)), dim3(NUM_THREADS), args, smem, st);
     return ce == cudaSuccess ? ZB_OK : ZB_ERR_CUDA;
 }
 
