@@ -36,6 +36,7 @@
 #include <cuda_runtime.h>
 
 #include <mutex>
+#include <type_traits>
 
 #include "zb_common.cuh"
 #include "zb_host.h"
@@ -472,8 +473,12 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
             }
             float m = -INFINITY;  // running max of the log2-domain logits (lazy)
             float l = 0.f;        // running sum of 2^(x - m)
-            for (int j = 0; j < n; ++j, ph ^= 1u) {
-                if (!mbar_wait(smem_addr(&b.s_full), ph, wc)) { ok = false; break; }
+            // One step (key tile or landmark chunk j), as a generic lambda so that
+            // the selected tiles and the landmark chunks each get a loop of
+            // their own (the selected-tile loop holds no landmark code).
+            auto step = [&](auto lm_tag, int j) -> bool {
+                constexpr bool is_lm = decltype(lm_tag)::value;
+                if (!mbar_wait(smem_addr(&b.s_full), ph, wc)) return false;
                 tc_fence_after();
                 float x[BN];
                 {
@@ -487,8 +492,7 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                 }
                 tc_fence_before();
                 mbar_arrive(smem_addr(&b.s_free));  // S is in registers: the next Q K^T may overwrite it
-                const bool is_lm = LM && j >= p.k;
-                if (!is_lm) {
+                if constexpr (!is_lm) {
                     // selected tile: mask the columns past the tile's length
                     const int valid = (j == p.k - 1) ? last_valid : p.tk;
                     if (valid < BN) {
@@ -496,14 +500,14 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                         for (int e = 0; e < BN; ++e)
                             if (e >= valid) x[e] = -INFINITY;
                     }
-                } else if constexpr (LM) {
+                } else {
                     // landmark chunk: x = s * scale + log2(t), or -inf for selected
                     // tiles (from the item's bitmap) and for columns past the last
                     // tile; the ragged last tile's landmark (in the item's last
                     // chunk) then gets log2(n_last) instead
                     const int j0 = (j - p.k) * BN;
                     if (j == p.k) {  // first landmark step: every thread's bits are in
-                        if (!mbar_wait(smem_addr(&sm.bm_ready[s][r & 1]), (r >> 1) & 1, wc)) { ok = false; break; }
+                        if (!mbar_wait(smem_addr(&sm.bm_ready[s][r & 1]), (r >> 1) & 1, wc)) return false;
                     }
                     uint32_t bits[BN / 32];
 #pragma unroll
@@ -562,7 +566,7 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                 const uint64_t cm2 = is_lm ? f2_pack(1.f, 1.f) : c2;  // landmark logits are already scaled
                 // P is free once P V of the previous step is done; O then holds
                 // every earlier step and can be rescaled
-                if (!mbar_wait(smem_addr(&b.p_free), ph ^ 1u, wc)) { ok = false; break; }
+                if (!mbar_wait(smem_addr(&b.p_free), ph ^ 1u, wc)) return false;
                 tc_fence_after();
                 if (rescale && j > 0) {
 #pragma unroll 1
@@ -609,6 +613,11 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                 tmem_wait_st();
                 tc_fence_before();
                 mbar_arrive(smem_addr(&b.p_full));
+                return true;
+            };
+            for (int j = 0; j < p.k && ok; ++j, ph ^= 1u) ok = step(std::false_type{}, j);
+            if constexpr (LM) {
+                for (int j = p.k; j < n && ok; ++j, ph ^= 1u) ok = step(std::true_type{}, j);
             }
             if (!ok) break;
             // ------------------------------------------------ epilogue ----
