@@ -61,6 +61,25 @@ inline size_t state_ws_bytes(int heads, long long n) {
     return static_cast<size_t>(g.pairs) * g.chunks * PARTIAL_FLOATS * sizeof(float);
 }
 
+ZB_DEVINL void named_bar_sync(int id, int threads) {
+    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(threads) : "memory");
+}
+
+// phi on a bf16 pair, in bf16 arithmetic (the result feeds a bf16 MMA operand):
+// max(x, 0) + 2^(min(x, 0) * log2(e)).  log2(e) rounded to bf16 (1.4453125)
+// perturbs e^x by a relative |x| * 1.8e-3, below the bf16 rounding of the
+// result for |x| < 2 and on outputs that are small for larger |x|.
+ZB_DEVINL uint32_t phi_bf16x2(uint32_t w) {
+    constexpr uint32_t kLog2eBf16x2 = 0x3FB93FB9u;
+    uint32_t pos, neg, e, r;
+    asm("max.bf16x2 %0, %1, %2;" : "=r"(pos) : "r"(w), "r"(0u));
+    asm("min.bf16x2 %0, %1, %2;" : "=r"(neg) : "r"(w), "r"(0u));
+    asm("mul.rn.bf16x2 %0, %1, %2;" : "=r"(neg) : "r"(neg), "r"(kLog2eBf16x2));
+    asm("ex2.approx.ftz.bf16x2 %0, %1;" : "=r"(e) : "r"(neg));
+    asm("add.rn.bf16x2 %0, %1, %2;" : "=r"(r) : "r"(pos), "r"(e));
+    return r;
+}
+
 // phi(x) = elu(x) + 1 = max(x, 0) + exp(min(x, 0))  (x + 1 for x > 0, e^x otherwise)
 __device__ __forceinline__ float phi(float x) {
     return fmaxf(x, 0.f) + ex2(fminf(x, 0.f) * 1.4426950408889634f);
@@ -272,26 +291,47 @@ __global__ void linear_state_reduce_kernel(const float* __restrict__ partial, in
 }
 
 // ============================================================== apply ====
-constexpr int AP_STAGES = 4;
-constexpr int AP_THREADS = 256;  // 8 warps: the phi pass spreads over all; two threads per output row
+// Warp-specialised, one persistent CTA per SM, each with a contiguous range of
+// (head, 128-row tile) items:
+//   warp 0       TMA producer of the Q tiles (ring of AP_STAGES);
+//   warp 1       MMA issuer: D[128 x 80] = phi(Q) B^T into one of D_BUFS TMEM
+//                accumulators (80 of 128 columns each);
+//   warps 2..7   phi in place on each Q tile in shared memory; warps 4..7
+//                also build the B operand / bias of each new head;
+//   warps 8..11  epilogue: one thread per row, O = D[:64] / D[64] + b', each
+//                thread writing its whole 128-byte bf16 row.
+// The roles only meet at mbarriers, so loads, phi, MMA and stores of
+// successive tiles overlap.
+constexpr int AP_STAGES = 6;
+constexpr int AP_THREADS = 384;
+constexpr int D_BUFS = 4;
 constexpr int BN_ROWS = 80;  // 64 columns of S A, one of z, 15 of zeros
 constexpr uint32_t B_BYTES = BN_ROWS * 128;
+constexpr int PHI_BAR = 1;   // named barrier of the operand builders (warps 4..7, 128 threads)
+constexpr int PHI_THREADS = 192;  // warps 2..7 apply phi
+constexpr int EPI_BAR = 2;        // named barrier of the epilogue warps (128 threads)
 
 struct ApplySmem {
     uint8_t q[AP_STAGES][TILE_BYTES];
+    uint8_t ost[2][TILE_BYTES];   // output tiles (128-byte swizzle) for the TMA store
     uint8_t bop[2][B_BYTES];
     float bvec[2][HD];
     float cvec[HD];
-    uint64_t full[AP_STAGES], mma_done[2], drain;
+    uint64_t q_full[AP_STAGES], q_empty[AP_STAGES], phi_done[AP_STAGES];
+    uint64_t mma_done[D_BUFS], d_free[D_BUFS];
+    uint64_t b_free[2];       // MMAs of the last head that used bop / bvec [i] are done
+    uint64_t bvec_ready[2];   // bvec [i] written for its head
+    uint64_t bvec_free[2];    // the epilogue is past the last head that read bvec [i]
+    uint64_t drain;
     uint32_t tmem_base;
     int abort_flag;
 };
 
-__global__ void __launch_bounds__(AP_THREADS, 2)
-linear_apply_kernel(const __grid_constant__ CUtensorMap tm_q, int heads, long long n_q,
-                    const float* __restrict__ S, const float* __restrict__ z,
-                    const float* __restrict__ A, const float* __restrict__ bias,
-                    uint16_t* __restrict__ O, int* status, unsigned long long timeout_ns) {
+__global__ void __launch_bounds__(AP_THREADS, 1)
+linear_apply_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_o,
+                    int heads, long long n_q, const float* __restrict__ S, const float* __restrict__ z,
+                    const float* __restrict__ A, const float* __restrict__ bias, int* status,
+                    unsigned long long timeout_ns) {
     extern __shared__ uint8_t smem_raw[];
     ApplySmem& sm = *reinterpret_cast<ApplySmem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -305,186 +345,263 @@ linear_apply_kernel(const __grid_constant__ CUtensorMap tm_q, int heads, long lo
 
     if (tid == 0) {
         sm.abort_flag = 0;
-        for (int s = 0; s < AP_STAGES; ++s) mbar_init(smem_addr(&sm.full[s]), 1);
-        for (int s = 0; s < 2; ++s) mbar_init(smem_addr(&sm.mma_done[s]), 1);
+        for (int s = 0; s < AP_STAGES; ++s) {
+            mbar_init(smem_addr(&sm.q_full[s]), 1);
+            mbar_init(smem_addr(&sm.q_empty[s]), 1);
+            mbar_init(smem_addr(&sm.phi_done[s]), PHI_THREADS);
+        }
+        for (int d = 0; d < D_BUFS; ++d) {
+            mbar_init(smem_addr(&sm.mma_done[d]), 1);
+            mbar_init(smem_addr(&sm.d_free[d]), 128);
+        }
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(smem_addr(&sm.b_free[i]), 1);
+            mbar_init(smem_addr(&sm.bvec_ready[i]), 128);
+            mbar_init(smem_addr(&sm.bvec_free[i]), 128);
+        }
         mbar_init(smem_addr(&sm.drain), 1);
         fence_mbar_init();
         tma_prefetch_desc(&tm_q);
     }
-    if (warp == 0) tmem_alloc(smem_addr(&sm.tmem_base), 256);
+    if (warp == 1) tmem_alloc(smem_addr(&sm.tmem_base), 512);
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = sm.tmem_base;
+    auto head_of = [&](int it) { return static_cast<int>((first + it) / Tn); };
 
-    auto issue_load = [&](int it) {
-        const long long item = first + it;
-        const int h = static_cast<int>(item / Tn), t = static_cast<int>(item % Tn);
-        const int s = it % AP_STAGES;
-        const uint32_t bar = smem_addr(&sm.full[s]);
-        mbar_arrive_expect_tx(bar, TILE_BYTES);
-        tma_load_3d(smem_addr(sm.q[s]), &tm_q, bar, 0, t * TILE, h);
-    };
-    uint32_t issued = 0;
-    if (tid == 0)
-        for (int it = 0; it < AP_STAGES && it < cnt; ++it) issue_load(it), ++issued;
-
-    constexpr uint32_t IDESC = idesc_bf16(128, BN_ROWS, 0, 0);
-    const int cg = tid & 7, rbase = tid >> 3;
-    const uint32_t lane_addr = static_cast<uint32_t>((warp & 3) * 32) << 16;  // warps w and w + 4 share lanes
-    int h_prev = -1;
-    int consumed = 0;
-    bool ok = true;
-
-    // epilogue of item `it`: O row = D[:64] / D[64] + b
-    auto epilogue = [&](int it) -> bool {
-        const int buf = it & 1;
-        if (!mbar_wait(smem_addr(&sm.mma_done[buf]), (it >> 1) & 1, wc)) return false;
-        tc_fence_after();
-        // this thread: row (warp & 3) * 32 + lane, output columns [32 half, 32 half + 32)
-        const int half = warp >> 2;
-        uint32_t r[32], den;
-        const uint32_t ta = tmem + lane_addr + buf * 128;
-        tmem_ld32(ta + half * 32, r);
-        asm volatile("tcgen05.ld.sync.aligned.32x32b.x1.b32 {%0}, [%1];" : "=r"(den) : "r"(ta + 64));
-        tmem_wait_ld_dep(r);
-        asm volatile("tcgen05.wait::ld.sync.aligned;" : "+r"(den)::"memory");
-        tc_fence_before();
-        const long long item = first + it;
-        const int h = static_cast<int>(item / Tn), t = static_cast<int>(item % Tn);
-        const long long row = static_cast<long long>(t) * TILE + (warp & 3) * 32 + lane;
-        if (row < n_q) {
-            const float inv = 1.f / __uint_as_float(den);
-            uint4* dst = reinterpret_cast<uint4*>(O + (static_cast<long long>(h) * n_q + row) * HD + half * 32);
-            const float* bb = sm.bvec[h & 1] + half * 32;
-#pragma unroll
-            for (int c = 0; c < 4; ++c) {
-                float o[8];
-#pragma unroll
-                for (int e = 0; e < 8; ++e) o[e] = fmaf(__uint_as_float(r[c * 8 + e]), inv, bb[c * 8 + e]);
-                dst[c] = make_uint4(pack_bf16x2(o[0], o[1]), pack_bf16x2(o[2], o[3]),
-                                    pack_bf16x2(o[4], o[5]), pack_bf16x2(o[6], o[7]));
+    if (warp == 0) {
+        if (lane == 0) {
+            // =============================================== producer ====
+            uint32_t issued = 0, consumed_par = 0, issued_mask = 0;
+            bool ok = true;
+            for (int it = 0; it < cnt && ok; ++it) {
+                const int s = it % AP_STAGES;
+                const uint32_t use = static_cast<uint32_t>(it / AP_STAGES);
+                if (!mbar_wait_sleep(smem_addr(&sm.q_empty[s]), (use & 1) ^ 1, wc, 20000)) { ok = false; break; }
+                const long long item = first + it;
+                const int h = static_cast<int>(item / Tn), t = static_cast<int>(item % Tn);
+                mbar_arrive_expect_tx(smem_addr(&sm.q_full[s]), TILE_BYTES);
+                tma_load_3d(smem_addr(sm.q[s]), &tm_q, smem_addr(&sm.q_full[s]), 0, t * TILE, h);
+                issued_mask |= 1u << s;
+                consumed_par = (consumed_par & ~(1u << s)) | ((use & 1u) << s);
+                ++issued;
             }
+            // leave no TMA write in flight (bounded, even after an abort)
+            volatile int no_abort = 0;
+            const WaitCtx w2{status, &no_abort, timeout_ns};
+            for (int s = 0; s < AP_STAGES; ++s)
+                if ((issued_mask >> s) & 1u) mbar_wait(smem_addr(&sm.q_full[s]), (consumed_par >> s) & 1u, w2);
         }
-        return true;
-    };
-
-    for (int it = 0; it < cnt; ++it) {
-        const long long item = first + it;
-        const int h = static_cast<int>(item / Tn);
-        if (h != h_prev) {
-            // B operand of head h into buffer (h & 1), K-major, 128-byte swizzle:
-            // rows n < 64 hold ((S - z c^T) A)[:, n], row 64 holds z, rows
-            // 65..79 zero; the bias becomes b' = c A + b.  Centring on
-            // c = 1^T S / 1^T z (the output for phi(q) = 1) is an exact identity
-            // (phi(q) z c^T / (phi(q) . z) = c^T) that keeps the bf16 operand
-            // small, so rounding it does not cancel against b'.
-            uint8_t* bo = sm.bop[h & 1];
-            const float* Sh = S + static_cast<size_t>(h) * HD * HD;
-            const float* zh = z + static_cast<size_t>(h) * HD;
-            const float* Ah = A ? A + static_cast<size_t>(h) * HD * HD : nullptr;
-            if (tid < HD) {
-                float cs = 0.f, zs = 0.f;
-                for (int k = 0; k < HD; ++k) {
-                    cs += __ldg(Sh + k * HD + tid);
-                    zs += __ldg(zh + k);
+        __syncwarp();
+    } else if (warp == 1) {
+        if (lane == 0) {
+            // ================================================= MMA issuer ====
+            constexpr uint32_t IDESC = idesc_bf16(128, BN_ROWS, 0, 0);
+            int h_prev = -1, nb = -1;  // head of the previous item, builds seen so far - 1
+            bool ok = true;
+            for (int it = 0; it < cnt && ok; ++it) {
+                const int h = head_of(it);
+                if (h != h_prev) {
+                    if (nb >= 0) umma_commit(smem_addr(&sm.b_free[nb & 1]));  // the previous head's B is done with
+                    ++nb;
+                    h_prev = h;
                 }
-                sm.cvec[tid] = cs / zs;
+                const int s = it % AP_STAGES, d = it % D_BUFS;
+                const uint32_t use = static_cast<uint32_t>(it / AP_STAGES), du = static_cast<uint32_t>(it / D_BUFS);
+                if (!mbar_wait_sleep(smem_addr(&sm.phi_done[s]), use & 1, wc, 20000)) { ok = false; break; }
+                if (!mbar_wait_sleep(smem_addr(&sm.d_free[d]), (du & 1) ^ 1, wc, 20000)) { ok = false; break; }
+                tc_fence_after();
+                const uint32_t a0 = smem_addr(sm.q[s]);
+                const uint32_t b0 = smem_addr(sm.bop[nb & 1]);
+#pragma unroll
+                for (int kk = 0; kk < HD / 16; ++kk) {
+                    const uint64_t ad = sdesc_sw128(a0 + kk * 32, 16, 1024);
+                    const uint64_t bd = sdesc_sw128(b0 + kk * 32, 16, 1024);
+                    umma_ss(tmem + d * 128, ad, bd, IDESC, kk > 0 ? 1u : 0u);
+                }
+                umma_commit(smem_addr(&sm.mma_done[d]));
+                umma_commit(smem_addr(&sm.q_empty[s]));
             }
-            __syncthreads();
-            if (tid < HD) {
-                float ca = 0.f;
-                for (int m = 0; m < HD; ++m) ca = fmaf(sm.cvec[m], Ah ? __ldg(Ah + m * HD + tid) : (m == tid ? 1.f : 0.f), ca);
-                sm.bvec[h & 1][tid] = ca + (bias ? bias[static_cast<size_t>(h) * HD + tid] : 0.f);
-            }
-            {
-                const int ncol = tid & 63;       // output column n
-                const int kpart = tid >> 6;      // rows k in [16 kpart, 16 kpart + 16)
-                float acol[HD];
-#pragma unroll
-                for (int m = 0; m < HD; ++m) acol[m] = Ah ? __ldg(Ah + m * HD + ncol) : (m == ncol ? 1.f : 0.f);
-                for (int kq = 0; kq < 16; kq += 2) {
-                    float v2[2];
-#pragma unroll
-                    for (int u = 0; u < 2; ++u) {
-                        const int k = kpart * 16 + kq + u;
-                        const float* srow = Sh + k * HD;
-                        const float zk = __ldg(zh + k);
-                        float acc = 0.f;
-#pragma unroll
-                        for (int m = 0; m < HD; ++m) acc = fmaf(fmaf(-zk, sm.cvec[m], __ldg(srow + m)), acol[m], acc);
-                        v2[u] = acc;
+            // no MMA may still run when TMEM is released
+            volatile int no_abort = 0;
+            const WaitCtx w2{status, &no_abort, timeout_ns};
+            umma_commit(smem_addr(&sm.drain));
+            mbar_wait(smem_addr(&sm.drain), 0, w2);
+        }
+        __syncwarp();
+    } else if (warp >= 2 && warp < 8) {
+        // ======================================= phi and per-head operands ====
+        // Every thread runs every iteration (after an abort it skips the waits
+        // and the work but keeps the builders' named barriers matched).
+        const int t = tid - 128;          // builder index (warps 4..7)
+        const int tp = tid - 64;          // phi index (warps 2..7)
+        const bool builder = warp >= 4;
+        int h_prev = -1, nb = -1;
+        bool ok = true;
+        for (int it = 0; it < cnt; ++it) {
+            const int h = head_of(it);
+            if (h != h_prev && !builder) h_prev = h;
+            if (h != h_prev) {
+                ++nb;
+                h_prev = h;
+                const int hb = nb & 1;
+                // bop / bvec [hb] were last used by the head two builds ago: its MMAs
+                // and its epilogue must be done with them
+                if (ok && nb >= 2 && !mbar_wait(smem_addr(&sm.b_free[hb]), ((nb - 2) >> 1) & 1, wc)) ok = false;
+                if (ok && nb >= 2 && !mbar_wait(smem_addr(&sm.bvec_free[hb]), ((nb - 2) >> 1) & 1, wc)) ok = false;
+                // B operand of head h, K-major, 128-byte swizzle: rows n < 64 hold
+                // ((S - z c^T) A)[:, n], row 64 holds z, rows 65..79 zero; the bias
+                // becomes b' = c A + b.  Centring on c = 1^T S / 1^T z (the output
+                // for phi(q) = 1) is an exact identity (phi(q) z c^T / (phi(q) . z)
+                // = c^T) that keeps the bf16 operand small, so rounding it does not
+                // cancel against b'.
+                uint8_t* bo = sm.bop[hb];
+                const float* Sh = S + static_cast<size_t>(h) * HD * HD;
+                const float* zh = z + static_cast<size_t>(h) * HD;
+                const float* Ah = A ? A + static_cast<size_t>(h) * HD * HD : nullptr;
+                if (ok && t < HD) {
+                    float cs = 0.f, zs = 0.f;
+                    for (int k = 0; k < HD; ++k) {
+                        cs += __ldg(Sh + k * HD + t);
+                        zs += __ldg(zh + k);
                     }
-                    const int k = kpart * 16 + kq;  // even: both land in one 32-bit word
-                    const int off = ncol * 128 + ((((k >> 3) ^ (ncol & 7))) << 4) + (k & 7) * 2;
-                    *reinterpret_cast<uint32_t*>(bo + off) = pack_bf16x2(v2[0], v2[1]);
+                    sm.cvec[t] = cs / zs;
+                }
+                named_bar_sync(PHI_BAR, 128);
+                if (ok && t < HD) {
+                    float ca = 0.f;
+                    for (int m = 0; m < HD; ++m) ca = fmaf(sm.cvec[m], Ah ? __ldg(Ah + m * HD + t) : (m == t ? 1.f : 0.f), ca);
+                    sm.bvec[hb][t] = ca + (bias ? bias[static_cast<size_t>(h) * HD + t] : 0.f);
+                }
+                if (ok) {
+                    const int ncol = t & 63;       // output column n
+                    const int kpart = t >> 6;      // rows k in [32 kpart, 32 kpart + 32)
+                    float acol[HD];
+#pragma unroll
+                    for (int m = 0; m < HD; ++m) acol[m] = Ah ? __ldg(Ah + m * HD + ncol) : (m == ncol ? 1.f : 0.f);
+                    for (int kq = 0; kq < 32; kq += 2) {
+                        float v2[2];
+#pragma unroll
+                        for (int u = 0; u < 2; ++u) {
+                            const int k = kpart * 32 + kq + u;
+                            const float* srow = Sh + k * HD;
+                            const float zk = __ldg(zh + k);
+                            float acc = 0.f;
+#pragma unroll
+                            for (int m = 0; m < HD; ++m) acc = fmaf(fmaf(-zk, sm.cvec[m], __ldg(srow + m)), acol[m], acc);
+                            v2[u] = acc;
+                        }
+                        const int k = kpart * 32 + kq;  // even: both land in one 32-bit word
+                        const int off = ncol * 128 + ((((k >> 3) ^ (ncol & 7))) << 4) + (k & 7) * 2;
+                        *reinterpret_cast<uint32_t*>(bo + off) = pack_bf16x2(v2[0], v2[1]);
+                    }
+                    for (int e = t; e < 16 * HD / 2; e += 128) {
+                        // rows 64..79: z then zeros, two values per word
+                        const int rr = 64 + e / (HD / 2);
+                        const int k = (e % (HD / 2)) * 2;
+                        const float a = rr == 64 ? __ldg(zh + k) : 0.f;
+                        const float b2 = rr == 64 ? __ldg(zh + k + 1) : 0.f;
+                        const int off = rr * 128 + ((((k >> 3) ^ (rr & 7))) << 4) + (k & 7) * 2;
+                        *reinterpret_cast<uint32_t*>(bo + off) = pack_bf16x2(a, b2);
+                    }
+                }
+                mbar_arrive(smem_addr(&sm.bvec_ready[hb]));  // bvec [hb] (written by t < 64) is in
+                named_bar_sync(PHI_BAR, 128);  // cvec is reused by the next build
+            }
+            // phi in place on this tile (the whole 16 KB, 128 bytes per thread pass)
+            const int s = it % AP_STAGES;
+            const uint32_t use = static_cast<uint32_t>(it / AP_STAGES);
+            if (ok && !mbar_wait(smem_addr(&sm.q_full[s]), use & 1, wc)) ok = false;
+            if (ok) {
+                // 1,024 16-byte chunks over 192 threads: all loads, then phi, then stores
+                uint8_t* qt = sm.q[s];
+                constexpr int PER = (TILE * 8 + PHI_THREADS - 1) / PHI_THREADS;
+                uint4 v[PER];
+#pragma unroll
+                for (int u = 0; u < PER; ++u) {
+                    const int c = tp + u * PHI_THREADS;
+                    if (c < TILE * 8) v[u] = *reinterpret_cast<const uint4*>(qt + c * 16);
+                }
+#pragma unroll
+                for (int u = 0; u < PER; ++u) {
+                    const int c = tp + u * PHI_THREADS;
+                    if (c < TILE * 8) {
+                        *reinterpret_cast<uint4*>(qt + c * 16) = make_uint4(phi_bf16x2(v[u].x), phi_bf16x2(v[u].y),
+                                                                            phi_bf16x2(v[u].z), phi_bf16x2(v[u].w));
+                    }
                 }
             }
-            for (int e = tid; e < 16 * HD / 2; e += AP_THREADS) {
-                // rows 64..79: z then zeros, two values per word
-                const int rr = 64 + e / (HD / 2);
-                const int k = (e % (HD / 2)) * 2;
-                const float a = rr == 64 ? z[static_cast<size_t>(h) * HD + k] : 0.f;
-                const float b = rr == 64 ? z[static_cast<size_t>(h) * HD + k + 1] : 0.f;
-                const int off = rr * 128 + ((((k >> 3) ^ (rr & 7))) << 4) + (k & 7) * 2;
-                *reinterpret_cast<uint32_t*>(bo + off) = pack_bf16x2(a, b);
+            fence_proxy_async_smem();  // the MMA reads phi(Q) and B through the async proxy
+            mbar_arrive(smem_addr(&sm.phi_done[s]));
+        }
+    } else if (warp >= 8) {
+        // ================================================== epilogue ====
+        // Each thread writes its row into a 128-byte-swizzled staging tile (no
+        // bank conflicts); one thread then stores the tile with TMA (rows past
+        // n_q are not written).  Every thread runs every iteration (after an
+        // abort it skips the waits and the work but keeps the named barriers
+        // matched).
+        const int row = (warp & 3) * 32 + lane;
+        const int et = tid - 256;
+        const uint32_t lane_addr = static_cast<uint32_t>((warp & 3) * 32) << 16;
+        int h_prev = -1, nb = -1;
+        bool ok = true;
+        for (int it = 0; it < cnt; ++it) {
+            const long long item = first + it;
+            const int h = static_cast<int>(item / Tn), t = static_cast<int>(item % Tn);
+            if (h != h_prev) {
+                if (nb >= 0) mbar_arrive(smem_addr(&sm.bvec_free[nb & 1]));  // done with the previous head's bvec
+                ++nb;
+                h_prev = h;
+                if (ok && !mbar_wait(smem_addr(&sm.bvec_ready[nb & 1]), (nb >> 1) & 1, wc)) ok = false;
             }
-            h_prev = h;
-        }
-        const int s = it % AP_STAGES;
-        if (!mbar_wait(smem_addr(&sm.full[s]), (it / AP_STAGES) & 1, wc)) ok = false;
-        else consumed = it + 1;
-        if (ok) {
-            uint8_t* qt = sm.q[s];
+            const int d = it % D_BUFS, ob = it & 1;
+            const uint32_t du = static_cast<uint32_t>(it / D_BUFS);
+            // the store from this staging buffer two tiles ago has read it
+            if (et == 0) bulk_wait_group_read<1>();
+            named_bar_sync(EPI_BAR, 128);
+            if (ok && !mbar_wait(smem_addr(&sm.mma_done[d]), du & 1, wc)) ok = false;
+            if (ok) {
+                tc_fence_after();
+                uint32_t r[64], den;
+                const uint32_t ta = tmem + lane_addr + d * 128;
+                tmem_ld32(ta, sub32(r, 0));
+                tmem_ld32(ta + 32, sub32(r, 32));
+                asm volatile("tcgen05.ld.sync.aligned.32x32b.x1.b32 {%0}, [%1];" : "=r"(den) : "r"(ta + 64));
+                tmem_wait_ld_dep(sub32(r, 0));
+                tmem_wait_ld_dep(sub32(r, 32));
+                asm volatile("tcgen05.wait::ld.sync.aligned;" : "+r"(den)::"memory");
+                tc_fence_before();
+                mbar_arrive(smem_addr(&sm.d_free[d]));
+                const float inv = 1.f / __uint_as_float(den);
+                const float* bb = sm.bvec[nb & 1];
+                uint8_t* orow = sm.ost[ob] + row * 128;
 #pragma unroll
-            for (int m = 0; m < TILE / (AP_THREADS / 8); ++m) {
-                const int r = rbase + (AP_THREADS / 8) * m;
-                uint4* p = reinterpret_cast<uint4*>(qt + r * 128 + ((cg ^ (r & 7)) << 4));
-                uint4 v = *p;
-                uint32_t w[4] = {v.x, v.y, v.z, v.w};
+                for (int c = 0; c < 8; ++c) {
+                    float o[8];
 #pragma unroll
-                for (int e = 0; e < 4; ++e) w[e] = pack_bf16x2(phi(bf16_lo(w[e])), phi(bf16_hi(w[e])));
-                *p = make_uint4(w[0], w[1], w[2], w[3]);
+                    for (int e = 0; e < 8; ++e) o[e] = fmaf(__uint_as_float(r[c * 8 + e]), inv, bb[c * 8 + e]);
+                    *reinterpret_cast<uint4*>(orow + ((c ^ (row & 7)) << 4)) =
+                        make_uint4(pack_bf16x2(o[0], o[1]), pack_bf16x2(o[2], o[3]), pack_bf16x2(o[4], o[5]),
+                                   pack_bf16x2(o[6], o[7]));
+                }
+            }
+            fence_proxy_async_smem();  // the TMA store reads the tile through the async proxy
+            named_bar_sync(EPI_BAR, 128);
+            if (et == 0 && ok) {
+                tma_store_3d(&tm_o, smem_addr(sm.ost[ob]), 0, t * TILE, h);
+                bulk_commit_group();
             }
         }
-        fence_proxy_async_smem();
-        if (__syncthreads_or(!ok)) { ok = false; break; }
-        if (tid == 0) {
-            tc_fence_after();
-            const uint32_t a0 = smem_addr(sm.q[s]);
-            const uint32_t b0 = smem_addr(sm.bop[h & 1]);
-            const uint32_t d = tmem + (it & 1) * 128;
-#pragma unroll
-            for (int kk = 0; kk < HD / 16; ++kk) {
-                const uint64_t ad = sdesc_sw128(a0 + kk * 32, 16, 1024);
-                const uint64_t bd = sdesc_sw128(b0 + kk * 32, 16, 1024);
-                umma_ss(d, ad, bd, IDESC, kk > 0 ? 1u : 0u);
-            }
-            umma_commit(smem_addr(&sm.mma_done[it & 1]));
-        }
-        if (it >= 1) {
-            if (!epilogue(it - 1)) ok = false;
-            // the stage of item it-1 is free (its MMA is done): refill it
-            if (tid == 0 && ok && it - 1 + AP_STAGES < cnt) issue_load(it - 1 + AP_STAGES), ++issued;
-        }
+        if (et == 0) bulk_wait_group<0>();  // every store done before the CTA exits
     }
-    if (ok && cnt > 0) {
-        if (!epilogue(cnt - 1)) ok = false;
-    }
-    // drain: no MMA may run and no TMA may write once TMEM and smem are released
-    if (tid == 0) {
-        volatile int no_abort = 0;
-        const WaitCtx w2{status, &no_abort, timeout_ns};
-        umma_commit(smem_addr(&sm.drain));
-        mbar_wait(smem_addr(&sm.drain), 0, w2);
-        for (uint32_t q = static_cast<uint32_t>(consumed); q < issued; ++q)
-            mbar_wait(smem_addr(&sm.full[q % AP_STAGES]), (q / AP_STAGES) & 1, w2);
-    }
+
     tc_fence_before();
     __syncthreads();
-    if (warp == 0) {
+    if (warp == 1) {
         tc_fence_after();
-        tmem_dealloc(tmem, 256);
+        tmem_dealloc(tmem, 512);
     }
 }
 
@@ -626,16 +743,17 @@ extern "C" zb_status zb_linear_apply(const uint16_t* Q, int32_t heads, int64_t n
             Q, heads, n_q, S, z, A, b, static_cast<float*>(O));
         return cudaGetLastError() == cudaSuccess ? ZB_OK : ZB_ERR_CUDA;
     }
-    CUtensorMap mq;
+    CUtensorMap mq, mo;
     if ((e = make_map_bf16_3d(&mq, Q, 64, n_q, heads, lin::TILE)) != ZB_OK) return e;
+    if ((e = make_map_bf16_3d(&mo, O, 64, n_q, heads, lin::TILE)) != ZB_OK) return e;
     const size_t smem = sizeof(lin::ApplySmem) + 1024;
     if (cudaFuncSetAttribute(lin::linear_apply_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              static_cast<int>(smem)) != cudaSuccess)
         return ZB_ERR_CUDA;
     const long long items = static_cast<long long>(heads) * ((n_q + lin::TILE - 1) / lin::TILE);
-    const long long grid = items < 2ll * dev.sm_count ? items : 2ll * dev.sm_count;
+    const long long grid = items < dev.sm_count ? items : dev.sm_count;
     lin::linear_apply_kernel<<<static_cast<unsigned>(grid), lin::AP_THREADS, smem, st>>>(
-        mq, heads, n_q, S, z, A, b, static_cast<uint16_t*>(O), dev.status, wait_timeout_ns());
+        mq, mo, heads, n_q, S, z, A, b, dev.status, wait_timeout_ns());
     return cudaGetLastError() == cudaSuccess ? ZB_OK : ZB_ERR_CUDA;
 }
 
