@@ -70,7 +70,7 @@ def recorded_traffic(workload: str):
     if fields.get("attn.cu sha256") != sha:
         return None, "kernel changed since the recorded ncu DRAM capture"
     try:
-        return float(fields["dram bytes per launch"]), path
+        return float(fields["dram bytes per launch"]), os.path.relpath(path, ROOT)
     except (KeyError, ValueError):
         return None, "ncu DRAM summary unreadable"
 
