@@ -17,10 +17,12 @@
 //        D[128 x 128] += [phi(K_h0)^T ; phi(K_h1)^T] . [V_h0 | V_h1]
 //    (both operands MN-major); the diagonal 64 x 64 blocks are S_h0, S_h1.
 //    Per-CTA partials are added in a fixed order by a second kernel.
-//  * apply: persistent CTAs over (head, 128-token tile); B = [ (S A)^T ; z ;
-//    0 ] (80 x 64, bf16) is built in shared memory once per head, each tile
-//    computes D[128 x 80] = phi(Q) B^T on the tensor core, and the epilogue
-//    forms D[:, :64] / D[:, 64] + b.
+//  * apply: persistent warp-specialised CTAs over (head, 128-token tile):
+//    B = [ ((S - z c^T) A)^T ; z ; 0 ] (80 x 64, bf16) is built in shared
+//    memory once per head, phi(Q) is applied in place in packed bf16, each
+//    tile computes D[128 x 80] = phi(Q) B^T on the tensor core, and the
+//    epilogue forms D[:, :64] / D[:, 64] + (c A + b) into a staging tile that
+//    is stored with TMA.
 #include <cuda.h>
 #include <cuda_runtime.h>
 
