@@ -6,10 +6,9 @@
 // tile is the pooled query used to score tile pairs.
 //
 // HBM-bound stream: each CTA walks (head, tile) pairs; a tile of one tensor is
-// one contiguous run of n_j rows x 128 bytes, read with 16-byte loads (thread
-// t holds column group t % 8 of rows t / 8, t / 8 + 32, ...), summed in fp64
-// (exact for bf16 inputs unless a tile spans > ~38 binades), reduced in a
-// fixed order, divided by n_j.
+// one contiguous run of n_j rows x 128 bytes, staged in shared memory by bulk
+// copies, summed in fp64 (exact for bf16 inputs unless a tile spans > ~38
+// binades), reduced in a fixed order, divided by n_j.
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
@@ -20,17 +19,8 @@ namespace zb {
 namespace lmk {
 
 constexpr int THREADS = 256;      // gather kernel
-constexpr int LM_THREADS = 512;   // landmark kernel: 16 warps, 8 rows each
+constexpr int LM_THREADS = 544;   // landmark kernel: 16 compute warps (8 rows each) + a producer warp
 constexpr int HD = 64;
-
-__device__ __forceinline__ void add8(double (&acc)[8], const uint4& v) {
-    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-    for (int e = 0; e < 4; ++e) {
-        acc[2 * e] += static_cast<double>(bf16_lo(w[e]));
-        acc[2 * e + 1] += static_cast<double>(bf16_hi(w[e]));
-    }
-}
 
 // Round-to-nearest-even of an fp64 value to bf16 bits, as one rounding: keep
 // the top 8 significant bits of the double's significand (ties to even), then
@@ -47,19 +37,28 @@ __device__ __forceinline__ uint16_t f64_to_bf16_rne(double x) {
 }
 
 // Persistent landmark kernel: one CTA per SM walks (head, tile) items
-// round-robin.  Thread 0 copies the Q, K, V runs of an item (n_j rows x 128 B
-// each, contiguous) into a LM_STAGES-deep shared-memory ring with bulk copies;
-// warp w sums rows [8 w, 8 w + 8) of each tensor, lane l columns 2l, 2l+1,
-// in fp64 (exact for bf16 inputs unless a tile spans > ~38 binades); the 16
-// warp partials are added in a fixed order by 192 threads, one output each.
-// 16 warps per SM hide the latency of the fp32 -> fp64 conversions.
+// round-robin, with roles that meet only at mbarriers (no CTA-wide barrier per
+// tile):
+//   warp 16 (one lane)  copies the Q, K, V runs of an item (n_j rows x 128 B
+//                       each, contiguous) into a LM_STAGES-deep ring with bulk
+//                       copies, once the 16 compute warps have read the stage;
+//   warps 0..15         warp w sums rows [8 w, 8 w + 8) of each tensor, lane l
+//                       columns 2l, 2l+1, in fp64 (exact for bf16 inputs unless
+//                       a tile spans > ~38 binades), into a double-buffered
+//                       partial table; warps 0..5 (192 threads, one output
+//                       each) then add the 16 partials of the item in a fixed
+//                       order and write the means, while the other warps
+//                       already sum the next item.
+// 16 compute warps per SM hide the latency of the fp32 -> fp64 conversions.
 constexpr int LM_STAGES = 3;
+constexpr int LM_WARPS = 16;  // compute warps
 constexpr uint32_t RUN_BYTES = 128 * HD * 2;  // one full tile of one tensor
 
 struct LmSmem {
     uint8_t buf[LM_STAGES][3][RUN_BYTES];
-    double part[2][LM_THREADS / 32][3][HD];
-    uint64_t full[LM_STAGES];
+    double part[2][LM_WARPS][3][HD];
+    uint64_t full[LM_STAGES], empty[LM_STAGES];
+    uint64_t pfull[2], pempty[2];
     int abort_flag;
 };
 
@@ -80,7 +79,14 @@ landmark_kernel(const uint16_t* __restrict__ Q, const uint16_t* __restrict__ K,
     const WaitCtx wc{status, &sm.abort_flag, timeout_ns};
     if (tid == 0) {
         sm.abort_flag = 0;
-        for (int s = 0; s < LM_STAGES; ++s) mbar_init(smem_addr(&sm.full[s]), 1);
+        for (int s = 0; s < LM_STAGES; ++s) {
+            mbar_init(smem_addr(&sm.full[s]), 1);
+            mbar_init(smem_addr(&sm.empty[s]), LM_WARPS);
+        }
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(smem_addr(&sm.pfull[b]), LM_WARPS);
+            mbar_init(smem_addr(&sm.pempty[b]), 3 * HD);
+        }
         fence_mbar_init();
     }
     __syncthreads();
@@ -91,88 +97,109 @@ landmark_kernel(const uint16_t* __restrict__ Q, const uint16_t* __restrict__ K,
         j = static_cast<int>(w % T);
         n = static_cast<int>(min(static_cast<long long>(tile), N - static_cast<long long>(j) * tile));
     };
-    auto issue = [&](int it) {
-        int h, j, n;
-        item_of(it, h, j, n);
-        const int s = it % LM_STAGES;
-        const uint32_t bar = smem_addr(&sm.full[s]);
-        const uint32_t bytes = static_cast<uint32_t>(n) * HD * 2;
-        const long long off = (static_cast<long long>(h) * N + static_cast<long long>(j) * tile) * HD;
-        mbar_arrive_expect_tx(bar, bytes * nt);
-        if (do_q) bulk_load(smem_addr(sm.buf[s][0]), Q + off, bytes, bar);
-        bulk_load(smem_addr(sm.buf[s][1]), K + off, bytes, bar);
-        bulk_load(smem_addr(sm.buf[s][2]), V + off, bytes, bar);
-    };
-    int issued = 0;
-    if (tid == 0)
-        for (int it = 0; it < LM_STAGES && it < cnt; ++it) issue(it), ++issued;
 
-    int consumed = 0;
-    for (int it = 0; it < cnt; ++it) {
-        const int s = it % LM_STAGES;
-        int h, j, n;
-        item_of(it, h, j, n);
-        const bool good = mbar_wait(smem_addr(&sm.full[s]), (it / LM_STAGES) & 1, wc);
-        if (good) consumed = it + 1;
-        const int r0 = warp * 8;
-        const int rows = good ? max(0, min(8, n - r0)) : 0;
+    if (warp == LM_WARPS) {
+        if (lane == 0) {
+            // ================================================= producer ====
+            uint32_t issued_mask = 0, par_mask = 0;
+            for (int it = 0; it < cnt; ++it) {
+                const int s = it % LM_STAGES;
+                const uint32_t use = static_cast<uint32_t>(it / LM_STAGES);
+                if (!mbar_wait_sleep(smem_addr(&sm.empty[s]), (use & 1) ^ 1, wc, 20000)) break;
+                int h, j, n;
+                item_of(it, h, j, n);
+                const uint32_t bar = smem_addr(&sm.full[s]);
+                const uint32_t bytes = static_cast<uint32_t>(n) * HD * 2;
+                const long long off = (static_cast<long long>(h) * N + static_cast<long long>(j) * tile) * HD;
+                mbar_arrive_expect_tx(bar, bytes * nt);
+                if (do_q) bulk_load(smem_addr(sm.buf[s][0]), Q + off, bytes, bar);
+                bulk_load(smem_addr(sm.buf[s][1]), K + off, bytes, bar);
+                bulk_load(smem_addr(sm.buf[s][2]), V + off, bytes, bar);
+                issued_mask |= 1u << s;
+                par_mask = (par_mask & ~(1u << s)) | ((use & 1u) << s);
+            }
+            // leave no bulk copy in flight (bounded, even after an abort)
+            volatile int no_abort = 0;
+            const WaitCtx w2{status, &no_abort, timeout_ns};
+            for (int s = 0; s < LM_STAGES; ++s)
+                if ((issued_mask >> s) & 1u) mbar_wait(smem_addr(&sm.full[s]), (par_mask >> s) & 1u, w2);
+        }
+        __syncwarp();
+    } else {
+        // ============================================ compute warps ====
+        for (int it = 0; it < cnt; ++it) {
+            const int s = it % LM_STAGES, pb = it & 1;
+            const uint32_t use = static_cast<uint32_t>(it / LM_STAGES), pu = static_cast<uint32_t>(it >> 1);
+            int h, j, n;
+            item_of(it, h, j, n);
+            if (!mbar_wait(smem_addr(&sm.full[s]), use & 1, wc)) break;
+            const int r0 = warp * 8;
+            const int rows = max(0, min(8, n - r0));
+            double acc[3][2];
 #pragma unroll
-        for (int t = 0; t < 3; ++t) {
-            double a0 = 0.0, a1 = 0.0;
-            if (t >= t0) {
-                const uint32_t* src = reinterpret_cast<const uint32_t*>(sm.buf[s][t]) + r0 * (HD / 2) + lane;
-                if (rows == 8) {
-                    // all loads first, then a tree of adds (sums are exact, order-free)
-                    uint32_t wv[8];
+            for (int t = 0; t < 3; ++t) {
+                double a0 = 0.0, a1 = 0.0;
+                if (t >= t0) {
+                    const uint32_t* src = reinterpret_cast<const uint32_t*>(sm.buf[s][t]) + r0 * (HD / 2) + lane;
+                    if (rows == 8) {
+                        // all loads first, then a tree of adds (sums are exact, order-free)
+                        uint32_t wv[8];
 #pragma unroll
-                    for (int r = 0; r < 8; ++r) wv[r] = src[r * (HD / 2)];
-                    double l[4], h[4];
+                        for (int r = 0; r < 8; ++r) wv[r] = src[r * (HD / 2)];
+                        double l[4], hh[4];
 #pragma unroll
-                    for (int r = 0; r < 4; ++r) {
-                        l[r] = static_cast<double>(bf16_lo(wv[2 * r])) + static_cast<double>(bf16_lo(wv[2 * r + 1]));
-                        h[r] = static_cast<double>(bf16_hi(wv[2 * r])) + static_cast<double>(bf16_hi(wv[2 * r + 1]));
+                        for (int r = 0; r < 4; ++r) {
+                            l[r] = static_cast<double>(bf16_lo(wv[2 * r])) + static_cast<double>(bf16_lo(wv[2 * r + 1]));
+                            hh[r] = static_cast<double>(bf16_hi(wv[2 * r])) + static_cast<double>(bf16_hi(wv[2 * r + 1]));
+                        }
+                        a0 = (l[0] + l[1]) + (l[2] + l[3]);
+                        a1 = (hh[0] + hh[1]) + (hh[2] + hh[3]);
+                    } else {
+                        for (int r = 0; r < rows; ++r) {
+                            const uint32_t wv = src[r * (HD / 2)];
+                            a0 += static_cast<double>(bf16_lo(wv));
+                            a1 += static_cast<double>(bf16_hi(wv));
+                        }
                     }
-                    a0 = (l[0] + l[1]) + (l[2] + l[3]);
-                    a1 = (h[0] + h[1]) + (h[2] + h[3]);
-                } else {
-                    for (int r = 0; r < rows; ++r) {
-                        const uint32_t wv = src[r * (HD / 2)];
-                        a0 += static_cast<double>(bf16_lo(wv));
-                        a1 += static_cast<double>(bf16_hi(wv));
+                }
+                acc[t][0] = a0;
+                acc[t][1] = a1;
+            }
+            // this warp is done with stage s
+            fence_proxy_async_smem();  // our reads precede the next bulk write into it
+            __syncwarp();
+            if (lane == 0) mbar_arrive(smem_addr(&sm.empty[s]));
+            // partial table pb is free once the item two back was reduced
+            if (!mbar_wait(smem_addr(&sm.pempty[pb]), (pu & 1) ^ 1, wc)) break;
+#pragma unroll
+            for (int t = 0; t < 3; ++t) {
+                sm.part[pb][warp][t][2 * lane] = acc[t][0];
+                sm.part[pb][warp][t][2 * lane + 1] = acc[t][1];
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(smem_addr(&sm.pfull[pb]));
+            if (tid < 3 * HD) {
+                // fixed-order reduction of the 16 partials, one output per thread
+                if (!mbar_wait(smem_addr(&sm.pfull[pb]), pu & 1, wc)) break;
+                const int t = tid / HD, col = tid % HD;
+                double sum = 0.0;
+#pragma unroll
+                for (int wp = 0; wp < LM_WARPS; ++wp) sum += sm.part[pb][wp][t][col];
+                mbar_arrive(smem_addr(&sm.pempty[pb]));
+                if (t >= t0) {
+                    const double mean = sum / static_cast<double>(n);
+                    const long long o = (static_cast<long long>(h) * T + j) * HD + col;
+                    if (t == 0) {
+                        Qbar[o] = mean;
+                    } else if (t == 1) {
+                        Kbar[o] = mean;
+                        Kb16[o] = f64_to_bf16_rne(mean);
+                    } else {
+                        Vb16[o] = f64_to_bf16_rne(mean);
                     }
                 }
             }
-            sm.part[it & 1][warp][t][2 * lane] = a0;
-            sm.part[it & 1][warp][t][2 * lane + 1] = a1;
         }
-        fence_proxy_async_smem();  // our reads of buf[s] precede the next bulk write into it
-        if (__syncthreads_or(!good)) break;
-        if (tid == 0 && it + LM_STAGES < cnt) issue(it + LM_STAGES), ++issued;
-        if (tid < 3 * HD) {
-            const int t = tid / HD, col = tid % HD;
-            if (t >= t0) {
-                double acc = 0.0;
-#pragma unroll
-                for (int wp = 0; wp < LM_THREADS / 32; ++wp) acc += sm.part[it & 1][wp][t][col];
-                const double mean = acc / static_cast<double>(n);
-                const long long o = (static_cast<long long>(h) * T + j) * HD + col;
-                if (t == 0) {
-                    Qbar[o] = mean;
-                } else if (t == 1) {
-                    Kbar[o] = mean;
-                    Kb16[o] = f64_to_bf16_rne(mean);
-                } else {
-                    Vb16[o] = f64_to_bf16_rne(mean);
-                }
-            }
-        }
-    }
-    // leave no bulk copy in flight
-    if (tid == 0) {
-        volatile int no_abort = 0;
-        const WaitCtx w2{status, &no_abort, timeout_ns};
-        for (int q = consumed; q < issued; ++q)
-            mbar_wait(smem_addr(&sm.full[q % LM_STAGES]), (q / LM_STAGES) & 1, w2);
     }
 }
 
