@@ -564,8 +564,33 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                 const float nm = (m == -INFINITY) ? 0.f : -m;
                 const uint64_t nm2 = f2_pack(nm, nm);
                 const uint64_t cm2 = is_lm ? f2_pack(1.f, 1.f) : c2;  // landmark logits are already scaled
+                // ---- p = 2^(x * scale - m): packed fp32x2 scaling, 2^x on MUFU, two
+                // partial row sums, P as bf16 pairs kept in registers until the
+                // previous P V is done
+                uint64_t acc0 = 0ull, acc1 = 0ull;
+                uint32_t pk[BN / 2];
+#pragma unroll
+                for (int c = 0; c < BN / 32; ++c) {
+#pragma unroll
+                    for (int q = 0; q < 16; ++q) {
+                        const uint64_t xs = f2_fma(f2_pack(x[c * 32 + 2 * q], x[c * 32 + 2 * q + 1]), cm2, nm2);
+                        float a0, a1;
+                        f2_unpack(xs, a0, a1);
+                        const uint64_t pv = f2_pack(ex2(a0), ex2(a1));
+                        if (q & 1) acc1 = f2_add(acc1, pv); else acc0 = f2_add(acc0, pv);
+                        float p0, p1;
+                        f2_unpack(pv, p0, p1);
+                        pk[c * 16 + q] = pack_bf16x2(p0, p1);
+                    }
+                }
+                {
+                    float s0, s1;
+                    f2_unpack(f2_add(acc0, acc1), s0, s1);
+                    l += s0 + s1;
+                }
                 // P is free once P V of the previous step is done; O then holds
-                // every earlier step and can be rescaled
+                // every earlier step and can be rescaled (the exponentials above
+                // overlap that P V)
                 if (!mbar_wait(smem_addr(&b.p_free), ph ^ 1u, wc)) return false;
                 tc_fence_after();
                 if (rescale && j > 0) {
@@ -580,36 +605,8 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                         tmem_wait_st();
                     }
                 }
-                // ---- p = 2^(x * scale - m): packed fp32x2 arithmetic, 1 of every
-                // 4 pairs on the FMA pipes (polynomial) and the rest on MUFU, two
-                // partial sums, bf16 pairs to TMEM per 32 columns
-                uint64_t acc0 = 0ull, acc1 = 0ull;
 #pragma unroll
-                for (int c = 0; c < BN / 32; ++c) {
-                    uint32_t pk[16];
-#pragma unroll
-                    for (int q = 0; q < 16; ++q) {
-                        const uint64_t xs = f2_fma(f2_pack(x[c * 32 + 2 * q], x[c * 32 + 2 * q + 1]), cm2, nm2);
-                        uint64_t pv;
-                        if ((q & 3) == 1) {
-                            pv = f2_exp2_poly(xs);
-                        } else {
-                            float a0, a1;
-                            f2_unpack(xs, a0, a1);
-                            pv = f2_pack(ex2(a0), ex2(a1));
-                        }
-                        if (q & 1) acc1 = f2_add(acc1, pv); else acc0 = f2_add(acc0, pv);
-                        float p0, p1;
-                        f2_unpack(pv, p0, p1);
-                        pk[q] = pack_bf16x2(p0, p1);
-                    }
-                    tmem_st16(tm_p + c * 16, pk);
-                }
-                {
-                    float s0, s1;
-                    f2_unpack(f2_add(acc0, acc1), s0, s1);
-                    l += s0 + s1;
-                }
+                for (int c = 0; c < BN / 32; ++c) tmem_st16(tm_p + c * 16, pk + c * 16);
                 tmem_wait_st();
                 tc_fence_before();
                 mbar_arrive(smem_addr(&b.p_full));

@@ -332,41 +332,10 @@ ZB_DEVINL uint64_t f2_add(uint64_t a, uint64_t b) {
     asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
     return d;
 }
-ZB_DEVINL uint64_t f2_add_rm(uint64_t a, uint64_t b) {
-    uint64_t d;
-    asm("add.rm.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
-    return d;
-}
 ZB_DEVINL float fmax3(float a, float b, float c) {
     float d;
     asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
     return d;
-}
-
-// 2^x for two values on the FMA pipes.  Cody-Waite style range reduction
-// 2^x = 2^floor(x) * 2^f with f in [0, 1): floor(x) comes from adding
-// 1.5 * 2^23 with round-toward-minus-infinity (its low mantissa bits then hold
-// floor(x)), 2^f from a cubic that minimises the maximum relative error on
-// [0, 1] with p(0) = 1 (coefficients derived by csrc/exp2_poly.py; max relative
-// error 8.6e-5), and 2^floor(x) is applied by adding floor(x) << 23 to the
-// result's bits.  Inputs are clamped at -127, where the result is exactly 0.
-ZB_DEVINL uint64_t f2_exp2_poly(uint64_t x) {
-    constexpr float kShift = 12582912.0f;  // 1.5 * 2^23
-    constexpr float kC1 = 0.695116758f, kC2 = 0.227644995f, kC3 = 0.0770670399f;
-    float a, b;
-    f2_unpack(x, a, b);
-    const uint64_t xc = f2_pack(fmaxf(a, -127.f), fmaxf(b, -127.f));
-    const uint64_t t = f2_add_rm(xc, f2_pack(kShift, kShift));
-    const uint64_t jf = f2_add(t, f2_pack(-kShift, -kShift));
-    const uint64_t f = f2_fma(jf, f2_pack(-1.f, -1.f), xc);
-    uint64_t p = f2_fma(f2_pack(kC3, kC3), f, f2_pack(kC2, kC2));
-    p = f2_fma(p, f, f2_pack(kC1, kC1));
-    p = f2_fma(p, f, f2_pack(1.f, 1.f));
-    float p0, p1, t0, t1;
-    f2_unpack(p, p0, p1);
-    f2_unpack(t, t0, t1);
-    return f2_pack(__uint_as_float(__float_as_uint(p0) + (__float_as_uint(t0) << 23)),
-                   __uint_as_float(__float_as_uint(p1) + (__float_as_uint(t1) << 23)));
 }
 
 ZB_DEVINL float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
