@@ -233,7 +233,7 @@ zb_status zb_affine_fit(const float* X, const float* Y, int32_t heads,
                         void* ws, size_t ws_bytes, void* stream);
 
 /*
- * Linear-attention state without a workspace.  The paper has no counterpart:
+ * Linear-attention state without a workspace.  The method has no counterpart:
  * this is a service entry point of the library.  Same result as
  * zb_linear_state, for callers that cannot allocate device memory at call
  * time (a process whose device memory is reserved by another allocator, or a

@@ -33,7 +33,9 @@ the top-k tie-break is the lower key-tile index; a landmark's logit carries a
 bias of ln(n_j) (natural log, n_j = tokens in tile j); softmax scale is
 1/sqrt(d); the linear feature map is elu(x)+1 on unscaled q and k,
 non-causal, with no epsilon; the affine map acts on row vectors, y = x A + b,
-fitted by least squares with an intercept.
+fitted by least squares with an intercept; "linear-centered" attention
+centres each head's keys by their mean over all tokens before phi, and leaves
+the queries as they are.
 """
 from __future__ import annotations
 
@@ -46,7 +48,8 @@ __all__ = [
     "tile_lengths", "landmark_means", "tile_scores", "select_tiles",
     "sparse_attention", "dense_attention", "elu_plus_one", "linear_state",
     "linear_apply", "linear_attention", "linear_attention_quadratic", "affine_fit",
-    "affine_apply", "calibration_rows", "RIDGE_REL",
+    "affine_apply", "calibration_rows", "RIDGE_REL", "key_mean", "linear_state_centered",
+    "linear_attention_centered",
 ]
 
 
@@ -241,6 +244,34 @@ def linear_attention_quadratic(Q, K, V) -> np.ndarray:
     W = np.matmul(fq, np.swapaxes(fk, -1, -2))
     W = W / W.sum(axis=-1, keepdims=True)
     return np.matmul(W, _f64(V))
+
+
+def key_mean(K) -> np.ndarray:
+    """mu_h = (1/N) sum_r k_r, the mean key of each head over all N tokens -> [H, d] (fp64)."""
+    K = _f64(K)
+    return K.sum(axis=-2) / K.shape[-2]
+
+
+def linear_state_centered(K, V):
+    """State of the linear-centered operator: ``linear_state`` of the centred keys k_r - mu_h.
+
+    [ABS] names "linear-centered" attention for the tolerant stages and Table 3
+    (a) of its page compares "Linear, uncentered fit" with "Linear-centered +
+    fit"; neither gives a formula.  Reading: the keys of each head are centred
+    by their mean over all tokens before the feature map, and the queries are
+    left as they are.  Softmax attention is unchanged by subtracting one vector
+    from every key (q . (k - mu) = q . k - q . mu is the same for all keys of a
+    query), so the dense layer the fit targets stays the same, while phi, not
+    being shift-invariant, sees zero-mean keys.
+    """
+    K = _f64(K)
+    return linear_state(K - key_mean(K)[..., None, :], V)
+
+
+def linear_attention_centered(Q, K, V, A=None, b=None) -> np.ndarray:
+    """Linear-centered attention: (phi(q_r) S_c / (phi(q_r) . z_c)) A + b, S_c, z_c of the centred keys."""
+    S, z = linear_state_centered(K, V)
+    return linear_apply(Q, S, z, A, b)
 
 
 def affine_apply(X, A=None, b=None) -> np.ndarray:

@@ -27,6 +27,12 @@ MUTATIONS = {
     "score transposed": ("np.matmul(Qbar, np.swapaxes(Kbar, -1, -2))",
                          "np.swapaxes(np.matmul(Qbar, np.swapaxes(Kbar, -1, -2)), -1, -2)"),
     "ragged tile divided by full size": ("out /= n[None, :, None].astype(np.float64)", "out /= float(tile)"),
+    "keys not centred": ("return linear_state(K - key_mean(K)[..., None, :], V)", "return linear_state(K, V)"),
+    "keys centred with the wrong sign": ("linear_state(K - key_mean(K)", "linear_state(K + key_mean(K)"),
+    "key mean over the features": ("K.sum(axis=-2) / K.shape[-2]", "K.sum(axis=-1) / K.shape[-1]"),
+    "key mean divided by d": ("K.sum(axis=-2) / K.shape[-2]", "K.sum(axis=-2) / K.shape[-1]"),
+    "queries centred instead of keys": ("S, z = linear_state_centered(K, V)\n    return linear_apply(Q, S, z, A, b)",
+                                        "S, z = linear_state(K, V)\n    return linear_apply(Q - key_mean(Q)[..., None, :], S, z, A, b)"),
 }
 
 

@@ -237,6 +237,59 @@ def test_linear_state_single_token():
     np.testing.assert_allclose(oracle.linear_attention(Q, K, V)[0, 0], V[0, 0], rtol=1e-14)
 
 
+# ------------------------------------------------------ linear-centered ----
+
+def test_key_mean_equals_exact_rational_mean():
+    # bf16 inputs: every partial sum is exact in fp64, so the mean is the
+    # correctly rounded exact rational mean
+    from fractions import Fraction
+    H, N, d = 2, 37, 5
+    K = _bf16_grid((H, N, d))
+    mu = oracle.key_mean(K)
+    assert mu.shape == (H, d)
+    for h in range(H):
+        for c in range(d):
+            exact = sum(Fraction(float(v)) for v in K[h, :, c]) / N
+            assert mu[h, c] == float(exact)
+
+
+def test_centered_linear_is_invariant_to_a_key_shift():
+    Q, K, V = _qkv(2, 40, 6, std=1.0)
+    shift = RNG.standard_normal((2, 1, 6))
+    A = RNG.standard_normal((2, 6, 6))
+    b = RNG.standard_normal((2, 6))
+    O = oracle.linear_attention_centered(Q, K, V, A, b)
+    np.testing.assert_allclose(oracle.linear_attention_centered(Q, K + shift, V, A, b), O,
+                               rtol=1e-11, atol=1e-12)
+    # not vacuous: the uncentred operator does move with the keys
+    moved = oracle.linear_attention(Q, K + shift, V) - oracle.linear_attention(Q, K, V)
+    assert np.abs(moved).max() > 1e-3
+
+
+def test_centered_linear_equals_quadratic_form_of_zero_mean_keys():
+    # the associative centred operator against the (separately pinned) quadratic
+    # form, fed keys whose column means are exactly zero by construction
+    Q, _, V = _qkv(2, 25, 8, std=1.0)
+    K = _bf16_grid((2, 25, 8))  # bf16 values: the column sums below are exact
+    Kz = np.concatenate([K, -K], axis=1)
+    Vz = np.concatenate([V, V[:, ::-1]], axis=1)
+    np.testing.assert_array_equal(oracle.key_mean(Kz), 0.0)
+    np.testing.assert_allclose(oracle.linear_attention_centered(Q, Kz, Vz),
+                               oracle.linear_attention_quadratic(Q, Kz, Vz), rtol=1e-12, atol=1e-13)
+    # shifted keys: centring must bring back the same output
+    shift = RNG.standard_normal((2, 1, 8))
+    np.testing.assert_allclose(oracle.linear_attention_centered(Q, Kz + shift, Vz),
+                               oracle.linear_attention_quadratic(Q, Kz, Vz), rtol=1e-11, atol=1e-12)
+
+
+def test_dense_attention_is_invariant_to_a_key_shift():
+    # why centring keeps the fit target: softmax ignores a constant per query
+    Q, K, V = _qkv(2, 30, 6)
+    shift = RNG.standard_normal((2, 1, 6))
+    np.testing.assert_allclose(oracle.dense_attention(Q, K + shift, V, 0.3),
+                               oracle.dense_attention(Q, K, V, 0.3), rtol=1e-12, atol=1e-13)
+
+
 # ----------------------------------------------------------- affine fit ----
 
 def test_affine_fit_recovers_planted_map():
