@@ -227,6 +227,69 @@ def run_reference(args, w):
     return 0
 
 
+def linear_centered_report(zb, w, layer, Q, K, V, stream, hbm, tensor_bytes, t_apply):
+    H, N, d = w.heads, w.n_tokens, w.head_dim
+    dev = Q.device
+    mu = torch.empty(H, d, dtype=torch.float32, device=dev)
+    ws_km = torch.empty(max(zb.key_mean_workspace_bytes(H, N, d), 16), dtype=torch.uint8, device=dev)
+    S_c = torch.empty_like(layer.S)
+    z_c = torch.empty_like(layer.z)
+
+    def centred_state(ev=None):
+        if ev is not None:
+            ev[0].record(stream)
+        zb.zb_key_mean(K, out=mu, ws=ws_km)
+        if ev is not None:
+            ev[1].record(stream)
+        zb.zb_linear_state_centered(K, V, mu, S_c, z_c, layer.ws_lin)
+        if ev is not None:
+            ev[2].record(stream)
+
+    centred_state()
+    torch.cuda.synchronize()
+    reps = 5
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(reps)]
+    for ev in evs:
+        centred_state(ev)
+    torch.cuda.synchronize()
+    zb.zb_last_device_status()
+    t_km = statistics.mean(ev[0].elapsed_time(ev[1]) for ev in evs) / 1e3
+    t_sc = statistics.mean(ev[1].elapsed_time(ev[2]) for ev in evs) / 1e3
+
+    # fit on the calibration rows (the step's dense rows Yc), then residuals of the
+    # fitted outputs, all computed by the library's kernels
+    Xc_c = torch.empty_like(layer.Xc)
+    zb.zb_linear_apply(layer.Qc, S_c, z_c, None, None, out=Xc_c, out_fp32=True)
+    A_c, b_c = zb.zb_affine_fit(Xc_c, layer.Yc, ws=layer.ws_fit)
+    T = w.n_tiles
+    m = len(layer.calib)
+    held = sorted({int((i + 0.5) * T / m) for i in range(m)} - set(layer.calib.tolist()) - {T - 1})
+    held_t = torch.as_tensor(held, dtype=torch.int32, device=dev)
+    Qh = zb.zb_gather_tiles(Q, w.tile, held_t)
+    Yh = zb.zb_dense_attn(Qh, K, V, layer.scale, out_fp32=True)
+
+    def resid(Qr, Y, S, z, A, b):
+        fit = zb.zb_linear_apply(Qr, S, z, A, b, out_fp32=True)
+        num = (fit - Y).double().flatten(1).norm(dim=1)
+        return float((num / Y.double().flatten(1).norm(dim=1)).max())
+
+    res = {"calibration_rows": {"uncentered": resid(layer.Qc, layer.Yc, layer.S, layer.z, layer.A, layer.b),
+                                "centered": resid(layer.Qc, layer.Yc, S_c, z_c, A_c, b_c)},
+           "held_out_rows": {"uncentered": resid(Qh, Yh, layer.S, layer.z, layer.A, layer.b),
+                             "centered": resid(Qh, Yh, S_c, z_c, A_c, b_c)}}
+    torch.cuda.synchronize()
+    zb.zb_last_device_status()
+    return {"zb_key_mean": {"bound": "hbm", "ms": t_km * 1e3, "achieved": tensor_bytes / t_km / 1e9, "peak": hbm,
+                            "unit": "GB/s", "frac": tensor_bytes / t_km / 1e9 / hbm},
+            "zb_linear_state_centered": {"bound": "hbm", "ms": t_sc * 1e3, "achieved": 2 * tensor_bytes / t_sc / 1e9,
+                                         "peak": hbm, "unit": "GB/s", "frac": 2 * tensor_bytes / t_sc / 1e9 / hbm},
+            "stage_ms_without_fit": (t_km + t_sc + t_apply) * 1e3,
+            "fit_residual": res,
+            "held_out_rows": len(held) * w.tile,
+            "note": "max over heads of |fitted linear output - dense output|_F / |dense output|_F; "
+                    "synthetic random inputs, not a trained model's activations"}
+
+
 def config_dict(w):
     return {"workload": f"{w.name}: {w.n_tokens // synth.TOKENS_PER_VIEW} views x {synth.TOKENS_PER_VIEW} "
                         f"tokens = {w.n_tokens} tokens, {w.heads} heads, d={w.head_dim}, bf16; tile "
@@ -249,6 +312,7 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--no-dense-ref", action="store_true", help="skip the dense-attention comparator")
+    ap.add_argument("--no-centered", action="store_true", help="skip the linear-centered measurements")
     ap.add_argument("--profile", action="store_true", help="short run for profilers: no JSON extras")
     args = ap.parse_args()
 
@@ -313,6 +377,9 @@ def main():
     zb.zb_last_device_status()
     if args.profile:
         step()
+        if not args.no_centered:  # one launch of each linear-centered kernel, for profilers
+            mu = zb.zb_key_mean(K)
+            zb.zb_linear_state_centered(K, V, mu, ws=layer.ws_lin)
         torch.cuda.synchronize()
         zb.zb_last_device_status()
         if rank == 0:
@@ -413,6 +480,15 @@ def main():
                      "note": "zb_dense_attn on head 0 at full length, scaled by the head count"}
         del Od
 
+    # -------------------------------------------- linear-centered variant ----
+    # Outside the timed step: the centred linear stage (keys shifted by their
+    # per-head mean) on the same inputs, its two new kernels against HBM, and
+    # the fitted output's residual against dense attention with and without
+    # centring, on the calibration rows and on as many held-out rows.
+    centered = None
+    if not args.no_centered:
+        centered = linear_centered_report(zb, w, layer, Q, K, V, stream, hbm, tensor_bytes, kt["linear_apply"])
+
     # ------------------------------------------------------------ e2e ----
     e2e = None
     if not args.no_e2e:
@@ -461,7 +537,7 @@ def main():
                 "config": config_dict(w), "e2e": e2e, "gpu_launches": layer.launches_per_step * args.steps,
                 "roofline": roofline, "kernel_roofline": kernel_rooflines, "stage_ms": stage_ms,
                 "kernel_ms": {n: v * 1e3 for n, v in kt.items()}, "clocks": clk, "cpu_baseline": cpu,
-                "hybrid_0.7L_mtokens_s": hybrid_07, "dense_reference": dense_ref,
+                "hybrid_0.7L_mtokens_s": hybrid_07, "dense_reference": dense_ref, "linear_centered": centered,
                 "peaks": peaks}
         print(json.dumps(line), flush=True)
     if world > 1:

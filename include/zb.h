@@ -211,6 +211,42 @@ zb_status zb_linear_attn(const uint16_t* Q, const uint16_t* K, const uint16_t* V
                          uint16_t* O, void* ws, size_t ws_bytes, void* stream);
 
 /*
+ * Mean key of each head over all tokens, mu_h = (1/N) sum_r k_r: the shift of
+ * the linear-centered variant (Abstract of "Zebra3D: Efficient Hybrid
+ * Foundation Models For Scalable 3D Reconstruction": linear-centered attention
+ * for the tolerant stages; Table 3 (a): "Linear-centered + fit").  The pages
+ * give no formula; the reading taken centres the keys only, by this mean.
+ *   in : K bf16 [H][N][d];  ws of >= zb_key_mean_workspace_bytes() bytes,
+ *        16-byte aligned, owned by the caller (per-chunk fp64 partial sums)
+ *   out: mu fp32 [H][d]
+ * Sums run in fp32 per thread over a few hundred rows, then fp64 in a fixed
+ * order (the result does not depend on scheduling).  Two kernel launches.
+ * Errors: ZB_ERR_NULL, ZB_ERR_SHAPE, ZB_ERR_ALIGN, ZB_ERR_UNSUPPORTED
+ * (H > 65535), ZB_ERR_WORKSPACE, ZB_ERR_CUDA.
+ */
+size_t zb_key_mean_workspace_bytes(int32_t heads, int64_t n_tokens, int32_t head_dim);
+zb_status zb_key_mean(const uint16_t* K, int32_t heads, int64_t n_tokens, int32_t head_dim,
+                      float* mu, void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * Linear-attention state of the linear-centered variant: zb_linear_state with
+ * every key shifted by its head's key_mean before the feature map,
+ *   S = sum_r phi(k_r - mu_h)^T v_r,  z = sum_r phi(k_r - mu_h),
+ * (k - mu in fp32, phi in fp32, rounded to bf16 for the tensor-core product
+ * as in zb_linear_state).  The output is then zb_linear_apply on the same Q,
+ * unchanged: only the keys are centred.  Softmax attention is unchanged by
+ * such a shift, so the affine fit keeps the same dense target.
+ *   in : K, V bf16 [H][N][d];  key_mean fp32 [H][d] (normally from
+ *        zb_key_mean);  ws of >= zb_linear_state_workspace_bytes() bytes
+ *   out: S fp32 [H][d][d], z fp32 [H][d]
+ * Errors: ZB_ERR_NULL, ZB_ERR_SHAPE, ZB_ERR_ALIGN, ZB_ERR_UNSUPPORTED,
+ * ZB_ERR_WORKSPACE, ZB_ERR_CUDA.
+ */
+zb_status zb_linear_state_centered(const uint16_t* K, const uint16_t* V, const float* key_mean,
+                                   int32_t heads, int64_t n_tokens, int32_t head_dim, float* S,
+                                   float* z, void* ws, size_t ws_bytes, void* stream);
+
+/*
  * Closed-form affine fit (Abstract: closed-form affine fitting makes the
  * conversion training-free; Table 3 (a) of "Zebra3D: Efficient Hybrid
  * Foundation Models ..." compares no fit with fitted variants): per head, the

@@ -28,7 +28,7 @@ __all__ = [
     "ZbError", "Landmarks", "zb_abi_version", "zb_landmark_build", "zb_tile_score_topk",
     "zb_tile_sparse_attn", "zb_dense_attn", "zb_linear_state", "zb_linear_apply", "zb_linear_attn",
     "zb_affine_fit", "zb_gather_tiles", "zb_last_device_status", "HybridLayer",
-    "LAUNCHES_PER_CALL",
+    "LAUNCHES_PER_CALL", "zb_key_mean", "zb_linear_state_centered",
 ]
 
 HEAD_DIM = 64
@@ -37,6 +37,7 @@ HEAD_DIM = 64
 LAUNCHES_PER_CALL = {
     "zb_landmark_build": 1, "zb_tile_score_topk": 2, "zb_tile_sparse_attn": 1, "zb_dense_attn": 1,
     "zb_linear_state": 2, "zb_linear_apply": 1, "zb_linear_attn": 3, "zb_affine_fit": 3, "zb_gather_tiles": 1,
+    "zb_key_mean": 2, "zb_linear_state_centered": 2,
 }
 
 
@@ -229,6 +230,39 @@ def zb_linear_state(K, V, S: Optional[torch.Tensor] = None, z: Optional[torch.Te
     return S, z
 
 
+def key_mean_workspace_bytes(heads: int, n_tokens: int, head_dim: int = HEAD_DIM) -> int:
+    return int(_lib_handle().zb_key_mean_workspace_bytes(heads, n_tokens, head_dim))
+
+
+def zb_key_mean(K, out: Optional[torch.Tensor] = None, ws: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """mu = mean of the keys of each head over all tokens, fp32 [H, d] (the linear-centered shift)."""
+    _need(K, torch.bfloat16, "K", 3)
+    H, N, d = K.shape
+    mu = _out((H, d), torch.float32, K.device, out, "mu")
+    ws = _ws(key_mean_workspace_bytes(H, N, d), K.device, ws)
+    st = _lib_handle().zb_key_mean(_ptr(K), H, N, d, _ptr(mu), _ptr(ws), ws.numel() * ws.element_size(), _stream())
+    _check(st, "zb_key_mean")
+    return mu
+
+
+def zb_linear_state_centered(K, V, mu, S: Optional[torch.Tensor] = None, z: Optional[torch.Tensor] = None,
+                             ws: Optional[torch.Tensor] = None):
+    """S = phi(K - mu)^T V [H, d, d] and z = sum phi(K - mu) [H, d] (fp32), mu fp32 [H, d]."""
+    _need(K, torch.bfloat16, "K", 3)
+    _need(V, torch.bfloat16, "V", 3)
+    _need(mu, torch.float32, "mu", 2)
+    H, N, d = K.shape
+    if tuple(mu.shape) != (H, d):
+        raise ValueError(f"mu must have shape {(H, d)}, got {tuple(mu.shape)}")
+    S = _out((H, d, d), torch.float32, K.device, S, "S")
+    z = _out((H, d), torch.float32, K.device, z, "z")
+    ws = _ws(linear_state_workspace_bytes(H, N, d), K.device, ws)
+    st = _lib_handle().zb_linear_state_centered(_ptr(K), _ptr(V), _ptr(mu), H, N, d, _ptr(S), _ptr(z), _ptr(ws),
+                                                ws.numel() * ws.element_size(), _stream())
+    _check(st, "zb_linear_state_centered")
+    return S, z
+
+
 def zb_linear_apply(Q, S, z, A: Optional[torch.Tensor] = None, b: Optional[torch.Tensor] = None,
                     out: Optional[torch.Tensor] = None, out_fp32: bool = False) -> torch.Tensor:
     """O = (phi(Q) S / (phi(Q) . z)) A + b: bf16 on the tensor cores, or fp32 on the CUDA cores."""
@@ -309,13 +343,16 @@ class HybridLayer:
     ``sparse(Q, K, V)`` runs the tile-sparse stage (landmarks, selection,
     attention), ``calibrate(Q, K, V)`` fits (A, b) of the linear stage against
     dense attention on whole calibration tiles, ``linear(Q, K, V)`` runs the
-    fitted linear stage.  Outputs live in the object's buffers and are
-    overwritten by the next call.
+    fitted linear stage.  With ``centered=True`` the linear stage is the
+    linear-centered variant: keys shifted by their per-head mean before the
+    feature map (zb_key_mean, zb_linear_state_centered).  Outputs live in the
+    object's buffers and are overwritten by the next call.
     """
 
     def __init__(self, heads: int, n_tokens: int, tile: int, k: int, calib_tiles: Sequence[int],
-                 device="cuda", scale: Optional[float] = None):
+                 device="cuda", scale: Optional[float] = None, centered: bool = False):
         d = HEAD_DIM
+        self.centered = centered
         self.heads, self.n_tokens, self.tile, self.k, self.d = heads, n_tokens, tile, k, d
         self.T = n_tiles(n_tokens, tile)
         self.scale = 1.0 / math.sqrt(d) if scale is None else scale
@@ -334,6 +371,9 @@ class HybridLayer:
         self.S = torch.empty(H, d, d, dtype=torch.float32, device=dev)
         self.z = torch.empty(H, d, dtype=torch.float32, device=dev)
         self.ws_lin = torch.empty(max(linear_state_workspace_bytes(H, N, d), 16), dtype=torch.uint8, device=dev)
+        self.mu = torch.empty(H, d, dtype=torch.float32, device=dev)
+        self.ws_km = torch.empty(max(key_mean_workspace_bytes(H, N, d), 16) if centered else 16, dtype=torch.uint8,
+                                 device=dev)
         self.calib = torch.as_tensor(list(calib_tiles), dtype=torch.int32).to(dev)
         R = len(calib_tiles) * tile
         self.R = R
@@ -362,8 +402,15 @@ class HybridLayer:
         return zb_tile_sparse_attn(Q, K, V, self.lm.Kbar_bf16, self.lm.Vbar_bf16, self.idx, self.k,
                                    self.tile, True, self.scale, out=self.O_sparse, ws=self.ws_attn)
 
+    def _state(self, K, V):
+        if self.centered:
+            zb_key_mean(K, out=self.mu, ws=self.ws_km)
+            zb_linear_state_centered(K, V, self.mu, self.S, self.z, self.ws_lin)
+        else:
+            zb_linear_state(K, V, self.S, self.z, self.ws_lin)
+
     def calibrate(self, Q, K, V):
-        zb_linear_state(K, V, self.S, self.z, self.ws_lin)
+        self._state(K, V)
         zb_gather_tiles(Q, self.tile, self.calib, out=self.Qc)
         zb_dense_attn(self.Qc, K, V, self.scale, out=self.Yc, out_fp32=True)
         zb_linear_apply(self.Qc, self.S, self.z, None, None, out=self.Xc, out_fp32=True)
@@ -372,7 +419,7 @@ class HybridLayer:
 
     def linear(self, Q, K, V, refresh_state: bool = False) -> torch.Tensor:
         if refresh_state:
-            zb_linear_state(K, V, self.S, self.z, self.ws_lin)
+            self._state(K, V)
         return zb_linear_apply(Q, self.S, self.z, self.A, self.b, out=self.O_linear)
 
     def step(self, Q, K, V):
@@ -384,4 +431,5 @@ class HybridLayer:
 
     @property
     def launches_per_step(self) -> int:
-        return self.LAUNCHES["sparse"] + self.LAUNCHES["calibrate"] + self.LAUNCHES["linear"]
+        extra = LAUNCHES_PER_CALL["zb_key_mean"] if self.centered else 0
+        return self.LAUNCHES["sparse"] + self.LAUNCHES["calibrate"] + extra + self.LAUNCHES["linear"]

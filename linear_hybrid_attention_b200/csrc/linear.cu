@@ -99,10 +99,13 @@ struct StateSmem {
     int abort_flag;
 };
 
-__global__ void __launch_bounds__(ST_THREADS, 1)
-linear_state_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
-                    int heads, long long n, StateGeom geo, float* __restrict__ partial, int* status,
-                    unsigned long long timeout_ns) {
+// Body of the state kernel.  CENTERED subtracts key_shift[h] (the head's mean
+// key, fp32 [H][d]) from every key before phi: the linear-centered variant.
+template <bool CENTERED>
+__device__ __forceinline__ void linear_state_body(const CUtensorMap& tm_k, const CUtensorMap& tm_v, int heads,
+                                                  long long n, StateGeom geo, float* __restrict__ partial,
+                                                  int* status, unsigned long long timeout_ns,
+                                                  const float* __restrict__ key_shift) {
     extern __shared__ uint8_t smem_raw[];
     StateSmem& sm = *reinterpret_cast<StateSmem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -153,6 +156,13 @@ linear_state_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
     float z0[8], z1[8];
 #pragma unroll
     for (int e = 0; e < 8; ++e) z0[e] = z1[e] = 0.f;
+    // the shifts of this thread's 8 features in both heads
+    float mu[2][8];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+        mu[0][e] = CENTERED ? __ldg(key_shift + h0 * HD + cg * 8 + e) : 0.f;
+        mu[1][e] = CENTERED ? __ldg(key_shift + h1 * HD + cg * 8 + e) : 0.f;
+    }
     bool ok = true;
     int consumed = 0;  // loads whose full barrier was waited on
 
@@ -176,8 +186,13 @@ linear_state_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
                     const bool valid = row0 + r < n;
 #pragma unroll
                     for (int e = 0; e < 4; ++e) {
-                        const float a = valid ? phi(bf16_lo(w[e])) : 0.f;
-                        const float b = valid ? phi(bf16_hi(w[e])) : 0.f;
+                        float xa = bf16_lo(w[e]), xb = bf16_hi(w[e]);
+                        if constexpr (CENTERED) {
+                            xa -= mu[hh][2 * e];
+                            xb -= mu[hh][2 * e + 1];
+                        }
+                        const float a = valid ? phi(xa) : 0.f;
+                        const float b = valid ? phi(xb) : 0.f;
                         w[e] = pack_bf16x2(a, b);
                         // z sums the bf16-rounded features that the MMA uses
                         if (hh == 0) { z0[2 * e] += bf16_lo(w[e]); z0[2 * e + 1] += bf16_hi(w[e]); }
@@ -276,6 +291,20 @@ linear_state_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
     }
 }
 
+__global__ void __launch_bounds__(ST_THREADS, 1)
+linear_state_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
+                    int heads, long long n, StateGeom geo, float* __restrict__ partial, int* status,
+                    unsigned long long timeout_ns) {
+    linear_state_body<false>(tm_k, tm_v, heads, n, geo, partial, status, timeout_ns, nullptr);
+}
+
+__global__ void __launch_bounds__(ST_THREADS, 1)
+linear_state_centered_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
+                             int heads, long long n, StateGeom geo, float* __restrict__ partial, int* status,
+                             unsigned long long timeout_ns, const float* __restrict__ key_shift) {
+    linear_state_body<true>(tm_k, tm_v, heads, n, geo, partial, status, timeout_ns, key_shift);
+}
+
 // Fixed-order sum of the per-CTA partials: S[h], z[h].
 __global__ void linear_state_reduce_kernel(const float* __restrict__ partial, int heads, StateGeom geo,
                                            float* __restrict__ S, float* __restrict__ z) {
@@ -290,6 +319,87 @@ __global__ void linear_state_reduce_kernel(const float* __restrict__ partial, in
         if (e < HD * HD) S[static_cast<size_t>(h) * HD * HD + e] = acc;
         else z[static_cast<size_t>(h) * HD + (e - HD * HD)] = acc;
     }
+}
+
+// =========================================================== key mean ====
+// Per-head mean key mu_h = (1/N) sum_r k_r, the shift of the linear-centered
+// variant.  HBM stream over K: grid (chunks, heads); a CTA owns a contiguous
+// run of rows of one head, thread t reads the 16-byte feature group t % 8 of
+// rows t / 8, t / 8 + 32, ... (consecutive threads read consecutive 16 bytes),
+// four rows in flight per thread, and sums them in fp32.  The 32 row lanes of
+// a feature group are added in fp64 in a fixed order, the chunks likewise in
+// a second kernel, so the result does not depend on scheduling.
+constexpr int KM_THREADS = 256;
+constexpr int KM_ROW_LANES = KM_THREADS / 8;  // rows per pass
+constexpr int KM_UNROLL = 4;
+constexpr int KM_TARGET_CTAS = 148 * 8;       // eight 256-thread CTAs per SM
+
+inline int key_mean_chunks(int heads, long long n) {
+    long long c = (KM_TARGET_CTAS + heads - 1) / heads;
+    const long long max_c = (n + KM_ROW_LANES * KM_UNROLL - 1) / (KM_ROW_LANES * KM_UNROLL);
+    if (c > max_c) c = max_c;
+    if (c < 1) c = 1;
+    return static_cast<int>(c);
+}
+
+ZB_DEVINL void add8_f32(float (&acc)[8], const uint4& v) {
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+        acc[2 * e] += bf16_lo(w[e]);
+        acc[2 * e + 1] += bf16_hi(w[e]);
+    }
+}
+
+__global__ void __launch_bounds__(KM_THREADS)
+key_sum_kernel(const uint16_t* __restrict__ K, long long n, int chunks, double* __restrict__ partial) {
+    __shared__ double red[KM_THREADS / 32][HD];
+    const int h = blockIdx.y, c = blockIdx.x;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int cg = tid & 7, rl = tid >> 3;
+    const long long per = (n + chunks - 1) / chunks;
+    const long long r0 = static_cast<long long>(c) * per;
+    const long long r1 = min(n, r0 + per);
+    const uint4* rows = reinterpret_cast<const uint4*>(K + static_cast<long long>(h) * n * HD);
+    float acc[8];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) acc[e] = 0.f;
+    long long r = r0 + rl;
+    for (; r + KM_ROW_LANES * (KM_UNROLL - 1) < r1; r += KM_ROW_LANES * KM_UNROLL) {
+        uint4 v[KM_UNROLL];
+#pragma unroll
+        for (int u = 0; u < KM_UNROLL; ++u) v[u] = __ldcs(rows + (r + KM_ROW_LANES * u) * 8 + cg);
+#pragma unroll
+        for (int u = 0; u < KM_UNROLL; ++u) add8_f32(acc, v[u]);
+    }
+    for (; r < r1; r += KM_ROW_LANES) add8_f32(acc, __ldcs(rows + r * 8 + cg));
+    // lanes l, l ^ 8, l ^ 16, l ^ 24 of a warp hold the same feature group
+    double dacc[8];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+        dacc[e] = static_cast<double>(acc[e]);
+        dacc[e] += __shfl_xor_sync(0xffffffffu, dacc[e], 8);
+        dacc[e] += __shfl_xor_sync(0xffffffffu, dacc[e], 16);
+    }
+    if (lane < 8) {
+#pragma unroll
+        for (int e = 0; e < 8; ++e) red[warp][cg * 8 + e] = dacc[e];
+    }
+    __syncthreads();
+    if (tid < HD) {
+        double sum = 0.0;
+#pragma unroll
+        for (int w = 0; w < KM_THREADS / 32; ++w) sum += red[w][tid];
+        partial[(static_cast<long long>(h) * chunks + c) * HD + tid] = sum;
+    }
+}
+
+__global__ void key_mean_reduce_kernel(const double* __restrict__ partial, int chunks, long long n,
+                                       float* __restrict__ mu) {
+    const int h = blockIdx.x, f = threadIdx.x;
+    double sum = 0.0;
+    for (int c = 0; c < chunks; ++c) sum += partial[(static_cast<long long>(h) * chunks + c) * HD + f];
+    mu[h * HD + f] = static_cast<float>(sum / static_cast<double>(n));
 }
 
 // ============================================================== apply ====
@@ -719,6 +829,65 @@ extern "C" zb_status zb_linear_state(const uint16_t* K, const uint16_t* V, int32
     float* part = static_cast<float*>(ws);
     lin::linear_state_kernel<<<geo.pairs * geo.chunks, lin::ST_THREADS, smem, st>>>(
         mk, mv, heads, n_tokens, geo, part, dev.status, wait_timeout_ns());
+    if (cudaGetLastError() != cudaSuccess) return ZB_ERR_CUDA;
+    lin::linear_state_reduce_kernel<<<heads, 256, 0, st>>>(part, heads, geo, S, z);
+    return cudaGetLastError() == cudaSuccess ? ZB_OK : ZB_ERR_CUDA;
+}
+
+extern "C" size_t zb_key_mean_workspace_bytes(int32_t heads, int64_t n_tokens, int32_t head_dim) {
+    if (heads < 1 || n_tokens < 1 || head_dim != 64) return 0;
+    return static_cast<size_t>(heads) * lin::key_mean_chunks(heads, n_tokens) * lin::HD * sizeof(double);
+}
+
+extern "C" zb_status zb_key_mean(const uint16_t* K, int32_t heads, int64_t n_tokens, int32_t head_dim,
+                                 float* mu, void* ws, size_t ws_bytes, void* stream) {
+    if (heads < 1 || n_tokens < 1) return ZB_ERR_SHAPE;
+    if (head_dim != 64) return ZB_ERR_UNSUPPORTED;
+    if (heads > 65535 || n_tokens > (1ll << 31) - 256) return ZB_ERR_UNSUPPORTED;
+    if (!K || !mu) return ZB_ERR_NULL;
+    if (!aligned16(K) || !aligned16(mu) || !aligned16(ws)) return ZB_ERR_ALIGN;
+    const size_t need = zb_key_mean_workspace_bytes(heads, n_tokens, head_dim);
+    if (!ws || ws_bytes < need) return ZB_ERR_WORKSPACE;
+    DeviceInfo dev;
+    zb_status e = current_device(&dev);
+    if (e != ZB_OK) return e;
+    const int chunks = lin::key_mean_chunks(heads, n_tokens);
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    double* part = static_cast<double*>(ws);
+    lin::key_sum_kernel<<<dim3(static_cast<unsigned>(chunks), static_cast<unsigned>(heads)), lin::KM_THREADS, 0, st>>>(
+        K, n_tokens, chunks, part);
+    if (cudaGetLastError() != cudaSuccess) return ZB_ERR_CUDA;
+    lin::key_mean_reduce_kernel<<<heads, lin::HD, 0, st>>>(part, chunks, n_tokens, mu);
+    return cudaGetLastError() == cudaSuccess ? ZB_OK : ZB_ERR_CUDA;
+}
+
+extern "C" zb_status zb_linear_state_centered(const uint16_t* K, const uint16_t* V, const float* key_mean,
+                                              int32_t heads, int64_t n_tokens, int32_t head_dim, float* S,
+                                              float* z, void* ws, size_t ws_bytes, void* stream) {
+    if (heads < 1 || n_tokens < 1) return ZB_ERR_SHAPE;
+    if (head_dim != 64) return ZB_ERR_UNSUPPORTED;
+    if (n_tokens > (1ll << 31) - 256) return ZB_ERR_UNSUPPORTED;
+    if (!K || !V || !key_mean || !S || !z) return ZB_ERR_NULL;
+    if (!aligned16(K) || !aligned16(V) || !aligned16(key_mean) || !aligned16(S) || !aligned16(z) ||
+        !aligned16(ws))
+        return ZB_ERR_ALIGN;
+    const size_t need = lin::state_ws_bytes(heads, n_tokens);
+    if (!ws || ws_bytes < need) return ZB_ERR_WORKSPACE;
+    DeviceInfo dev;
+    zb_status e = current_device(&dev);
+    if (e != ZB_OK) return e;
+    CUtensorMap mk, mv;
+    if ((e = make_map_bf16_3d(&mk, K, 64, n_tokens, heads, lin::TILE)) != ZB_OK) return e;
+    if ((e = make_map_bf16_3d(&mv, V, 64, n_tokens, heads, lin::TILE)) != ZB_OK) return e;
+    const lin::StateGeom geo = lin::state_geom(heads, n_tokens);
+    const size_t smem = sizeof(lin::StateSmem) + 1024;
+    if (cudaFuncSetAttribute(lin::linear_state_centered_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(smem)) != cudaSuccess)
+        return ZB_ERR_CUDA;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    float* part = static_cast<float*>(ws);
+    lin::linear_state_centered_kernel<<<geo.pairs * geo.chunks, lin::ST_THREADS, smem, st>>>(
+        mk, mv, heads, n_tokens, geo, part, dev.status, wait_timeout_ns(), key_mean);
     if (cudaGetLastError() != cudaSuccess) return ZB_ERR_CUDA;
     lin::linear_state_reduce_kernel<<<heads, 256, 0, st>>>(part, heads, geo, S, z);
     return cudaGetLastError() == cudaSuccess ? ZB_OK : ZB_ERR_CUDA;

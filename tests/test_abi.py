@@ -28,7 +28,8 @@ def test_header_declares_the_calls():
     names = _declared()
     for n in ["zb_landmark_build", "zb_tile_score_topk", "zb_tile_sparse_attn", "zb_dense_attn",
               "zb_linear_state", "zb_linear_apply", "zb_linear_attn", "zb_affine_fit", "zb_gather_tiles",
-              "zb_last_device_status", "zb_status_string", "zb_abi_version"]:
+              "zb_last_device_status", "zb_status_string", "zb_abi_version", "zb_key_mean",
+              "zb_linear_state_centered"]:
         assert n in names
 
 
@@ -118,6 +119,23 @@ def test_validation_errors_before_launch(lib):
     assert lib.zb_affine_fit(FAKE, FAKE, 2, 64, 64, FAKE, FAKE, FAKE, 1 << 30, None) == 2
     wsn = lib.zb_affine_fit_workspace_bytes(2, 300, 64)
     assert lib.zb_affine_fit(FAKE, FAKE, 2, 300, 64, FAKE, FAKE, FAKE, wsn - 8, None) == 5
+    # linear-centered: key mean and centred state
+    kmw = lib.zb_key_mean_workspace_bytes(2, 256, 64)
+    assert kmw > 0 and kmw % (64 * 8) == 0
+    assert lib.zb_key_mean_workspace_bytes(2, 256, 32) == 0
+    assert lib.zb_key_mean(FAKE, 2, 0, 64, FAKE, FAKE, kmw, None) == 2
+    assert lib.zb_key_mean(FAKE, 2, 256, 32, FAKE, FAKE, kmw, None) == 4
+    assert lib.zb_key_mean(FAKE, 70000, 256, 64, FAKE, FAKE, 1 << 40, None) == 4
+    assert lib.zb_key_mean(None, 2, 256, 64, FAKE, FAKE, kmw, None) == 1
+    assert lib.zb_key_mean(FAKE, 2, 256, 64, None, FAKE, kmw, None) == 1
+    assert lib.zb_key_mean(FAKE, 2, 256, 64, FAKE + 4, FAKE, kmw, None) == 3
+    assert lib.zb_key_mean(FAKE, 2, 256, 64, FAKE, FAKE, kmw - 8, None) == 5
+    assert lib.zb_key_mean(FAKE, 2, 256, 64, FAKE, None, kmw, None) == 5
+    assert lib.zb_linear_state_centered(FAKE, FAKE, None, 2, 256, 64, FAKE, FAKE, FAKE, need, None) == 1
+    assert lib.zb_linear_state_centered(FAKE, FAKE, FAKE + 4, 2, 256, 64, FAKE, FAKE, FAKE, need, None) == 3
+    assert lib.zb_linear_state_centered(FAKE, FAKE, FAKE, 2, 256, 64, FAKE, FAKE, FAKE, need - 1, None) == 5
+    assert lib.zb_linear_state_centered(FAKE, FAKE, FAKE, 2, 256, 16, FAKE, FAKE, FAKE, need, None) == 4
+    assert lib.zb_linear_state_centered(FAKE, FAKE, FAKE, 0, 256, 64, FAKE, FAKE, FAKE, need, None) == 2
     # gather
     assert lib.zb_gather_tiles(FAKE, S, FAKE, 0, FAKE, None) == 2
     assert lib.zb_gather_tiles(FAKE, S, None, 2, FAKE, None) == 1
