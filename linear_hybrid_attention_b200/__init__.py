@@ -33,12 +33,26 @@ __all__ = [
 
 HEAD_DIM = 64
 
-# kernels each entry point launches (for counting launches in a timed region)
+# kernels each entry point launches (for counting launches in a timed region);
+# zb_tile_score_topk launches 2 per pass over the heads its workspace holds
+# (topk_launches gives the count of one call)
 LAUNCHES_PER_CALL = {
     "zb_landmark_build": 1, "zb_tile_score_topk": 2, "zb_tile_sparse_attn": 1, "zb_dense_attn": 1,
     "zb_linear_state": 2, "zb_linear_apply": 1, "zb_linear_attn": 3, "zb_affine_fit": 3, "zb_gather_tiles": 1,
     "zb_key_mean": 2, "zb_linear_state_centered": 2,
 }
+
+
+def topk_launches(heads: int, n_tiles_: int, k: int, ws_bytes: int) -> int:
+    """Kernels one zb_tile_score_topk call launches: none for k = 0, one fill kernel for
+    k = T, else a score GEMM and a select kernel per pass over as many heads as the
+    workspace holds (T * T doubles per head)."""
+    if k == 0:
+        return 0
+    if k == n_tiles_:
+        return 1
+    per_pass = min(heads, ws_bytes // (n_tiles_ * n_tiles_ * 8))
+    return 2 * (-(-heads // per_pass))
 
 
 class ZbError(RuntimeError):
@@ -385,10 +399,10 @@ class HybridLayer:
         self.ws_fit = torch.empty(max(affine_fit_workspace_bytes(H, max(R, d + 1), d), 16), dtype=torch.uint8,
                                   device=dev)
 
-    # kernel launches of each method
+    # kernel launches of each method (the selection's count depends on the
+    # shape and workspace: see launches_per_step)
     LAUNCHES = {
-        "sparse": LAUNCHES_PER_CALL["zb_landmark_build"] + LAUNCHES_PER_CALL["zb_tile_score_topk"]
-        + LAUNCHES_PER_CALL["zb_tile_sparse_attn"],
+        "sparse": LAUNCHES_PER_CALL["zb_landmark_build"] + LAUNCHES_PER_CALL["zb_tile_sparse_attn"],
         "calibrate": LAUNCHES_PER_CALL["zb_linear_state"] + LAUNCHES_PER_CALL["zb_gather_tiles"]
         + LAUNCHES_PER_CALL["zb_dense_attn"] + LAUNCHES_PER_CALL["zb_linear_apply"]
         + LAUNCHES_PER_CALL["zb_affine_fit"],
@@ -432,4 +446,5 @@ class HybridLayer:
     @property
     def launches_per_step(self) -> int:
         extra = LAUNCHES_PER_CALL["zb_key_mean"] if self.centered else 0
-        return self.LAUNCHES["sparse"] + self.LAUNCHES["calibrate"] + extra + self.LAUNCHES["linear"]
+        topk = topk_launches(self.heads, self.T, self.k, self.ws_topk.numel())
+        return self.LAUNCHES["sparse"] + topk + self.LAUNCHES["calibrate"] + extra + self.LAUNCHES["linear"]

@@ -149,3 +149,16 @@ def test_binding_refuses_cpu_tensors():
         zb.zb_landmark_build(x, x, x, 64)
     with pytest.raises(ValueError, match="CUDA"):
         zb.zb_linear_state(x, x)
+
+
+def test_topk_launch_count_follows_the_launcher():
+    # zb_tile_score_topk: nothing for k = 0, one fill kernel for k = T, else a score
+    # GEMM and a select per pass over the heads that the workspace holds
+    from linear_hybrid_attention_b200 import topk_launches
+    T = 10992
+    assert topk_launches(16, T, 660, 4 * T * T * 8) == 8
+    assert topk_launches(16, T, 660, 16 * T * T * 8) == 2
+    assert topk_launches(16, T, 660, 5 * T * T * 8 - 1) == 8   # 4 heads per pass
+    assert topk_launches(3, T, 660, 2 * T * T * 8) == 4        # passes of 2 and 1 heads
+    assert topk_launches(16, T, 0, 0) == 0
+    assert topk_launches(16, T, T, 0) == 1
