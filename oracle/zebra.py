@@ -49,7 +49,7 @@ __all__ = [
     "sparse_attention", "dense_attention", "elu_plus_one", "linear_state",
     "linear_apply", "linear_attention", "linear_attention_quadratic", "affine_fit",
     "affine_apply", "calibration_rows", "RIDGE_REL", "key_mean", "linear_state_centered",
-    "linear_attention_centered",
+    "linear_attention_centered", "block_mass", "top_mass_fraction", "selected_mass_fraction",
 ]
 
 
@@ -319,6 +319,53 @@ def affine_fit(X, Y, ridge_rel: float = RIDGE_REL):
         A[h] = W
         b[h] = ym - xm @ W
     return A, b
+
+
+def block_mass(Q, K, scale: float, block: int) -> np.ndarray:
+    """Softmax mass of every (query block, key block) pair of dense attention -> [H, T, T] (fp64).
+
+    M[h, a, b] = sum over query rows r of block a and keys c of block b of
+    p_rc, p = softmax over all keys of scale * q_r . k_c.  Blocks are runs of
+    ``block`` tokens in sequence order, the last one ragged (the tiling of
+    ``tile_lengths``).  The pages measure this with 64 x 64 token blocks on a
+    dense pass to judge how concentrated attention is ([ABS]'s page, Figure 2
+    (b) and Figure 8: mass kept by the heaviest 20% of 64 x 64 blocks).
+    """
+    Q, K = _f64(Q), _f64(K)
+    H, N, _ = Q.shape
+    nb = tile_lengths(N, block)
+    starts = np.arange(len(nb)) * block
+    out = np.zeros((H, len(nb), len(nb)), dtype=np.float64)
+    for h in range(H):
+        for a in range(len(nb)):
+            r0 = a * block
+            P = _softmax_rows(scale * Q[h, r0:r0 + nb[a]] @ K[h].T)
+            out[h, a] = np.add.reduceat(P.sum(axis=0), starts)
+    return out
+
+
+def top_mass_fraction(M, m: int) -> np.ndarray:
+    """Share of each query block's mass held by its m heaviest key blocks -> [H, T].
+
+    Reading of the pages' "highest-mass 20% of 64 x 64 token blocks" (Figure 2
+    (b), Figure 8): the selection is made per query block, like the method's
+    per-query-tile selection, with m = ceil(0.2 T) supplied by the caller.
+    """
+    M = _f64(M)
+    heavy_first = -np.sort(-M, axis=-1)
+    return heavy_first[..., :m].sum(axis=-1) / M.sum(axis=-1)
+
+
+def selected_mass_fraction(M, idx) -> np.ndarray:
+    """Share of each query tile's mass held by the key tiles in its index list -> [H, T].
+
+    M: block masses at the tile size ([H, T, T]); idx: [H, T, k] selected key
+    tiles (from ``select_tiles``), so this is the dense-softmax mass that the
+    method's mean-pooled selection keeps exactly.
+    """
+    M = _f64(M)
+    kept = np.take_along_axis(M, np.asarray(idx, dtype=np.int64), axis=-1)
+    return kept.sum(axis=-1) / M.sum(axis=-1)
 
 
 def calibration_rows(n_tokens: int, tile: int, tiles: Sequence[int]) -> np.ndarray:

@@ -33,6 +33,11 @@ MUTATIONS = {
     "key mean divided by d": ("K.sum(axis=-2) / K.shape[-2]", "K.sum(axis=-2) / K.shape[-1]"),
     "queries centred instead of keys": ("S, z = linear_state_centered(K, V)\n    return linear_apply(Q, S, z, A, b)",
                                         "S, z = linear_state(K, V)\n    return linear_apply(Q - key_mean(Q)[..., None, :], S, z, A, b)"),
+    "block mass without the scale": ("P = _softmax_rows(scale * Q[h, r0:r0 + nb[a]] @ K[h].T)",
+                                     "P = _softmax_rows(Q[h, r0:r0 + nb[a]] @ K[h].T)"),
+    "block mass averaged over rows": ("np.add.reduceat(P.sum(axis=0), starts)", "np.add.reduceat(P.mean(axis=0), starts)"),
+    "lightest blocks kept": ("heavy_first = -np.sort(-M, axis=-1)", "heavy_first = np.sort(M, axis=-1)"),
+    "selected mass not normalised": ("return kept.sum(axis=-1) / M.sum(axis=-1)", "return kept.sum(axis=-1)"),
 }
 
 

@@ -290,6 +290,64 @@ def test_dense_attention_is_invariant_to_a_key_shift():
                                oracle.dense_attention(Q, K, V, 0.3), rtol=1e-12, atol=1e-13)
 
 
+# ---------------------------------------------- block-mass diagnostic ----
+
+def test_block_mass_rows_hold_one_unit_per_query():
+    # every query row's probabilities sum to 1, so a block row holds its length
+    Q, K, _ = _qkv(2, 300, 8, std=1.0)
+    M = oracle.block_mass(Q, K, 0.4, 64)
+    assert M.shape == (2, 5, 5)
+    np.testing.assert_allclose(M.sum(axis=-1), np.broadcast_to(oracle.tile_lengths(300, 64), (2, 5)), rtol=1e-13)
+    assert (M >= 0).all()
+
+
+def test_block_mass_of_uniform_attention():
+    # all-zero keys: p = 1/N everywhere, M[a, b] = n_a n_b / N
+    Q, _, _ = _qkv(1, 150, 4)
+    n = oracle.tile_lengths(150, 64)
+    M = oracle.block_mass(Q, np.zeros_like(Q), 0.5, 64)
+    np.testing.assert_allclose(M[0], np.outer(n, n) / 150.0, rtol=1e-13)
+
+
+def test_block_mass_is_attention_with_block_indicator_values():
+    # dense attention (pinned against the library's SDPA) with V = the one-hot
+    # key-block indicator gives each row's mass per key block; summing the rows
+    # of a query block gives M
+    H, N, d, B = 2, 130, 8, 64
+    Q, K, _ = _qkv(H, N, d, std=1.0)
+    T = -(-N // B)
+    E = np.zeros((N, T))
+    E[np.arange(N), np.arange(N) // B] = 1.0
+    R = oracle.dense_attention(Q, K, np.broadcast_to(E, (H, N, T)).copy(), 0.7)
+    want = np.stack([np.stack([R[h, a * B:(a + 1) * B].sum(axis=0) for a in range(T)]) for h in range(H)])
+    np.testing.assert_allclose(oracle.block_mass(Q, K, 0.7, B), want, rtol=1e-12, atol=1e-14)
+    # block size 1: the probability matrix itself
+    np.testing.assert_allclose(oracle.block_mass(Q[:, :9], K[:, :9], 0.7, 1),
+                               oracle.dense_attention(Q[:, :9], K[:, :9], np.broadcast_to(np.eye(9), (H, 9, 9)).copy(), 0.7),
+                               rtol=1e-12, atol=1e-14)
+
+
+def test_top_mass_fraction_is_the_best_subset():
+    M = RNG.random((2, 3, 7))
+    for m in range(0, 8):
+        got = oracle.top_mass_fraction(M, m)
+        for h in range(2):
+            for a in range(3):
+                best = max((sum(M[h, a, list(c)]) for c in itertools.combinations(range(7), m)), default=0.0)
+                assert abs(got[h, a] - best / M[h, a].sum()) <= 1e-14
+
+
+def test_selected_mass_fraction_of_the_top_tiles_and_of_all():
+    M = RNG.random((2, 4, 6))
+    idx = np.sort(np.argsort(-M, axis=-1)[..., :2], axis=-1)
+    np.testing.assert_allclose(oracle.selected_mass_fraction(M, idx), oracle.top_mass_fraction(M, 2), rtol=1e-14)
+    every = np.broadcast_to(np.arange(6), (2, 4, 6))
+    np.testing.assert_allclose(oracle.selected_mass_fraction(M, every), 1.0, rtol=1e-14)
+    # one hand-worked row
+    M1 = np.array([[[1.0, 2.0, 3.0, 4.0]]])
+    assert oracle.selected_mass_fraction(M1, np.array([[[0, 2]]]))[0, 0] == 0.4
+
+
 # ----------------------------------------------------------- affine fit ----
 
 def test_affine_fit_recovers_planted_map():
