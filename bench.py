@@ -290,6 +290,45 @@ def linear_centered_report(zb, w, layer, Q, K, V, stream, hbm, tensor_bytes, t_a
                     "synthetic random inputs, not a trained model's activations"}
 
 
+def block_mass_report(zb, w, layer, Q, K, V, stream):
+    """Dense-softmax mass kept by selections, on head 0 (the heads are alike):
+    the heaviest 20% of 64 x 64 blocks, the heaviest 20% and the heaviest k of
+    the tiles, and the method's own k selected tiles (mean-pooled scores)."""
+    q1, k1, v1 = Q[:1], K[:1], V[:1]
+    _, lse = zb.zb_dense_attn(q1, k1, v1, layer.scale, want_lse=True)
+    M64 = zb.zb_block_mass(q1, k1, lse, 64, layer.scale)
+    torch.cuda.synchronize()
+    a = torch.cuda.Event(enable_timing=True)
+    bb = torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    zb.zb_block_mass(q1, k1, lse, 64, layer.scale, out=M64)
+    bb.record(stream)
+    torch.cuda.synchronize()
+    t = a.elapsed_time(bb) / 1e3
+    T64 = M64.shape[-1]
+    top64 = zb.zb_block_mass_top_fraction(M64, math.ceil(0.2 * T64))
+    Mt = zb.zb_block_mass(q1, k1, lse, w.tile, layer.scale)
+    T = Mt.shape[-1]
+    top_t20 = zb.zb_block_mass_top_fraction(Mt, math.ceil(0.2 * T))
+    top_tk = zb.zb_block_mass_top_fraction(Mt, w.k)
+    sel = zb.zb_block_mass_selected_fraction(Mt, layer.idx[:1].contiguous())
+    torch.cuda.synchronize()
+    zb.zb_last_device_status()
+    n = w.n_tokens
+    exps = float(n) * n
+    mufu_bound = 16.0 * torch.cuda.get_device_properties(Q.device).multi_processor_count * 1.965e9
+    out = {"head": 0, "block_mass_64_ms": t * 1e3, "qk_tflops": 2.0 * n * n * w.head_dim / t / 1e12,
+           "exp_per_s": exps / t, "frac_of_mufu_bound": exps / t / mufu_bound,
+           "mufu_bound_note": "16 exponentials per clock per SM at the 1,965 MHz maximum clock",
+           "retained_mass": {"top20pct_64x64_blocks": float(top64.mean()),
+                             f"top20pct_{w.tile}_tiles": float(top_t20.mean()),
+                             f"top{w.k}_{w.tile}_tiles": float(top_tk.mean()),
+                             f"method_selected_{w.k}_tiles": float(sel.mean())},
+           "note": "mean over query blocks of head 0; synthetic inputs with planted tiles"}
+    del M64, Mt
+    return out
+
+
 def config_dict(w):
     return {"workload": f"{w.name}: {w.n_tokens // synth.TOKENS_PER_VIEW} views x {synth.TOKENS_PER_VIEW} "
                         f"tokens = {w.n_tokens} tokens, {w.heads} heads, d={w.head_dim}, bf16; tile "
@@ -313,6 +352,7 @@ def main():
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--no-dense-ref", action="store_true", help="skip the dense-attention comparator")
     ap.add_argument("--no-centered", action="store_true", help="skip the linear-centered measurements")
+    ap.add_argument("--no-block-mass", action="store_true", help="skip the block-mass diagnostic")
     ap.add_argument("--profile", action="store_true", help="short run for profilers: no JSON extras")
     args = ap.parse_args()
 
@@ -489,6 +529,11 @@ def main():
     if not args.no_centered:
         centered = linear_centered_report(zb, w, layer, Q, K, V, stream, hbm, tensor_bytes, kt["linear_apply"])
 
+    # --------------------------------------------- block-mass diagnostic ----
+    block_mass = None
+    if not args.no_block_mass:
+        block_mass = block_mass_report(zb, w, layer, Q, K, V, stream)
+
     # ------------------------------------------------------------ e2e ----
     e2e = None
     if not args.no_e2e:
@@ -538,6 +583,7 @@ def main():
                 "roofline": roofline, "kernel_roofline": kernel_rooflines, "stage_ms": stage_ms,
                 "kernel_ms": {n: v * 1e3 for n, v in kt.items()}, "clocks": clk, "cpu_baseline": cpu,
                 "hybrid_0.7L_mtokens_s": hybrid_07, "dense_reference": dense_ref, "linear_centered": centered,
+                "block_mass": block_mass,
                 "peaks": peaks}
         print(json.dumps(line), flush=True)
     if world > 1:

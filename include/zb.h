@@ -247,6 +247,41 @@ zb_status zb_linear_state_centered(const uint16_t* K, const uint16_t* V, const f
                                    float* z, void* ws, size_t ws_bytes, void* stream);
 
 /*
+ * Block-mass diagnostic (Figure 2 (b) and Figure 8 of "Zebra3D: Efficient
+ * Hybrid Foundation Models For Scalable 3D Reconstruction": the attention mass
+ * kept by the heaviest 20% of 64 x 64 token blocks, from a dense pass).
+ *
+ * zb_block_mass: M[h][a][b] = sum over query rows r of block a and keys c of
+ * block b of p_rc = exp(scale q_r . k_c - lse[h][r]), the dense softmax
+ * probabilities.  Blocks are runs of s.tile (64 or 128) tokens, the last one
+ * ragged.  lse is each row's log-sum-exp in natural log, as zb_dense_attn
+ * returns it for the same Q, K and scale.
+ *   in : Q, K bf16 [H][N][d];  lse fp32 [H][N]
+ *   out: M fp32 [H][Tb][Tb], Tb = ceil(N / s.tile)   (every entry written)
+ * S = Q K^T is recomputed on the tensor cores; every entry of M is stored
+ * once, summed in a fixed order.
+ * Errors: ZB_ERR_NULL, ZB_ERR_SHAPE (scale <= 0), ZB_ERR_ALIGN,
+ * ZB_ERR_UNSUPPORTED (H > 65535, Tb > 49152), ZB_ERR_CUDA.
+ *
+ * zb_block_mass_top_fraction: per row of M [heads * n_blocks][n_blocks], the
+ * sum of its m largest entries over the row sum (fp64 sums), 0 <= m <= n_blocks;
+ * frac fp32 [heads * n_blocks].  Errors: ZB_ERR_NULL, ZB_ERR_SHAPE,
+ * ZB_ERR_ALIGN, ZB_ERR_UNSUPPORTED (n_blocks > 49152), ZB_ERR_CUDA.
+ *
+ * zb_block_mass_selected_fraction: per row of M (masses at the tile size), the
+ * mass in the k key tiles that idx [heads][n_blocks][k] lists for that row
+ * (zb_tile_score_topk's selection) over the row sum.  Indices out of range
+ * count nothing and set ZB_ERR_INDEX in the device status.  Errors:
+ * ZB_ERR_NULL, ZB_ERR_SHAPE, ZB_ERR_ALIGN, ZB_ERR_CUDA.
+ */
+zb_status zb_block_mass(const uint16_t* Q, const uint16_t* K, const float* lse, zb_shape s, float scale,
+                        float* M, void* stream);
+zb_status zb_block_mass_top_fraction(const float* M, int32_t heads, int32_t n_blocks, int32_t m, float* frac,
+                                     void* stream);
+zb_status zb_block_mass_selected_fraction(const float* M, int32_t heads, int32_t n_blocks, const int32_t* idx,
+                                          int32_t k, float* frac, void* stream);
+
+/*
  * Closed-form affine fit (Abstract: closed-form affine fitting makes the
  * conversion training-free; Table 3 (a) of "Zebra3D: Efficient Hybrid
  * Foundation Models ..." compares no fit with fitted variants): per head, the

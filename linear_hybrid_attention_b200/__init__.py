@@ -28,7 +28,8 @@ __all__ = [
     "ZbError", "Landmarks", "zb_abi_version", "zb_landmark_build", "zb_tile_score_topk",
     "zb_tile_sparse_attn", "zb_dense_attn", "zb_linear_state", "zb_linear_apply", "zb_linear_attn",
     "zb_affine_fit", "zb_gather_tiles", "zb_last_device_status", "HybridLayer",
-    "LAUNCHES_PER_CALL", "zb_key_mean", "zb_linear_state_centered",
+    "LAUNCHES_PER_CALL", "zb_key_mean", "zb_linear_state_centered", "zb_block_mass",
+    "zb_block_mass_top_fraction", "zb_block_mass_selected_fraction",
 ]
 
 HEAD_DIM = 64
@@ -39,7 +40,8 @@ HEAD_DIM = 64
 LAUNCHES_PER_CALL = {
     "zb_landmark_build": 1, "zb_tile_score_topk": 2, "zb_tile_sparse_attn": 1, "zb_dense_attn": 1,
     "zb_linear_state": 2, "zb_linear_apply": 1, "zb_linear_attn": 3, "zb_affine_fit": 3, "zb_gather_tiles": 1,
-    "zb_key_mean": 2, "zb_linear_state_centered": 2,
+    "zb_key_mean": 2, "zb_linear_state_centered": 2, "zb_block_mass": 1, "zb_block_mass_top_fraction": 1,
+    "zb_block_mass_selected_fraction": 1,
 }
 
 
@@ -212,6 +214,50 @@ def zb_dense_attn(Q, K, V, scale: Optional[float] = None, out: Optional[torch.Te
                                      1 if out_fp32 else 0, _ptr(lse), _stream())
     _check(st, "zb_dense_attn")
     return (O, lse) if lse is not None else O
+
+
+def zb_block_mass(Q, K, lse, block: int = 64, scale: Optional[float] = None,
+                  out: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """Dense-softmax mass of every (query block, key block) pair, fp32 [H, Tb, Tb].
+
+    lse: fp32 [H, N], the rows' log-sum-exp from zb_dense_attn(Q, K, V, scale, want_lse=True)."""
+    _need(Q, torch.bfloat16, "Q", 3)
+    _need(K, torch.bfloat16, "K", 3)
+    _need(lse, torch.float32, "lse", 2)
+    H, N, d = Q.shape
+    if tuple(K.shape) != (H, N, d) or tuple(lse.shape) != (H, N):
+        raise ValueError("Q, K must be [H, N, d] and lse [H, N]")
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    Tb = n_tiles(N, block)
+    M = _out((H, Tb, Tb), torch.float32, Q.device, out, "M")
+    st = _lib_handle().zb_block_mass(_ptr(Q), _ptr(K), _ptr(lse), _lib.ZbShape(H, N, d, block), float(scale),
+                                     _ptr(M), _stream())
+    _check(st, "zb_block_mass")
+    return M
+
+
+def zb_block_mass_top_fraction(M, m: int, out: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """Per query block: the share of its mass held by its m heaviest key blocks, fp32 [H, Tb]."""
+    _need(M, torch.float32, "M", 3)
+    H, Tb, _ = M.shape
+    frac = _out((H, Tb), torch.float32, M.device, out, "frac")
+    st = _lib_handle().zb_block_mass_top_fraction(_ptr(M), H, Tb, int(m), _ptr(frac), _stream())
+    _check(st, "zb_block_mass_top_fraction")
+    return frac
+
+
+def zb_block_mass_selected_fraction(M, idx, out: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """Per query tile: the share of its mass held by the key tiles of its index list, fp32 [H, T]."""
+    _need(M, torch.float32, "M", 3)
+    _need(idx, torch.int32, "idx", 3)
+    H, T, _ = M.shape
+    if tuple(idx.shape[:2]) != (H, T):
+        raise ValueError(f"idx must be [{H}, {T}, k], got {tuple(idx.shape)}")
+    frac = _out((H, T), torch.float32, M.device, out, "frac")
+    st = _lib_handle().zb_block_mass_selected_fraction(_ptr(M), H, T, _ptr(idx), idx.shape[2], _ptr(frac), _stream())
+    _check(st, "zb_block_mass_selected_fraction")
+    return frac
 
 
 def linear_state_workspace_bytes(heads: int, n_tokens: int, head_dim: int = HEAD_DIM) -> int:

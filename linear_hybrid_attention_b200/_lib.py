@@ -41,6 +41,9 @@ PROTOTYPES = {
     "zb_key_mean_workspace_bytes": (c_sz, [c_i32, c_i64, c_i32]),
     "zb_key_mean": (c_i32, [c_vp, c_i32, c_i64, c_i32, c_vp, c_vp, c_sz, c_vp]),
     "zb_linear_state_centered": (c_i32, [c_vp, c_vp, c_vp, c_i32, c_i64, c_i32, c_vp, c_vp, c_vp, c_sz, c_vp]),
+    "zb_block_mass": (c_i32, [c_vp, c_vp, c_vp, ZbShape, c_f32, c_vp, c_vp]),
+    "zb_block_mass_top_fraction": (c_i32, [c_vp, c_i32, c_i32, c_i32, c_vp, c_vp]),
+    "zb_block_mass_selected_fraction": (c_i32, [c_vp, c_i32, c_i32, c_vp, c_i32, c_vp, c_vp]),
     "zb_affine_fit_workspace_bytes": (c_sz, [c_i32, c_i64, c_i32]),
     "zb_affine_fit": (c_i32, [c_vp, c_vp, c_i32, c_i64, c_i32, c_vp, c_vp, c_vp, c_sz, c_vp]),
     "zb_gather_tiles": (c_i32, [c_vp, ZbShape, c_vp, c_i32, c_vp, c_vp]),

@@ -136,6 +136,19 @@ def test_validation_errors_before_launch(lib):
     assert lib.zb_linear_state_centered(FAKE, FAKE, FAKE, 2, 256, 64, FAKE, FAKE, FAKE, need - 1, None) == 5
     assert lib.zb_linear_state_centered(FAKE, FAKE, FAKE, 2, 256, 16, FAKE, FAKE, FAKE, need, None) == 4
     assert lib.zb_linear_state_centered(FAKE, FAKE, FAKE, 0, 256, 64, FAKE, FAKE, FAKE, need, None) == 2
+    # block-mass diagnostic
+    assert lib.zb_block_mass(FAKE, FAKE, FAKE, _shape(t=96), 0.125, FAKE, None) == 4
+    assert lib.zb_block_mass(FAKE, FAKE, None, S, 0.125, FAKE, None) == 1
+    assert lib.zb_block_mass(FAKE, FAKE, FAKE, S, 0.0, FAKE, None) == 2
+    assert lib.zb_block_mass(FAKE + 2, FAKE, FAKE, S, 0.125, FAKE, None) == 3
+    assert lib.zb_block_mass(FAKE, FAKE, FAKE, _shape(N=64 * 50000), 0.125, FAKE, None) == 4  # Tb > 49152
+    assert lib.zb_block_mass_top_fraction(FAKE, 2, 4, 5, FAKE, None) == 2                     # m > n_blocks
+    assert lib.zb_block_mass_top_fraction(FAKE, 2, 4, -1, FAKE, None) == 2
+    assert lib.zb_block_mass_top_fraction(None, 2, 4, 1, FAKE, None) == 1
+    assert lib.zb_block_mass_top_fraction(FAKE, 2, 60000, 1, FAKE, None) == 4
+    assert lib.zb_block_mass_selected_fraction(FAKE, 2, 4, FAKE, 0, FAKE, None) == 2
+    assert lib.zb_block_mass_selected_fraction(FAKE, 2, 4, None, 2, FAKE, None) == 1
+    assert lib.zb_block_mass_selected_fraction(FAKE + 4, 2, 4, FAKE, 2, FAKE, None) == 3
     # gather
     assert lib.zb_gather_tiles(FAKE, S, FAKE, 0, FAKE, None) == 2
     assert lib.zb_gather_tiles(FAKE, S, None, 2, FAKE, None) == 1
