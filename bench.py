@@ -336,8 +336,17 @@ def config_dict(w):
                         f"fit on {len(synth.calibration_tiles(w.n_tiles, w.calib_tiles)) * w.tile} rows; "
                         f"0.5L/0.5S hybrid",
             "heads": w.heads, "n_tokens": w.n_tokens, "head_dim": w.head_dim, "tile": w.tile, "k": w.k,
-            "linear_fraction": 0.5, "l2": "inputs larger than L2 (each of Q, K, V, O is "
-            f"{w.heads * w.n_tokens * w.head_dim * 2 / 1e9:.2f} GB)"}
+            "linear_fraction": 0.5, "l2": l2_note(w.heads * w.n_tokens * w.head_dim * 2)}
+
+
+L2_BYTES = 126e6
+
+
+def l2_note(tensor_bytes: float) -> str:
+    size = f"each of Q, K, V, O is {tensor_bytes / 1e9:.2f} GB"
+    if tensor_bytes > L2_BYTES:
+        return f"inputs larger than L2 ({size})"
+    return f"inputs smaller than L2 ({size}; the four together {4 * tensor_bytes / 1e9:.2f} GB)"
 
 
 def main():
