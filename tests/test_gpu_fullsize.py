@@ -85,3 +85,30 @@ def test_linear_stage_1024_views_full_size_sampled():
     got = host(o_l[h, srows])
     err = np.abs(got - want).max() / np.abs(want).max()
     assert err <= REL_TOL, err
+
+
+def test_linear_stage_512_views_layer1_full_size_sampled():
+    """A linear layer of the 512-view stack (layer 1, its own seed): 16 x 703,488 tokens,
+    calibration and output on the GPU, one head fitted in full by the oracle."""
+    import linear_hybrid_attention_b200 as zb
+    w = workload("stack512")
+    assert 1 in w.linear_layers
+    Q, K, V = synth.make_qkv(w, device="cuda", seed=synth.default_seed(w, layer=1))
+    calib = synth.calibration_tiles(w.n_tiles, w.calib_tiles)
+    layer = zb.HybridLayer(w.heads, w.n_tokens, w.tile, w.k, calib)
+    layer.calibrate(Q, K, V)
+    o_l = layer.linear(Q, K, V)
+    sync_ok()
+    h = 10
+    q64, k64, v64 = host(Q[h:h + 1]), host(K[h:h + 1]), host(V[h:h + 1])
+    rows = oracle.calibration_rows(w.n_tokens, w.tile, calib)
+    X = oracle.linear_attention(q64[:, rows], k64, v64)
+    Y = np.concatenate([oracle.dense_attention(q64[:, rows[c:c + 128]], k64, v64, 1 / 8)
+                        for c in range(0, len(rows), 128)], axis=1)
+    A, b = oracle.affine_fit(X, Y)
+    tiles = [0, 2748, w.n_tiles - 1]
+    srows = oracle.calibration_rows(w.n_tokens, w.tile, tiles)
+    want = oracle.linear_attention(q64[:, srows], k64, v64, A, b)[0]
+    got = host(o_l[h, srows])
+    err = np.abs(got - want).max() / np.abs(want).max()
+    assert err <= REL_TOL, err
