@@ -347,8 +347,8 @@ def block_mass(Q, K, scale: float, block: int) -> np.ndarray:
 def top_mass_fraction(M, m: int) -> np.ndarray:
     """Share of each query block's mass held by its m heaviest key blocks -> [H, T].
 
-    Reading of the pages' "highest-mass 20% of 64 x 64 token blocks" (Figure 2
-    (b), Figure 8): the selection is made per query block, like the method's
+    Reading: the pages' selection of the heaviest 20% of 64 x 64 token blocks
+    (Figure 2 (b), Figure 8) is made per query block, like the method's
     per-query-tile selection, with m = ceil(0.2 T) supplied by the caller.
     """
     M = _f64(M)
