@@ -285,9 +285,11 @@ zb_status zb_block_mass_selected_fraction(const float* M, int32_t heads, int32_t
  * Closed-form affine fit (Abstract: closed-form affine fitting makes the
  * conversion training-free; Table 3 (a) of "Zebra3D: Efficient Hybrid
  * Foundation Models ..." compares no fit with fitted variants): per head, the
- * least-squares solution of [X 1] [A; b] = Y over R calibration rows, with a
- * vanishing ridge lam = 1e-8 * max_i ((X - mean X)^T (X - mean X))_ii on A so
- * that calibration outputs varying in fewer than d directions stay solvable.
+ * least-squares solution of [X 1] [A; b] = Y over R calibration rows whose A
+ * has minimum norm, computed with a vanishing ridge
+ * lam = 1e-8 * max_i ((X - mean X)^T (X - mean X))_ii on A, so that calibration
+ * outputs varying in fewer than d directions stay solvable (the linear stage's
+ * outputs always do: each row satisfies O . (S^-1 z) = 1).
  * Solved in fp64: row means, centred Gram matrices, Cholesky factorisation.
  *   in : X fp32 [H][R][d] (unfitted linear output), Y fp32 [H][R][d] (dense
  *        output on the same rows);  R >= d + 1;  ws of >=

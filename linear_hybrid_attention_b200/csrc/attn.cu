@@ -355,7 +355,7 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
             if (p.wave)
                 for (int r = arrived + 1; r < R; ++r) atomicAdd(p.wave, 1u);
             volatile int no_abort = 0;
-            const WaitCtx w2{p.status, &no_abort, p.timeout_ns};
+            const WaitCtx w2{p.status, &no_abort, drain_timeout_ns(p.timeout_ns)};
             for (int st = 0; st < K_STAGES; ++st)
                 if ((k_issued >> st) & 1u) mbar_wait(smem_addr(&b.k_full[st]), (k_par >> st) & 1u, w2);
             for (int st = 0; st < V_STAGES; ++st)
@@ -421,7 +421,7 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
             // no tcgen05.mma of this thread may still run when TMEM is released
             umma_commit(smem_addr(&b.drain));
             volatile int no_abort = 0;
-            const WaitCtx w2{p.status, &no_abort, p.timeout_ns};
+            const WaitCtx w2{p.status, &no_abort, drain_timeout_ns(p.timeout_ns)};
             mbar_wait(smem_addr(&b.drain), 0, w2);
         }
         __syncwarp();
@@ -478,7 +478,7 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
             // their own (the selected-tile loop holds no landmark code).
             auto step = [&](auto lm_tag, int j) -> bool {
                 constexpr bool is_lm = decltype(lm_tag)::value;
-                if (!mbar_wait(smem_addr(&b.s_full), ph, wc)) return false;
+                if (!mbar_wait_warp(smem_addr(&b.s_full), ph, wc)) return false;
                 tc_fence_after();
                 float x[BN];
                 {
@@ -507,7 +507,7 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                     // chunk) then gets log2(n_last) instead
                     const int j0 = (j - p.k) * BN;
                     if (j == p.k) {  // first landmark step: every thread's bits are in
-                        if (!mbar_wait(smem_addr(&sm.bm_ready[s][r & 1]), (r >> 1) & 1, wc)) return false;
+                        if (!mbar_wait_warp(smem_addr(&sm.bm_ready[s][r & 1]), (r >> 1) & 1, wc)) return false;
                     }
                     uint32_t bits[BN / 32];
 #pragma unroll
@@ -591,7 +591,7 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                 // P is free once P V of the previous step is done; O then holds
                 // every earlier step and can be rescaled (the exponentials above
                 // overlap that P V)
-                if (!mbar_wait(smem_addr(&b.p_free), ph ^ 1u, wc)) return false;
+                if (!mbar_wait_warp(smem_addr(&b.p_free), ph ^ 1u, wc)) return false;
                 tc_fence_after();
                 if (rescale && j > 0) {
 #pragma unroll 1
@@ -620,7 +620,7 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
             // ------------------------------------------------ epilogue ----
             // P V of the item's last step (parity ph ^ 1) has completed, so every
             // thread of the slot is past its landmark steps: clear this item's bits
-            if (!mbar_wait(smem_addr(&b.p_free), ph ^ 1u, wc)) { ok = false; break; }
+            if (!mbar_wait_warp(smem_addr(&b.p_free), ph ^ 1u, wc)) { ok = false; break; }
             tc_fence_after();
             if (list && p.lm_chunks) {
                 for (int q = row; q < p.k; q += BM) {

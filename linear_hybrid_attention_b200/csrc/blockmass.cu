@@ -203,7 +203,7 @@ block_mass_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant_
     // ---- drain: no MMA may run and no TMA may write once TMEM and shared memory go
     {
         volatile int no_abort = 0;
-        const WaitCtx w2{status, &no_abort, timeout_ns};
+        const WaitCtx w2{status, &no_abort, drain_timeout_ns(timeout_ns)};
         if (tid == 0) {
             umma_commit(smem_addr(&sm.done));
             mbar_wait(smem_addr(&sm.done), 0, w2);

@@ -120,7 +120,7 @@ landmark_kernel(const uint16_t* __restrict__ Q, const uint16_t* __restrict__ K,
             }
             // leave no bulk copy in flight (bounded, even after an abort)
             volatile int no_abort = 0;
-            const WaitCtx w2{status, &no_abort, timeout_ns};
+            const WaitCtx w2{status, &no_abort, drain_timeout_ns(timeout_ns)};
             for (int s = 0; s < LM_STAGES; ++s)
                 if ((issued_mask >> s) & 1u) mbar_wait(smem_addr(&sm.full[s]), (par_mask >> s) & 1u, w2);
         }
@@ -132,7 +132,7 @@ landmark_kernel(const uint16_t* __restrict__ Q, const uint16_t* __restrict__ K,
             const uint32_t use = static_cast<uint32_t>(it / LM_STAGES), pu = static_cast<uint32_t>(it >> 1);
             int h, j, n;
             item_of(it, h, j, n);
-            if (!mbar_wait(smem_addr(&sm.full[s]), use & 1, wc)) break;
+            if (!mbar_wait_warp(smem_addr(&sm.full[s]), use & 1, wc)) break;
             const int r0 = warp * 8;
             const int rows = max(0, min(8, n - r0));
             double acc[3][2];
@@ -170,7 +170,7 @@ landmark_kernel(const uint16_t* __restrict__ Q, const uint16_t* __restrict__ K,
             __syncwarp();
             if (lane == 0) mbar_arrive(smem_addr(&sm.empty[s]));
             // partial table pb is free once the item two back was reduced
-            if (!mbar_wait(smem_addr(&sm.pempty[pb]), (pu & 1) ^ 1, wc)) break;
+            if (!mbar_wait_warp(smem_addr(&sm.pempty[pb]), (pu & 1) ^ 1, wc)) break;
 #pragma unroll
             for (int t = 0; t < 3; ++t) {
                 sm.part[pb][warp][t][2 * lane] = acc[t][0];
@@ -180,7 +180,7 @@ landmark_kernel(const uint16_t* __restrict__ Q, const uint16_t* __restrict__ K,
             if (lane == 0) mbar_arrive(smem_addr(&sm.pfull[pb]));
             if (tid < 3 * HD) {
                 // fixed-order reduction of the 16 partials, one output per thread
-                if (!mbar_wait(smem_addr(&sm.pfull[pb]), pu & 1, wc)) break;
+                if (!mbar_wait_warp(smem_addr(&sm.pfull[pb]), pu & 1, wc)) break;
                 const int t = tid / HD, col = tid % HD;
                 double sum = 0.0;
 #pragma unroll

@@ -231,7 +231,7 @@ __device__ __forceinline__ void linear_state_body(const CUtensorMap& tm_k, const
     // ---- drain: no MMA may run and no TMA may write once we read and free
     {
         volatile int no_abort = 0;
-        const WaitCtx w2{status, &no_abort, timeout_ns};
+        const WaitCtx w2{status, &no_abort, drain_timeout_ns(timeout_ns)};
         if (tid == 0) {
             umma_commit(smem_addr(&sm.done));
             for (uint32_t q = static_cast<uint32_t>(consumed); q < issued; ++q)
@@ -501,7 +501,7 @@ linear_apply_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
             }
             // leave no TMA write in flight (bounded, even after an abort)
             volatile int no_abort = 0;
-            const WaitCtx w2{status, &no_abort, timeout_ns};
+            const WaitCtx w2{status, &no_abort, drain_timeout_ns(timeout_ns)};
             for (int s = 0; s < AP_STAGES; ++s)
                 if ((issued_mask >> s) & 1u) mbar_wait(smem_addr(&sm.q_full[s]), (consumed_par >> s) & 1u, w2);
         }
@@ -537,7 +537,7 @@ linear_apply_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
             }
             // no MMA may still run when TMEM is released
             volatile int no_abort = 0;
-            const WaitCtx w2{status, &no_abort, timeout_ns};
+            const WaitCtx w2{status, &no_abort, drain_timeout_ns(timeout_ns)};
             umma_commit(smem_addr(&sm.drain));
             mbar_wait(smem_addr(&sm.drain), 0, w2);
         }

@@ -94,6 +94,14 @@ struct WaitCtx {
     uint64_t timeout_ns;
 };
 
+// Limit of a drain wait: after an abort, a role still waits for the bulk
+// copies and MMAs it has already issued before the CTA frees its shared memory
+// and TMEM.  Those waits use at least this limit, whatever limit the aborted
+// waits had, so a short configured limit never lets a CTA exit while a copy or
+// an MMA still writes its memory.
+constexpr uint64_t DRAIN_FLOOR_NS = 2000000000ull;  // 2 s
+ZB_DEVINL uint64_t drain_timeout_ns(uint64_t t) { return t > DRAIN_FLOOR_NS ? t : DRAIN_FLOOR_NS; }
+
 // Wait until the phase of `bar` with the given parity has completed.  Gives up
 // (returns false) when another role of the CTA aborted or after timeout_ns;
 // in the latter case records ZB_ERR_TIMEOUT and raises the CTA abort flag.
@@ -129,6 +137,14 @@ ZB_DEVINL bool mbar_wait_sleep(uint32_t bar, uint32_t parity, const WaitCtx& w, 
             }
         }
     }
+}
+
+// mbar_wait for code in which a whole warp waits together and then runs
+// warp-collective instructions (tcgen05.ld / st, __syncwarp): the lanes agree
+// on the outcome, a give-up by any lane being a give-up by all, so a warp never
+// reaches such an instruction with only part of its lanes.
+ZB_DEVINL bool mbar_wait_warp(uint32_t bar, uint32_t parity, const WaitCtx& w) {
+    return __all_sync(0xffffffffu, mbar_wait(bar, parity, w));
 }
 
 // ------------------------------------------------------------------ TMA ----

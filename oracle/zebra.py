@@ -293,14 +293,16 @@ def affine_fit(X, Y, ridge_rel: float = RIDGE_REL):
     in closed form (no gradient descent) against the dense layer's output on
     calibration rows.  X, Y: [H, R, d] -> A [H, d, d], b [H, d].
 
-    Reading: ordinary least squares with an intercept, plus a vanishing ridge
+    Reading: least squares with an intercept and, among its minimisers, the
+    one whose A has minimum norm, computed with a vanishing ridge
     lam = ridge_rel * max_i ((X - mean X)^T (X - mean X))_ii on A (not on b).
-    The intercept absorbs the means, so this equals OLS on the centred data,
-    A = argmin ||Xc A - Yc||^2 + lam ||A||^2, b = mean(Y) - mean(X) A.  Without
-    the ridge the problem is singular whenever the calibration outputs vary in
-    fewer than d directions (which the linear stage's outputs often nearly
-    do); the ridge only damps directions carrying under sqrt(ridge_rel) of the
-    largest singular value.  Solved as an augmented least-squares problem
+    The intercept absorbs the means, so this is least squares on the centred
+    data, A = argmin ||Xc A - Yc||^2 + lam ||A||^2, b = mean(Y) - mean(X) A,
+    which tends to the minimum-norm solution as lam -> 0.  The minimiser is
+    not unique for the linear stage: its output rows all satisfy
+    O . (S^-1 z) = 1, so the centred calibration matrix has rank d - 1.  The
+    ridge only damps directions carrying under sqrt(ridge_rel) of the largest
+    singular value.  Solved as an augmented least-squares problem
     [Xc; sqrt(lam) I] A = [Yc; 0] with an fp64 least-squares routine.
     """
     X, Y = _f64(X), _f64(Y)

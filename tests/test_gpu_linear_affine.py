@@ -120,6 +120,58 @@ def test_affine_fit_degenerate_calibration_is_finite():
     assert (fit - Y).abs().max().item() <= 1e-3 * Y.abs().max().item()
 
 
+def test_affine_fit_recovers_planted_map_to_the_ridge_bias():
+    # Y = X A0 + b0 in fp64, rounded once to fp32.  The fp64 solve returns A0, b0
+    # up to the ridge's relative bias (1e-8 * max diag G / s_min^2, about 2e-8
+    # here) and the fp32 roundings of Y and of the result (about 1e-7).
+    zb = _zb()
+    rng = np.random.default_rng(41)
+    H, R = 2, 2048
+    X = rng.standard_normal((H, R, 64)).astype(np.float32)
+    A0 = rng.standard_normal((H, 64, 64)) * 0.2
+    b0 = rng.standard_normal((H, 64))
+    Y = (X.astype(np.float64) @ A0 + b0[:, None, :]).astype(np.float32)
+    A, b = zb.zb_affine_fit(torch.from_numpy(X).cuda(), torch.from_numpy(Y).cuda())
+    sync_ok()
+    np.testing.assert_allclose(A.cpu().numpy(), A0, rtol=0, atol=1e-5)
+    np.testing.assert_allclose(b.cpu().numpy(), b0, rtol=0, atol=1e-5)
+
+
+def test_affine_fit_rank_deficient_gives_the_minimum_norm_solution():
+    # Centred calibration rows of rank 40 < 64 (explicit SVD, singular values
+    # 1..10): every least-squares minimiser fits Y, and the ridge picks the one
+    # of minimum norm, A_mn = P A* with P the projector on the rows' span and
+    # b = b* + xm (I - P) A* (closed form).  X and Y are rounded to fp32 once,
+    # which adds directions far below the ridge's cut (1e-4 of the largest).
+    zb = _zb()
+    rng = np.random.default_rng(42)
+    H, R, d, r = 2, 1024, 64, 40
+    Xs, Ys, As, bs = [], [], [], []
+    for _ in range(H):
+        U, _ = np.linalg.qr(rng.standard_normal((R, r)))
+        U -= U.mean(axis=0)
+        U, _ = np.linalg.qr(U)
+        Vr, _ = np.linalg.qr(rng.standard_normal((d, r)))
+        xm = rng.standard_normal(d)
+        X = xm + (U * np.linspace(1.0, 10.0, r)) @ Vr.T
+        A0 = rng.standard_normal((d, d))
+        b0 = rng.standard_normal(d)
+        P = Vr @ Vr.T
+        Xs.append(X)
+        Ys.append(X @ A0 + b0)
+        As.append(P @ A0)
+        bs.append(b0 + xm @ (np.eye(d) - P) @ A0)
+    X32 = np.stack(Xs).astype(np.float32)
+    Y32 = np.stack(Ys).astype(np.float32)
+    A, b = zb.zb_affine_fit(torch.from_numpy(X32).cuda(), torch.from_numpy(Y32).cuda())
+    sync_ok()
+    A_mn, b_mn = np.stack(As), np.stack(bs)
+    np.testing.assert_allclose(A.cpu().numpy(), A_mn, rtol=0, atol=1e-4 * np.abs(A_mn).max())
+    np.testing.assert_allclose(b.cpu().numpy(), b_mn, rtol=0, atol=1e-4 * np.abs(b_mn).max())
+    fit = oracle.affine_apply(X32.astype(np.float64), A.double().cpu().numpy(), b.double().cpu().numpy())
+    assert np.abs(fit - np.stack(Ys)).max() <= 1e-5 * np.abs(np.stack(Ys)).max()
+
+
 def test_linear_apply_fp32_matches_oracle():
     zb = _zb()
     w = workload("linear256", heads=3, n_tokens=5000)

@@ -401,6 +401,62 @@ def test_affine_fit_rank_deficient_calibration_is_finite():
     np.testing.assert_allclose(oracle.affine_apply(X, A, b), Y, atol=1e-6)
 
 
+def _rank_deficient_case(seed, R=300, d=16, r=10):
+    """X with centred rank r < d built from an explicit SVD Xc = U_r diag(s) V_r^T
+    (singular values 1..10), and Y = X A* + b* exactly, for a planted A* that has
+    components in the null space of Xc too."""
+    rng = np.random.default_rng(seed)
+    U, _ = np.linalg.qr(rng.standard_normal((R, r)))
+    U -= U.mean(axis=0)                      # columns orthogonal to the all-ones vector
+    U, _ = np.linalg.qr(U)
+    Vr, _ = np.linalg.qr(rng.standard_normal((d, r)))
+    s = np.linspace(1.0, 10.0, r)
+    xm = rng.standard_normal(d)
+    X = xm + (U * s) @ Vr.T
+    A0 = rng.standard_normal((d, d))
+    b0 = rng.standard_normal(d)
+    Y = X @ A0 + b0
+    return X, Y, xm, Vr, A0, b0
+
+
+def test_affine_fit_rank_deficient_is_the_minimum_norm_solution():
+    # With centred rank r < d the least-squares minimisers form an affine family;
+    # the minimum-norm one has A_mn = P A* (P = V_r V_r^T, the projector on the
+    # row space of Xc) and b = b* + xm (I - P) A*, in closed form.  The ridge
+    # (lam -> 0) converges to it: its bias is lam / s_i^2 <= 1e-8 * (10 / 1)^2.
+    for seed in (1, 2):
+        X, Y, xm, Vr, A0, b0 = _rank_deficient_case(seed)
+        P = Vr @ Vr.T
+        A_mn = P @ A0
+        b_mn = b0 + xm @ (np.eye(len(xm)) - P) @ A0
+        A, b = oracle.affine_fit(X[None], Y[None])
+        np.testing.assert_allclose(A[0], A_mn, rtol=0, atol=1e-5 * np.abs(A_mn).max())
+        np.testing.assert_allclose(b[0], b_mn, rtol=0, atol=1e-5 * np.abs(b_mn).max())
+        # fitted rows: the ridge's relative bias is at most 1e-8 * (s_max / s_min)^2 = 1e-6
+        np.testing.assert_allclose(oracle.affine_apply(X[None], A, b)[0], Y, rtol=0, atol=2e-6 * np.abs(Y).max())
+
+
+def test_linear_output_lies_on_a_hyperplane_and_the_fit_ignores_its_normal():
+    # O_r = u_r S with u_r = phi(q_r) / (phi(q_r) . z), and u_r . z = 1, so every
+    # linear-attention output row satisfies O_r . (S^-1 z) = 1: the centred
+    # calibration matrix X is rank-deficient by one for this operator, and the
+    # fitted A (the minimum-norm minimiser) has no component along v = S^-1 z.
+    rng = np.random.default_rng(5)
+    H, N, d = 2, 600, 16
+    Q = rng.standard_normal((H, N, d)) / 4
+    K = rng.standard_normal((H, N, d)) / 4
+    V = rng.standard_normal((H, N, d))
+    S, z = oracle.linear_state(K, V)
+    X = oracle.linear_attention(Q[:, :200], K, V)
+    Y = oracle.dense_attention(Q[:, :200], K, V, 0.25)
+    A, _ = oracle.affine_fit(X, Y)
+    for h in range(H):
+        v = np.linalg.solve(S[h], z[h])
+        np.testing.assert_allclose(X[h] @ v, 1.0, rtol=0, atol=1e-9)
+        vn = v / np.linalg.norm(v)
+        assert np.abs(vn @ A[h]).max() <= 1e-6 * np.abs(A[h]).max()
+
+
 def test_calibration_rows():
     rows = oracle.calibration_rows(200, 64, [3, 0])
     assert rows.tolist() == list(range(192, 200)) + list(range(0, 64))
