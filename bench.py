@@ -133,6 +133,42 @@ class ClockSampler:
                 "sm_max_mhz": max(smax) if smax else None, "reasons": reasons, "samples": len(rows)}
 
 
+# ------------------------------------------------------------ L2 / HBM ----
+L2_FLUSH_BYTES = 256 << 20   # twice the B200's 126 MB L2
+SPEC_HBM_GBS = 7700.0        # nominal HBM3e bandwidth of an HGX B200
+
+
+class L2Flush:
+    """Writes a buffer twice the size of L2, evicting whatever an earlier call left there."""
+
+    def __init__(self, device):
+        self.buf = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.int32, device=device)
+
+    def __call__(self):
+        self.buf.fill_(1)
+
+
+def read_stream_gbs(device, gib: int = 4, reps: int = 5) -> float:
+    """Read-dominated HBM rate: a sum over a buffer far larger than L2 (the
+    driver's peak is a copy, half writes), with L2 flushed between repetitions."""
+    x = torch.ones(gib << 28, dtype=torch.float32, device=device)
+    flush = L2Flush(device)
+    x.sum()
+    times = []
+    for _ in range(reps):
+        flush()
+        a = torch.cuda.Event(enable_timing=True)
+        b = torch.cuda.Event(enable_timing=True)
+        a.record()
+        x.sum()
+        b.record()
+        torch.cuda.synchronize()
+        times.append(a.elapsed_time(b) / 1e3)
+    nbytes = x.numel() * 4
+    del x, flush
+    return nbytes / min(times) / 1e9
+
+
 # --------------------------------------------------------------- CPU oracle ----
 def oracle_sample(w, Q, K, V, calib_tiles, sample_tiles=4, calib_rows=16, head=0):
     """Time the fp64 oracle on a bounded sample of one head and extrapolate.
@@ -249,7 +285,9 @@ def linear_centered_report(zb, w, layer, Q, K, V, stream, hbm, tensor_bytes, t_a
     torch.cuda.synchronize()
     reps = 5
     evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(reps)]
+    flush = L2Flush(Q.device)
     for ev in evs:
+        flush()
         centred_state(ev)
     torch.cuda.synchronize()
     zb.zb_last_device_status()
@@ -329,6 +367,56 @@ def block_mass_report(zb, w, layer, Q, K, V, stream):
     return out
 
 
+def stack_report(zb, rank, dev, stream, passes=2):
+    """The 512-view stack: 24 freshly seeded layers (12 linear at VGGT's 0.5L
+    positions, 12 tile-sparse keeping 20% of the tiles), all inputs resident
+    (24 x 3 x 1.44 GB), run by HybridStack.  Reports one serial pass with
+    per-layer events (the sum of the parts) and `passes` timed passes with the
+    next layer's input side issued ahead on a second stream."""
+    from linear_hybrid_attention_b200.stack import HybridStack
+    w = synth.WORKLOADS["stack512"]
+    L = w.layers
+    inputs = [synth.make_qkv(w, layer=l, device=dev,
+                             seed=replicas.rank_seed(synth.default_seed(w, layer=l), rank)) for l in range(L)]
+    calib = synth.calibration_tiles(w.n_tiles, w.calib_tiles)
+    stack = HybridStack(w.heads, w.n_tokens, w.tile, w.k, calib, L, w.linear_layers, device=dev)
+    stack.run(inputs)                                     # warm-up
+    torch.cuda.synchronize()
+    zb.zb_last_device_status()
+    lev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(L)]
+    a = torch.cuda.Event(enable_timing=True)
+    b = torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    stack.run(inputs, lookahead=False, layer_events=lev)
+    b.record(stream)
+    torch.cuda.synchronize()
+    serial_ms = a.elapsed_time(b)
+    per_layer = [e0.elapsed_time(e1) for e0, e1 in lev]
+    a.record(stream)
+    for _ in range(passes):
+        stack.run(inputs)
+    b.record(stream)
+    torch.cuda.synchronize()
+    zb.zb_last_device_status()
+    ahead_ms = a.elapsed_time(b) / passes
+    lin = [per_layer[l] for l in range(L) if l in stack.linear]
+    sp = [per_layer[l] for l in range(L) if l not in stack.linear]
+    out = {"workload": f"stack512: 24 layers (linear at {list(w.linear_layers)}, the others tile-sparse keeping "
+                       f"{w.k}/{w.n_tiles} tiles + landmarks), each freshly seeded; 16 heads x {w.n_tokens} tokens",
+           "mtokens_s": w.n_tokens / (ahead_ms / 1e3) / 1e6,
+           "ms_per_pass": ahead_ms, "passes": passes,
+           "serial_pass_ms": serial_ms, "sum_of_layers_ms": sum(per_layer),
+           "lookahead_saved_ms": serial_ms - ahead_ms,
+           "per_layer_ms": [round(x, 3) for x in per_layer],
+           "sparse_layer_ms_mean": statistics.mean(sp), "linear_layer_ms_mean": statistics.mean(lin),
+           "gpu_launches_per_pass": stack.launches(),
+           "note": "Mtokens/s = tokens through all 24 layers / time of one pass; linear layers include "
+                   "their calibration (dense rows + fit); inputs resident in HBM"}
+    del stack, inputs
+    torch.cuda.empty_cache()
+    return out
+
+
 def config_dict(w):
     return {"workload": f"{w.name}: {w.n_tokens // synth.TOKENS_PER_VIEW} views x {synth.TOKENS_PER_VIEW} "
                         f"tokens = {w.n_tokens} tokens, {w.heads} heads, d={w.head_dim}, bf16; tile "
@@ -362,6 +450,7 @@ def main():
     ap.add_argument("--no-dense-ref", action="store_true", help="skip the dense-attention comparator")
     ap.add_argument("--no-centered", action="store_true", help="skip the linear-centered measurements")
     ap.add_argument("--no-block-mass", action="store_true", help="skip the block-mass diagnostic")
+    ap.add_argument("--no-stack", action="store_true", help="skip the 24-layer 512-view stack")
     ap.add_argument("--profile", action="store_true", help="short run for profilers: no JSON extras")
     args = ap.parse_args()
 
@@ -584,16 +673,46 @@ def main():
         cpu = {"value": tokens_per_step / t_cpu / 1e6, "unit": UNIT, "cores": cores, "kind": "oracle",
                "sample": desc}
 
+    # read-only HBM stream rate (a second denominator for the HBM-bound kernels)
+    read_gbs = read_stream_gbs(dev)
+    for kr in kernel_rooflines.values():
+        if kr.get("bound") == "hbm":
+            kr["frac_of_read_stream"] = kr["achieved"] / read_gbs
+            kr["frac_of_spec"] = kr["achieved"] / SPEC_HBM_GBS
+    if centered is not None:
+        for kr in (centered["zb_key_mean"], centered["zb_linear_state_centered"]):
+            kr["frac_of_read_stream"] = kr["achieved"] / read_gbs
+            kr["frac_of_spec"] = kr["achieved"] / SPEC_HBM_GBS
+    hbm_peaks = {"copy_gbs (MEASURED_PEAKS.json, the roofline peak)": hbm, "read_stream_gbs (measured here)": read_gbs,
+                 "spec_gbs": SPEC_HBM_GBS}
+
+    # the step without calibration: the affine fit done once, offline, and the
+    # fitted (A, b) reused -- the linear stage is then its two passes
+    t_offline = kt["landmark"] + kt["topk"] + kt["sparse_attn"] + kt["linear_state"] + kt["linear_apply"]
+    value_fit_offline = tokens_per_step / t_offline / 1e6 * world
+
+    gpu_launches = layer.launches_per_step * args.steps
+    stack = None
+    if not args.no_stack and w.name == "views1024":
+        del Q, K, V, layer
+        torch.cuda.empty_cache()
+        stack = stack_report(zb, rank, dev, stream)
+
     if rank == 0:
         line = {"metric": METRIC, "value": tput / 1e6, "unit": UNIT, "n_gpus": world, "steps": args.steps,
                 "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
                 "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-                "config": config_dict(w), "e2e": e2e, "gpu_launches": layer.launches_per_step * args.steps,
+                "config": config_dict(w), "e2e": e2e, "gpu_launches": gpu_launches,
                 "roofline": roofline, "kernel_roofline": kernel_rooflines, "stage_ms": stage_ms,
                 "kernel_ms": {n: v * 1e3 for n, v in kt.items()}, "clocks": clk, "cpu_baseline": cpu,
                 "hybrid_0.7L_mtokens_s": hybrid_07, "dense_reference": dense_ref, "linear_centered": centered,
-                "block_mass": block_mass,
-                "peaks": peaks}
+                "block_mass": block_mass, "stack512": stack,
+                "value_definition": "value = 2 N / t_step with every call of the hot path in the step, the "
+                                    "calibration (dense attention on 4,096 rows) and the affine fit included",
+                "value_fit_offline": value_fit_offline,
+                "value_fit_offline_definition": "2 N / (landmarks + selection + tile-sparse attention + linear "
+                                                "state + fitted linear output): the fit done once, offline",
+                "hbm_peaks": hbm_peaks, "peaks": peaks}
         print(json.dumps(line), flush=True)
     if world > 1:
         torch.distributed.destroy_process_group()

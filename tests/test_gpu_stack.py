@@ -1,0 +1,164 @@
+"""GPU parity of the layer stack: every layer of a 0.5L/0.8S hybrid stack.
+
+The stack ("Zebra3D: Efficient Hybrid Foundation Models For Scalable 3D
+Reconstruction", Table 20 caption for the xL/yS notation, Table 6 for the
+linear layers' positions in VGGT's 24 global-attention layers) runs through
+``HybridStack``, the runner the bench times, with the input side of each layer
+issued ahead on a second stream.  Checks:
+
+  * the outputs are bit-identical with and without that lookahead;
+  * small stack (4 layers, ragged tiles): every output of every layer against
+    the fp64 oracle;
+  * the 512-view stack at full size (24 layers, 16 heads x 703,488 tokens,
+    k = 1,100 of 5,496 tiles, each layer freshly seeded): for every layer,
+    sampled (head, query tile) pairs -- selection bit-exact and tile-sparse
+    output within the bar for sparse layers, the fitted output (the oracle fits
+    the head on the full 4,096 calibration rows) within the bar for linear
+    layers -- and the convex-combination bound on every row of every sparse
+    layer.  The oracle runs in spawned worker processes.
+"""
+import concurrent.futures as cf
+import math
+import multiprocessing as mp
+import os
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import synth
+from tests import stack_oracle_jobs as jobs
+from tests.gpu_helpers import REL_TOL, host, rel_err_per_head, sync_ok, workload
+
+pytestmark = pytest.mark.gpu
+
+
+def _stack(w, L, linear_layers):
+    from linear_hybrid_attention_b200.stack import HybridStack
+    calib = synth.calibration_tiles(w.n_tiles, w.calib_tiles)
+    return HybridStack(w.heads, w.n_tokens, w.tile, w.k, calib, L, linear_layers), calib
+
+
+def _checksum(O):
+    return O.view(torch.int16).to(torch.int64).sum()
+
+
+def test_small_stack_matches_oracle_with_and_without_lookahead():
+    w = workload("stack512", heads=2, n_tokens=5000)          # T = 40 (ragged 8-row tile), k = 8
+    L, lin = 4, (1, 2)
+    inputs = [synth.make_qkv(w, layer=l, device="cuda") for l in range(L)]
+    stack, calib = _stack(w, L, lin)
+    outs = {}
+    for look in (True, False):
+        got = {}
+        stack.run(inputs, lookahead=look, on_layer_done=lambda l, O: got.__setitem__(l, O.clone()))
+        sync_ok()
+        outs[look] = got
+    s = 1 / math.sqrt(w.head_dim)
+    for l in range(L):
+        assert torch.equal(outs[True][l], outs[False][l]), l
+        Q64, K64, V64 = (host(t) for t in inputs[l])
+        if l in lin:
+            rows = oracle.calibration_rows(w.n_tokens, w.tile, calib)
+            A, b = oracle.affine_fit(oracle.linear_attention(Q64[:, rows], K64, V64),
+                                     oracle.dense_attention(Q64[:, rows], K64, V64, s))
+            ref = oracle.linear_attention(Q64, K64, V64, A, b)
+        else:
+            idx = oracle.select_tiles(oracle.tile_scores(oracle.landmark_means(Q64, w.tile),
+                                                         oracle.landmark_means(K64, w.tile)), w.k)
+            ref = oracle.sparse_attention(Q64, K64, V64, w.tile, idx, s)
+        err = rel_err_per_head(host(outs[True][l]), ref)
+        assert err <= REL_TOL, (l, err)
+
+
+def test_stack_512_views_all_24_layers_full_size_sampled():
+    w = workload("stack512")
+    L, lin = w.layers, w.linear_layers
+    T, t = w.n_tiles, w.tile
+    s = 1 / math.sqrt(w.head_dim)
+    torch.cuda.empty_cache()
+    inputs = [synth.make_qkv(w, layer=l, device="cuda") for l in range(L)]
+    stack, calib = _stack(w, L, lin)
+    # sampled (head, query tiles) per layer; the last tile is always among them
+    plan = {}
+    for l in range(L):
+        tiles = sorted({(977 * l + 13) % T, (2748 + 331 * l) % T, T - 1})
+        heads = [(5 * l) % w.heads] if l in lin else [(5 * l) % w.heads, (5 * l + 11) % w.heads]
+        plan[l] = (heads, tiles)
+    got, sums, bound_ok = {}, {}, {}
+
+    def hook(l, O):
+        heads, tiles = plan[l]
+        rows = torch.as_tensor(oracle.calibration_rows(w.n_tokens, t, tiles), device=O.device)
+        got[l] = {"O": O[heads][:, rows].clone(), "idx": None}
+        if l not in lin:
+            got[l]["idx"] = stack.bufs[l & 1].idx[heads][:, tiles].clone()
+            V = inputs[l][2]
+            vmax = V.amax(dim=1, keepdim=True)
+            vmin = V.amin(dim=1, keepdim=True)
+            Of = O.float()
+            bound_ok[l] = ((Of <= vmax.float() + 1e-2) & (Of >= vmin.float() - 1e-2)).all()
+            del Of
+        sums.setdefault(l, []).append(_checksum(O))
+
+    stack.run(inputs, lookahead=True, on_layer_done=hook)
+    sync_ok()
+    first = {l: (got[l]["O"].cpu(), None if got[l]["idx"] is None else got[l]["idx"].cpu()) for l in range(L)}
+    stack.run(inputs, lookahead=False, on_layer_done=lambda l, O: sums[l].append(_checksum(O)))
+    sync_ok()
+    for l in range(L):
+        assert int(sums[l][0]) == int(sums[l][1]), f"layer {l}: lookahead changed the output"
+        if l not in lin:
+            assert bool(bound_ok[l]), f"layer {l}: output outside the convex hull of V"
+
+    # oracle jobs in spawned workers, at most a few heads' inputs in flight
+    cores = len(os.sched_getaffinity(0))
+    workers = max(1, min(12, cores // 2))
+    futures = {}
+    with cf.ProcessPoolExecutor(max_workers=workers, mp_context=mp.get_context("spawn"),
+                                initializer=jobs.limit_threads, initargs=(2,)) as ex:
+        import tempfile
+        with tempfile.TemporaryDirectory() as tmp:
+            pending = set()
+            for l in range(L):
+                heads, tiles = plan[l]
+                for h in heads:
+                    while len(pending) >= workers + 2:
+                        done, pending = cf.wait(pending, return_when=cf.FIRST_COMPLETED)
+                        for f in done:
+                            for p in f.paths:
+                                os.remove(p)
+                    paths = []
+                    for name, x in zip("QKV", inputs[l]):
+                        p = os.path.join(tmp, f"l{l}_h{h}_{name}.npy")
+                        np.save(p, synth.bf16_bits(x[h]))
+                        paths.append(p)
+                    if l in lin:
+                        f = ex.submit(jobs.linear_job, paths, t, [int(c) for c in calib], tiles, s)
+                    else:
+                        f = ex.submit(jobs.sparse_job, paths, t, w.k, tiles, s)
+                    f.paths = paths
+                    pending.add(f)
+                    futures[(l, h)] = f
+                inputs[l] = None                       # this layer's inputs are no longer needed
+            del inputs
+            torch.cuda.empty_cache()
+            results = {key: f.result() for key, f in futures.items()}
+    n = oracle.tile_lengths(w.n_tokens, t)
+    for l in range(L):
+        heads, tiles = plan[l]
+        O, idx = first[l]
+        for slot, h in enumerate(heads):
+            res = results[(l, h)]
+            ref = res if l in lin else res[1]
+            if l not in lin:
+                assert np.array_equal(idx[slot].numpy(), res[0]), (l, h)
+            gotO = host(O[slot])
+            off = 0
+            for m, i in enumerate(tiles):
+                want = ref[m * t: m * t + n[i]] if l not in lin else ref[off: off + n[i]]
+                part = gotO[off: off + n[i]]
+                err = np.abs(part - want).max() / np.abs(want).max()
+                assert err <= REL_TOL, (l, h, i, err)
+                off += n[i]
