@@ -417,6 +417,50 @@ def stack_report(zb, rank, dev, stream, passes=2):
     return out
 
 
+def spatial_report(zb, dev, stream):
+    """Spatial tiles on the 32-view recipe with 2-D positional locality (16 heads,
+    k = 69 of 344 tiles): time of the tile-sparse stage with the tokens reordered
+    into 8 x 16 patch windows (gathers in and out included) against the plain
+    stage, and the dense-softmax mass each tiling keeps on head 0: the heaviest
+    k tiles, and the k tiles the method selects."""
+    w = synth.WORKLOADS["spatial32"]
+    views = w.n_tokens // synth.TOKENS_PER_VIEW
+    Q, K, V = synth.make_qkv(w, device=dev)
+    geom = (views, synth.GRID, synth.SPECIALS, 8, 16)
+    plain = zb.HybridLayer(w.heads, w.n_tokens, w.tile, w.k, [0], device=dev)
+    spat = zb.HybridLayer(w.heads, w.n_tokens, w.tile, w.k, [0], device=dev, spatial=geom)
+    out = {"workload": f"spatial32: {views} views x {synth.TOKENS_PER_VIEW} tokens, 16 heads, keep {w.k}/{w.n_tiles} "
+                       f"tiles; queries and keys carry a 2-D positional component (scale {w.pos_scale}, length "
+                       f"{w.pos_length} patches)", "windows": "8 x 16 patches"}
+    for name, layer in (("row_major_tiles", plain), ("window_tiles", spat)):
+        layer.sparse(Q, K, V)
+        torch.cuda.synchronize()
+        a = torch.cuda.Event(enable_timing=True)
+        b = torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(3):
+            layer.sparse(Q, K, V)
+        b.record(stream)
+        torch.cuda.synchronize()
+        zb.zb_last_device_status()
+        q1 = (layer.Qp if layer.spatial else Q)[:1].contiguous()
+        k1 = (layer.Kp if layer.spatial else K)[:1].contiguous()
+        v1 = (layer.Vp if layer.spatial else V)[:1].contiguous()
+        _, lse = zb.zb_dense_attn(q1, k1, v1, layer.scale, want_lse=True)
+        M = zb.zb_block_mass(q1, k1, lse, w.tile, layer.scale)
+        top = zb.zb_block_mass_top_fraction(M, w.k)
+        sel = zb.zb_block_mass_selected_fraction(M, layer.idx[:1].contiguous())
+        torch.cuda.synchronize()
+        zb.zb_last_device_status()
+        out[name] = {"stage_ms": a.elapsed_time(b) / 3, "retained_mass_top_k_tiles": float(top.mean()),
+                     "retained_mass_method_selection": float(sel.mean())}
+    out["note"] = ("retained mass: mean over query tiles of head 0 of the dense-softmax mass in the kept key "
+                   "tiles; the window stage time includes the three gathers in and the one out")
+    del plain, spat, Q, K, V
+    torch.cuda.empty_cache()
+    return out
+
+
 def config_dict(w):
     return {"workload": f"{w.name}: {w.n_tokens // synth.TOKENS_PER_VIEW} views x {synth.TOKENS_PER_VIEW} "
                         f"tokens = {w.n_tokens} tokens, {w.heads} heads, d={w.head_dim}, bf16; tile "
@@ -445,16 +489,22 @@ def main():
     ap.add_argument("--workload", default="views1024", choices=sorted(synth.WORKLOADS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--keep-frac", type=float, default=None, help="override the kept fraction of key tiles")
+    ap.add_argument("--heads", type=int, default=None,
+                    help="override the head count (a reduced case at full length, for profilers)")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--no-dense-ref", action="store_true", help="skip the dense-attention comparator")
     ap.add_argument("--no-centered", action="store_true", help="skip the linear-centered measurements")
     ap.add_argument("--no-block-mass", action="store_true", help="skip the block-mass diagnostic")
     ap.add_argument("--no-stack", action="store_true", help="skip the 24-layer 512-view stack")
+    ap.add_argument("--no-spatial", action="store_true", help="skip the spatial-tiles measurement")
     ap.add_argument("--profile", action="store_true", help="short run for profilers: no JSON extras")
     args = ap.parse_args()
 
     w = synth.WORKLOADS[args.workload]
+    if args.heads is not None:
+        import dataclasses
+        w = dataclasses.replace(w, heads=args.heads)
     if args.keep_frac is not None:
         import dataclasses
         w = dataclasses.replace(w, keep_frac=args.keep_frac, k_fixed=None)
@@ -692,6 +742,9 @@ def main():
     value_fit_offline = tokens_per_step / t_offline / 1e6 * world
 
     gpu_launches = layer.launches_per_step * args.steps
+    spatial = None
+    if not args.no_spatial and w.name == "views1024":
+        spatial = spatial_report(zb, dev, stream)
     stack = None
     if not args.no_stack and w.name == "views1024":
         del Q, K, V, layer
@@ -706,7 +759,7 @@ def main():
                 "roofline": roofline, "kernel_roofline": kernel_rooflines, "stage_ms": stage_ms,
                 "kernel_ms": {n: v * 1e3 for n, v in kt.items()}, "clocks": clk, "cpu_baseline": cpu,
                 "hybrid_0.7L_mtokens_s": hybrid_07, "dense_reference": dense_ref, "linear_centered": centered,
-                "block_mass": block_mass, "stack512": stack,
+                "block_mass": block_mass, "stack512": stack, "spatial_tiles": spatial,
                 "value_definition": "value = 2 N / t_step with every call of the hot path in the step, the "
                                     "calibration (dense attention on 4,096 rows) and the affine fit included",
                 "value_fit_offline": value_fit_offline,

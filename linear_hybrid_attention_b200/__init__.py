@@ -29,7 +29,7 @@ __all__ = [
     "zb_tile_sparse_attn", "zb_dense_attn", "zb_linear_state", "zb_linear_apply", "zb_linear_attn",
     "zb_affine_fit", "zb_gather_tiles", "zb_last_device_status", "HybridLayer",
     "LAUNCHES_PER_CALL", "zb_key_mean", "zb_linear_state_centered", "zb_block_mass",
-    "zb_block_mass_top_fraction", "zb_block_mass_selected_fraction",
+    "zb_block_mass_top_fraction", "zb_block_mass_selected_fraction", "zb_spatial_order", "zb_gather_rows",
 ]
 
 HEAD_DIM = 64
@@ -41,7 +41,7 @@ LAUNCHES_PER_CALL = {
     "zb_landmark_build": 1, "zb_tile_score_topk": 2, "zb_tile_sparse_attn": 1, "zb_dense_attn": 1,
     "zb_linear_state": 2, "zb_linear_apply": 1, "zb_linear_attn": 3, "zb_affine_fit": 3, "zb_gather_tiles": 1,
     "zb_key_mean": 2, "zb_linear_state_centered": 2, "zb_block_mass": 1, "zb_block_mass_top_fraction": 1,
-    "zb_block_mass_selected_fraction": 1,
+    "zb_block_mass_selected_fraction": 1, "zb_gather_rows": 1, "zb_spatial_order": 0,
 }
 
 
@@ -391,6 +391,30 @@ def zb_gather_tiles(X, tile: int, tiles: torch.Tensor, out: Optional[torch.Tenso
     return O
 
 
+def zb_spatial_order(views: int, grid: int = 37, specials: int = 5, win_rows: int = 8, win_cols: int = 16):
+    """Token order grouping each view's patches into 2-D windows, and its inverse
+    (int32 CPU tensors of views * (specials + grid^2) entries; see zb.h)."""
+    n = views * (specials + grid * grid)
+    order = torch.empty(n, dtype=torch.int32)
+    inverse = torch.empty(n, dtype=torch.int32)
+    st = _lib_handle().zb_spatial_order(views, grid, specials, win_rows, win_cols, order.data_ptr(),
+                                        inverse.data_ptr())
+    _check(st, "zb_spatial_order")
+    return order, inverse
+
+
+def zb_gather_rows(X, rows: torch.Tensor, out: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """out[h, r] = X[h, rows[r]] for a bf16 [H, N, d] tensor (rows: int32 CUDA tensor)."""
+    _need(X, torch.bfloat16, "X", 3)
+    _need(rows, torch.int32, "rows", 1)
+    H, N, d = X.shape
+    n = rows.numel()
+    O = _out((H, n, d), torch.bfloat16, X.device, out, "out")
+    st = _lib_handle().zb_gather_rows(_ptr(X), H, N, n, d, _ptr(rows), _ptr(O), _stream())
+    _check(st, "zb_gather_rows")
+    return O
+
+
 def zb_last_device_status() -> None:
     """Synchronise the current stream and raise if a kernel recorded a device-side error."""
     st = _lib_handle().zb_last_device_status(_stream())
@@ -410,7 +434,8 @@ class HybridLayer:
     """
 
     def __init__(self, heads: int, n_tokens: int, tile: int, k: int, calib_tiles: Sequence[int],
-                 device="cuda", scale: Optional[float] = None, centered: bool = False):
+                 device="cuda", scale: Optional[float] = None, centered: bool = False,
+                 spatial: Optional[Sequence[int]] = None):
         d = HEAD_DIM
         self.centered = centered
         self.heads, self.n_tokens, self.tile, self.k, self.d = heads, n_tokens, tile, k, d
@@ -444,6 +469,17 @@ class HybridLayer:
         self.b = torch.empty(H, d, dtype=torch.float32, device=dev)
         self.ws_fit = torch.empty(max(affine_fit_workspace_bytes(H, max(R, d + 1), d), 16), dtype=torch.uint8,
                                   device=dev)
+        # spatial tiles: (views, grid, specials, win_rows, win_cols); the sparse stage
+        # runs on the tokens gathered into zb_spatial_order's order
+        self.spatial = None
+        if spatial is not None:
+            order, inverse = zb_spatial_order(*spatial)
+            if order.numel() != N:
+                raise ValueError(f"spatial geometry gives {order.numel()} tokens, the layer has {N}")
+            self.spatial = tuple(spatial)
+            self.order, self.inverse = order.to(dev), inverse.to(dev)
+            self.Qp, self.Kp, self.Vp, self.Op = (torch.empty(H, N, d, dtype=torch.bfloat16, device=dev)
+                                                  for _ in range(4))
 
     # kernel launches of each method (the selection's count depends on the
     # shape and workspace: see launches_per_step)
@@ -456,11 +492,21 @@ class HybridLayer:
     }
 
     def sparse(self, Q, K, V) -> torch.Tensor:
+        if self.spatial is not None:
+            # spatial tiles: the same stage on the reordered tokens, the output put back
+            zb_gather_rows(Q, self.order, out=self.Qp)
+            zb_gather_rows(K, self.order, out=self.Kp)
+            zb_gather_rows(V, self.order, out=self.Vp)
+            Q, K, V = self.Qp, self.Kp, self.Vp
         zb_landmark_build(Q, K, V, self.tile, out=self.lm)
         zb_tile_score_topk(self.lm.Qbar, self.lm.Kbar, self.n_tokens, self.tile, self.k, out=self.idx,
                            ws=self.ws_topk)
-        return zb_tile_sparse_attn(Q, K, V, self.lm.Kbar_bf16, self.lm.Vbar_bf16, self.idx, self.k,
-                                   self.tile, True, self.scale, out=self.O_sparse, ws=self.ws_attn)
+        out = self.O_sparse if self.spatial is None else self.Op
+        O = zb_tile_sparse_attn(Q, K, V, self.lm.Kbar_bf16, self.lm.Vbar_bf16, self.idx, self.k,
+                                self.tile, True, self.scale, out=out, ws=self.ws_attn)
+        if self.spatial is not None:
+            O = zb_gather_rows(O, self.inverse, out=self.O_sparse)
+        return O
 
     def _state(self, K, V):
         if self.centered:
@@ -492,5 +538,7 @@ class HybridLayer:
     @property
     def launches_per_step(self) -> int:
         extra = LAUNCHES_PER_CALL["zb_key_mean"] if self.centered else 0
+        if self.spatial is not None:
+            extra += 4 * LAUNCHES_PER_CALL["zb_gather_rows"]
         topk = topk_launches(self.heads, self.T, self.k, self.ws_topk.numel())
         return self.LAUNCHES["sparse"] + topk + self.LAUNCHES["calibrate"] + extra + self.LAUNCHES["linear"]

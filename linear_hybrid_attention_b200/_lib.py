@@ -36,6 +36,8 @@ PROTOTYPES = {
     "zb_linear_state_static_scratch_bytes": (c_sz, []),
     "zb_linear_state_static": (c_i32, [c_vp, c_vp, c_i32, c_i64, c_i32, c_vp, c_vp, c_vp]),
     "zb_linear_apply": (c_i32, [c_vp, c_i32, c_i64, c_i32, c_vp, c_vp, c_vp, c_vp, c_vp, c_i32, c_vp]),
+    "zb_spatial_order": (c_i32, [c_i32, c_i32, c_i32, c_i32, c_i32, c_vp, c_vp]),
+    "zb_gather_rows": (c_i32, [c_vp, c_i32, c_i64, c_i64, c_i32, c_vp, c_vp, c_vp]),
     "zb_linear_attn_workspace_bytes": (c_sz, [c_i32, c_i64, c_i32]),
     "zb_linear_attn": (c_i32, [c_vp, c_vp, c_vp, c_i32, c_i64, c_i32, c_vp, c_vp, c_vp, c_vp, c_sz, c_vp]),
     "zb_key_mean_workspace_bytes": (c_sz, [c_i32, c_i64, c_i32]),

@@ -593,14 +593,17 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                 // overlap that P V)
                 if (!mbar_wait_warp(smem_addr(&b.p_free), ph ^ 1u, wc)) return false;
                 tc_fence_after();
-                if (rescale && j > 0) {
+                // the rescale is decided per row, but tcgen05.ld / st are warp-collective:
+                // the whole warp takes the branch and rows without a rescale multiply by 1
+                if (__any_sync(0xffffffffu, rescale && j > 0)) {
+                    const float a = (rescale && j > 0) ? alpha : 1.f;
 #pragma unroll 1
                     for (int c = 0; c < HD / 32; ++c) {
                         uint32_t ro[32];
                         tmem_ld32(tm_o + c * 32, ro);
                         tmem_wait_ld_dep(ro);
 #pragma unroll
-                        for (int e = 0; e < 32; ++e) ro[e] = __float_as_uint(__uint_as_float(ro[e]) * alpha);
+                        for (int e = 0; e < 32; ++e) ro[e] = __float_as_uint(__uint_as_float(ro[e]) * a);
                         tmem_st32(tm_o + c * 32, ro);
                         tmem_wait_st();
                     }

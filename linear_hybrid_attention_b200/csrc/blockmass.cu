@@ -146,7 +146,10 @@ block_mass_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant_
         const int s = j & 1;
         bool good = true;
         if (tid == 0 && j + 1 < T) good = issue_mma(j + 1);
-        if (good) good = mbar_wait(smem_addr(&sm.s_full[s]), (j >> 1) & 1, wc);
+        // the lanes of a warp agree before the warp-collective TMEM loads below
+        // (lane 0 of warp 0 may have given up in issue_mma)
+        good = __all_sync(0xffffffffu, good);
+        if (good) good = mbar_wait_warp(smem_addr(&sm.s_full[s]), (j >> 1) & 1, wc);
         float sum0 = 0.f, sum1 = 0.f;
         if (good) {
             tc_fence_after();

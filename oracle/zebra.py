@@ -50,6 +50,7 @@ __all__ = [
     "linear_apply", "linear_attention", "linear_attention_quadratic", "affine_fit",
     "affine_apply", "calibration_rows", "RIDGE_REL", "key_mean", "linear_state_centered",
     "linear_attention_centered", "block_mass", "top_mass_fraction", "selected_mass_fraction",
+    "spatial_order", "inverse_order", "spatial_sparse_attention",
 ]
 
 
@@ -375,3 +376,51 @@ def calibration_rows(n_tokens: int, tile: int, tiles: Sequence[int]) -> np.ndarr
     n = tile_lengths(n_tokens, tile)
     rows = [np.arange(j * tile, j * tile + n[j]) for j in tiles]
     return np.concatenate(rows).astype(np.int64)
+
+
+def spatial_order(views: int, grid: int = 37, specials: int = 5, win_rows: int = 8, win_cols: int = 16) -> np.ndarray:
+    """Token order that groups each view's patch tokens into 2-D windows -> int64 [views * tokens].
+
+    "3D reconstruction drops dense attention layer by layer ...", synopsis:
+    exact softmax over selected *spatial* tiles.  Reading: a view holds
+    ``specials`` camera/register tokens followed by its grid x grid patch
+    tokens in row-major order (patch (y, x) at offset specials + grid*y + x).
+    The new order keeps the views in sequence; inside a view the special
+    tokens come first, then the patches window by window -- windows of
+    win_rows x win_cols patches (those at the right and bottom edges smaller),
+    taken in row-major order over the window grid, patches row-major inside a
+    window.  Position p of the new sequence holds original token order[p];
+    contiguous tiles of the new sequence then cover compact 2-D regions.
+    """
+    per_view = specials + grid * grid
+    one = list(range(specials))
+    for wy in range(0, grid, win_rows):
+        for wx in range(0, grid, win_cols):
+            for y in range(wy, min(wy + win_rows, grid)):
+                for x in range(wx, min(wx + win_cols, grid)):
+                    one.append(specials + grid * y + x)
+    one = np.asarray(one, dtype=np.int64)
+    return np.concatenate([v * per_view + one for v in range(views)])
+
+
+def inverse_order(order) -> np.ndarray:
+    """inv with inv[order[p]] = p: position of each original token in the new order."""
+    order = np.asarray(order, dtype=np.int64)
+    inv = np.empty_like(order)
+    inv[order] = np.arange(order.shape[0], dtype=np.int64)
+    return inv
+
+
+def spatial_sparse_attention(Q, K, V, tile: int, order, scale: float, k: int,
+                             use_landmarks: bool = True) -> np.ndarray:
+    """Tile-sparse attention over spatial tiles: the tokens are put in ``order``
+    (``spatial_order``), tiled, selected (mean-pooled scores, top k) and attended
+    exactly as in ``sparse_attention``, and each output row goes back to its
+    token's original position.  Softmax attention itself does not depend on the
+    token order; only which tokens share a tile does.  Returns (O, idx) with
+    idx the selection on the reordered tiles."""
+    order = np.asarray(order, dtype=np.int64)
+    Qp, Kp, Vp = _f64(Q)[:, order], _f64(K)[:, order], _f64(V)[:, order]
+    idx = select_tiles(tile_scores(landmark_means(Qp, tile), landmark_means(Kp, tile)), k)
+    Op = sparse_attention(Qp, Kp, Vp, tile, idx, scale, use_landmarks=use_landmarks)
+    return Op[:, inverse_order(order)], idx

@@ -17,6 +17,7 @@ views32     16     32 views     128   69     3-5, uniform
 linear256   16     256 views    128   --     none (linear stage)
 stack512    16     512 views    128   1100   3-5, uniform (per layer)
 views1024   16     1,024 views  128   660    3-5, within +-2 views
+spatial32   16     32 views     128   69     none; 2-D positional locality
 ==========  =====  ===========  ====  =====  ==========================
 
 Planting recipe (one reading of "each query tile shares a unit direction with
@@ -59,6 +60,8 @@ class Workload:
     calib_tiles: Optional[int] = 32     # calibration query tiles for the affine fit
     layers: int = 1
     linear_layers: Tuple[int, ...] = ()
+    pos_scale: float = 0.0              # 2-D positional component of patch-token queries and keys
+    pos_length: float = 3.0             # its length scale, in patches
 
     @property
     def n_tiles(self) -> int:
@@ -94,7 +97,11 @@ WORKLOADS = {
     "views1024": Workload("views1024", 5, heads=16, n_tokens=1024 * TOKENS_PER_VIEW,
                           keep_frac=0.06, v_std=1.0, plant_lo=3, plant_hi=5,
                           plant_window=22),
+    "spatial32": Workload("spatial32", 6, heads=16, n_tokens=32 * TOKENS_PER_VIEW,
+                          keep_frac=0.20, v_std=1.0, pos_scale=8.0, pos_length=3.0),
 }
+GRID = 37        # patches per side of a view
+SPECIALS = 5     # camera/register tokens at the start of each view
 
 
 def default_seed(w: Workload, layer: int = 0) -> int:
@@ -181,6 +188,27 @@ def make_qkv(w: Workload, layer: int = 0, device="cpu", seed: Optional[int] = No
         K.add_(kadd_t.view(H, T, d)[:, row_tile, :])
         del u_host, kadd, kadd_t
         del U, row_tile
+    if w.pos_scale > 0:
+        # 2-D locality: patch (y, x) of every view gets pos_scale * E(y, x) added to
+        # its query and key, E_c = sqrt(2/d) cos(w_c . (y, x) + phi_c) with per-head
+        # random w_c ~ N(0, I / pos_length^2), phi_c ~ U(0, 2 pi): random Fourier
+        # features, so E(p) . E(p') approximates exp(-|p - p'|^2 / (2 pos_length^2))
+        # and nearby patches (in any view) attend to each other
+        per_view = SPECIALS + GRID * GRID
+        if N % per_view:
+            raise ValueError("positional planting needs whole views")
+        om = torch.randn(H, d, 2, generator=g, device=dev, dtype=torch.float32) / w.pos_length
+        phi = torch.rand(H, d, generator=g, device=dev, dtype=torch.float32) * (2 * math.pi)
+        yy, xx = torch.meshgrid(torch.arange(GRID, device=dev, dtype=torch.float32),
+                                torch.arange(GRID, device=dev, dtype=torch.float32), indexing="ij")
+        pos = torch.stack([yy.reshape(-1), xx.reshape(-1)], dim=-1)                   # [P, 2]
+        E = math.sqrt(2.0 / d) * torch.cos(torch.einsum("pk,hck->hpc", pos, om) + phi[:, None, :])
+        add = torch.zeros(H, per_view, d, device=dev, dtype=torch.float32)
+        add[:, SPECIALS:] = w.pos_scale * E
+        add = add.repeat(1, N // per_view, 1)
+        Q.add_(add)
+        K.add_(add)
+        del add, E
     return (Q.to(torch.bfloat16), K.to(torch.bfloat16), V.to(torch.bfloat16))
 
 

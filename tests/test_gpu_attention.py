@@ -54,6 +54,35 @@ def test_sparse_attention_matches_oracle(name, over, k):
     assert err <= REL_TOL, err
 
 
+def test_sparse_attention_rescales_o_when_the_row_max_grows():
+    """Keys scaled up tile by tile (tile j by 1 + 0.75 j) and queries by 4: each
+    row's running max grows by more than the lazy-rescale threshold (8 in log2
+    units) partway through its item, at different steps for different rows of
+    one warp, so the O rescale runs inside items and with rows that disagree."""
+    w = workload("views32", heads=2, n_tokens=3000)          # T = 24, ragged 56-row last tile
+    Q, K, V = synth.make_qkv(w, device="cuda")
+    grow = 1.0 + 0.75 * (torch.arange(w.n_tokens, device="cuda") // w.tile).float()
+    Q = (Q.float() * 4).to(torch.bfloat16)
+    K = (K.float() * 4 * grow[None, :, None]).to(torch.bfloat16)
+    k = 12
+    O, idx = _sparse_gpu(w, Q, K, V, k)
+    Q64, K64, V64 = host(Q), host(K), host(V)
+    ref_idx = _oracle_idx(w, Q64, K64, k)
+    assert np.array_equal(idx.cpu().numpy(), ref_idx)
+    # the planted rescale really happens: row maxima of the first and last
+    # selected tiles differ by more than 8 in log2 units for many rows
+    s = 1 / math.sqrt(64)
+    lg = np.log2(np.e) * s
+    first = np.array([[(Q64[h, i * 128:(i + 1) * 128] @ K64[h, j0 * 128:(j0 + 1) * 128].T).max(1)
+                       for i, j0 in enumerate(ref_idx[h, :, 0][:23])] for h in range(2)])
+    last = np.array([[(Q64[h, i * 128:(i + 1) * 128] @ K64[h, j1 * 128:min(j1 * 128 + 128, w.n_tokens)].T).max(1)
+                      for i, j1 in enumerate(ref_idx[h, :, -1][:23])] for h in range(2)])
+    assert ((last - first) * lg > 8).mean() > 0.2
+    ref = oracle.sparse_attention(Q64, K64, V64, w.tile, ref_idx, s)
+    err = rel_err_per_head(host(O), ref)
+    assert err <= REL_TOL, err
+
+
 def test_sparse_lse_matches_oracle_logsumexp():
     w = workload("tiny")
     Q, K, V = synth.make_qkv(w, device="cuda")

@@ -462,3 +462,58 @@ def test_calibration_rows():
     assert rows.tolist() == list(range(192, 200)) + list(range(0, 64))
     assert synth.calibration_tiles(2748, 32)[:3].tolist() == [0, 85, 171]
     assert synth.calibration_tiles(4, None).tolist() == [0, 1, 2, 3]
+
+
+# ------------------------------------------------------- spatial tiles ----
+
+def test_spatial_order_hand_worked_small_grid():
+    # 5 x 5 patches after 1 special token, windows of 2 x 3 patches, worked by
+    # hand from the definition: window rows {0,1}, {2,3}, {4}; window columns
+    # {0,1,2}, {3,4}; patch (y, x) is token 1 + 5 y + x
+    want = [0, 1, 2, 3, 6, 7, 8, 4, 5, 9, 10, 11, 12, 13, 16, 17, 18, 14, 15, 19, 20,
+            21, 22, 23, 24, 25]
+    got = oracle.spatial_order(2, grid=5, specials=1, win_rows=2, win_cols=3)
+    assert got[:26].tolist() == want
+    assert got[26:].tolist() == [26 + t for t in want]
+
+
+def test_spatial_order_is_a_permutation_with_compact_windows():
+    views, grid, sp = 3, 37, 5
+    order = oracle.spatial_order(views)
+    N = views * (sp + grid * grid)
+    assert sorted(order.tolist()) == list(range(N))
+    X = RNG.standard_normal((2, N, 3))
+    np.testing.assert_array_equal(X[:, order][:, oracle.inverse_order(order)], X)
+    per_view = sp + grid * grid
+    for v in range(views):
+        seg = order[v * per_view:(v + 1) * per_view] - v * per_view
+        assert seg[:sp].tolist() == list(range(sp))          # specials first, inside their view
+        y, x = np.divmod(seg[sp:] - sp, grid)
+        # each of the 4 full-height window rows holds 8 x 16 + 8 x 16 + 8 x 5 = 296
+        # patches; its first two windows are full (128 patches each, a contiguous run
+        # covering an 8 x 16 rectangle), the third is the ragged right edge
+        for wy in range(4):
+            for wx, width in ((0, 128), (128, 128), (256, 40)):
+                a = 296 * wy + wx
+                yy, xx = y[a:a + width], x[a:a + width]
+                assert yy.min() == 8 * wy and yy.max() == 8 * wy + 7
+                assert xx.max() - xx.min() == (15 if width == 128 else 4)
+        assert len(seg) == per_view
+
+
+def test_spatial_sparse_attention_keep_all_is_dense_and_identity_order_is_plain():
+    H, views, grid, sp, t = 2, 2, 7, 1, 16
+    N = views * (sp + grid * grid)
+    Q, K, V = _qkv(H, N, 8)
+    order = oracle.spatial_order(views, grid=grid, specials=sp, win_rows=4, win_cols=4)
+    T = len(oracle.tile_lengths(N, t))
+    O, idx = oracle.spatial_sparse_attention(Q, K, V, t, order, 0.3, k=T)
+    np.testing.assert_allclose(O, oracle.dense_attention(Q, K, V, 0.3), rtol=1e-12, atol=1e-14)
+    ident = np.arange(N)
+    O1, idx1 = oracle.spatial_sparse_attention(Q, K, V, t, ident, 0.3, k=2)
+    want_idx = oracle.select_tiles(oracle.tile_scores(oracle.landmark_means(Q, t), oracle.landmark_means(K, t)), 2)
+    np.testing.assert_array_equal(idx1, want_idx)
+    np.testing.assert_array_equal(O1, oracle.sparse_attention(Q, K, V, t, want_idx, 0.3))
+    # with a real reordering and k < T the result differs from the plain tiling
+    O2, _ = oracle.spatial_sparse_attention(Q, K, V, t, order, 0.3, k=2)
+    assert np.abs(O2 - O1).max() > 1e-6
