@@ -1,10 +1,17 @@
-"""Host-side logic for running the layer as independent replicas on several GPUs.
+"""Host-side logic for running the layer on several GPUs, one process per GPU.
 
 The hybrid layer has no exchange step on one sample: every head and every
-query tile is independent.  Data parallelism therefore gives each rank its own
-problem (its own synthetic batch element, seeded per rank) with no collective
-on the data path; the only collectives are the timing barrier and the
-max-over-ranks of the measured time.
+query tile is independent.  Two ways to use G GPUs follow from that:
+
+  * replicas (what the bench runs under torchrun): each rank processes its own
+    problem (its own synthetic batch element, seeded per rank) with no
+    collective on the data path; the only collectives are the timing barrier
+    and the max-over-ranks of the measured time (weak scaling);
+  * a head partition of ONE sample: rank r runs the heads head_range(H, r, G)
+    of every call (landmarks, selection, attention, linear state and fit are
+    all per head), and the outputs are gathered only if the caller needs them
+    in one place (gather_heads: one all-gather of H * N * d values; strong
+    scaling of one layer).
 """
 from __future__ import annotations
 
@@ -57,3 +64,32 @@ def job_throughput(tokens_per_rank_step: float, steps: int, seconds_per_rank: fl
     t_max = max_over_ranks(seconds_per_rank, device)
     total = sum_over_ranks(tokens_per_rank_step * steps, device)
     return total / t_max, t_max
+
+
+def head_range(heads: int, rank: int, world: int) -> Tuple[int, int]:
+    """Contiguous, balanced block of heads [h0, h1) owned by `rank` (the first
+    heads % world ranks hold one more head)."""
+    if not 0 <= rank < world:
+        raise ValueError("rank out of range")
+    base, extra = divmod(heads, world)
+    h0 = rank * base + min(rank, extra)
+    return h0, h0 + base + (1 if rank < extra else 0)
+
+
+def gather_heads(local: torch.Tensor, heads: int) -> torch.Tensor:
+    """All-gather the per-rank head blocks [h1 - h0, ...] of a head partition into
+    the full [heads, ...] tensor on every rank.  Blocks are padded to the largest
+    block so that one equal-size all-gather serves uneven partitions."""
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return local
+    world, rank = dist.get_world_size(), dist.get_rank()
+    h0, h1 = head_range(heads, rank, world)
+    if local.shape[0] != h1 - h0:
+        raise ValueError(f"rank {rank} holds {local.shape[0]} heads, its block is {h1 - h0}")
+    width = -(-heads // world)
+    pad = local.new_zeros((width,) + tuple(local.shape[1:]))
+    pad[: h1 - h0] = local
+    parts = [torch.empty_like(pad) for _ in range(world)]
+    dist.all_gather(parts, pad)
+    return torch.cat([parts[r][: head_range(heads, r, world)[1] - head_range(heads, r, world)[0]]
+                      for r in range(world)], dim=0)

@@ -56,3 +56,48 @@ def test_single_process_identity():
     assert replicas.max_over_ranks(3.5) == 3.5
     tput, tmax = replicas.job_throughput(10.0, 4, 2.0)
     assert tmax == 2.0 and tput == 20.0
+
+
+def _head_worker(rank, world, port, heads, q):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK=str(rank),
+                      WORLD_SIZE=str(world), LOCAL_RANK=str(rank))
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    from linear_hybrid_attention_b200 import replicas
+    g = torch.Generator().manual_seed(9)
+    full_in = torch.randn(heads, 40, 8, generator=g)      # the same sample on every rank
+    h0, h1 = replicas.head_range(heads, rank, world)
+    local = full_in[h0:h1] * 2.0 + torch.arange(h0, h1, dtype=torch.float32)[:, None, None]
+    out = replicas.gather_heads(local, heads)
+    q.put((rank, h0, h1, out))
+    dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("heads", [16, 5])
+def test_head_partition_gathers_the_per_head_results_in_order(heads):
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_head_worker, args=(r, 2, port, heads, q)) for r in range(2)]
+    for p in procs:
+        p.start()
+    res = sorted((q.get(timeout=120) for _ in range(2)), key=lambda t: t[0])
+    for p in procs:
+        p.join(120)
+        assert p.exitcode == 0
+    g = torch.Generator().manual_seed(9)
+    full_in = torch.randn(heads, 40, 8, generator=g)
+    want = full_in * 2.0 + torch.arange(heads, dtype=torch.float32)[:, None, None]
+    (r0, a0, b0, o0), (r1, a1, b1, o1) = res
+    assert (a0, b1) == (0, heads) and b0 == a1                 # the blocks tile the heads
+    assert torch.equal(o0, want) and torch.equal(o1, want)
+
+
+def test_head_range_balanced():
+    from linear_hybrid_attention_b200 import replicas
+    for H in (1, 5, 16, 17):
+        for G in (1, 2, 3, 8):
+            blocks = [replicas.head_range(H, r, G) for r in range(G)]
+            assert blocks[0][0] == 0 and blocks[-1][1] == H
+            assert all(blocks[r][1] == blocks[r + 1][0] for r in range(G - 1))
+            sizes = [b - a for a, b in blocks]
+            assert max(sizes) - min(sizes) <= 1
