@@ -10,9 +10,9 @@
 //  * score_gemm_kernel: register-tiled fp64 GEMM, 128 x 128 scores per CTA,
 //    8 x 8 per thread, full d = 64 staged (transposed) in shared memory; each
 //    score is one FMA chain over d in index order.  Scores go to the workspace.
-//  * select_kernel: one CTA per (head, query tile); the T scores are copied to
-//    shared memory, the k-th largest is found by an 8-bit-digit radix select on
-//    order-preserving 64-bit keys (warp-aggregated histogram atomics, early
+//  * select_kernel: one CTA per (head, query tile); the T scores become
+//    order-preserving 64-bit keys in shared memory, the k-th largest is found
+//    by an 11-bit-digit radix select (2,048-bin shared-memory histogram, early
 //    exit once the bucket holds exactly the remaining count), and the kept
 //    indices are written in ascending order with two block-wide prefix sums.
 #include <cuda_runtime.h>
@@ -117,91 +117,110 @@ __device__ __forceinline__ int block_excl_scan(int v, int* scratch, int* total) 
     return wsum + x - v;
 }
 
+// Block-wide exclusive suffix sum (the sum over higher-numbered threads) of one
+// int per thread (STHREADS threads).
+__device__ __forceinline__ int block_excl_suffix(int v, int* scratch) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    int x = v;  // inclusive suffix sum within the warp
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_down_sync(0xffffffffu, x, o);
+        if (lane + o < 32) x += y;
+    }
+    if (lane == 0) scratch[warp] = x;
+    __syncthreads();
+    int above = 0;
+#pragma unroll
+    for (int w = 0; w < STHREADS / 32; ++w)
+        if (w > warp) above += scratch[w];
+    __syncthreads();
+    return above + x - v;
+}
+
 // ----------------------------------------------------------- select ----
-// grid: heads in group x T rows.  Scores of the row in shared memory when they
-// fit (`in_smem`), else read from the workspace on every pass.
+// grid: heads in group x T rows.  The row's scores become order keys in shared
+// memory when they fit (`in_smem`), else they are read from the workspace on
+// every pass.  Radix select of the k-th largest key from the top in 11-bit
+// digits (2,048 bins, one shared-memory atomic per counted key); after each
+// digit the bucket that holds the k-th key is found with a block-wide suffix
+// sum, and the search stops as soon as that bucket holds exactly the keys
+// still needed (usually after three digits).
+constexpr int DIGIT = 11;
+constexpr int NBINS = 1 << DIGIT;                 // 4 bins per thread
+static_assert(NBINS == 4 * STHREADS, "bins per thread");
+
 __global__ void __launch_bounds__(STHREADS)
 select_kernel(const double* __restrict__ scores, int T, int k, int h0, int in_smem,
               int32_t* __restrict__ idx) {
     extern __shared__ __align__(16) uint8_t smem_raw[];
-    __shared__ unsigned int hist[256];
+    __shared__ unsigned int hist[NBINS];
     __shared__ int scan_scratch[STHREADS / 32];
     __shared__ int sel_bucket, sel_above;
     const int tid = threadIdx.x;
     const int hl = blockIdx.x / T, i = blockIdx.x % T;
     const double* grow = scores + (static_cast<long long>(hl) * T + i) * T;
-    const double* row = grow;
+    unsigned long long* skey = reinterpret_cast<unsigned long long*>(smem_raw);
     if (in_smem) {
-        double* srow = reinterpret_cast<double*>(smem_raw);
-        for (int j = tid; j < T; j += STHREADS) srow[j] = grow[j];
-        row = srow;
+        for (int j = tid; j < T; j += STHREADS) skey[j] = order_key(grow[j]);
         __syncthreads();
     }
+    auto key_of = [&](int j) -> unsigned long long { return in_smem ? skey[j] : order_key(grow[j]); };
     int32_t* out = idx + (static_cast<long long>(h0 + hl) * T + i) * static_cast<long long>(k);
 
-    // ---- radix select of the k-th largest key, 8 bits per pass from the top
     unsigned long long prefix = 0, mask = 0;
     int need = k;
-    for (int shift = 56; shift >= 0; shift -= 8) {
-        for (int b = tid; b < 256; b += STHREADS) hist[b] = 0u;
+    for (int shift = 64 - DIGIT;; shift -= DIGIT) {
+        const int sh = shift < 0 ? 0 : shift;
+        const int width = shift < 0 ? shift + DIGIT : DIGIT;
+        const unsigned int dmask = (1u << width) - 1u;
+#pragma unroll
+        for (int e = 0; e < 4; ++e) hist[4 * tid + e] = 0u;
         __syncthreads();
-        for (int j0 = 0; j0 < T; j0 += STHREADS) {  // uniform trip count (warp collectives)
-            const int j = j0 + tid;
-            const unsigned long long key = j < T ? order_key(row[j]) : 0ull;
-            const bool m = j < T && (key & mask) == prefix;
-            const unsigned int digit = static_cast<unsigned int>((key >> shift) & 0xFFu);
-            const unsigned int active = __ballot_sync(0xffffffffu, m);
-            if (m) {
-                const unsigned int peers = __match_any_sync(active, digit);
-                if ((__ffs(peers) - 1) == (tid & 31)) atomicAdd(&hist[digit], __popc(peers));
-            }
+        for (int j = tid; j < T; j += STHREADS) {
+            const unsigned long long key = key_of(j);
+            if ((key & mask) == prefix) atomicAdd(&hist[static_cast<unsigned int>(key >> sh) & dmask], 1u);
         }
         __syncthreads();
-        if (tid < 32) {
-            unsigned int c[8], lsum = 0;
+        unsigned int c[4];
+        int local = 0;
 #pragma unroll
-            for (int e = 0; e < 8; ++e) lsum += (c[e] = hist[tid * 8 + e]);
-            unsigned int x = lsum;  // inclusive suffix sum over lanes
+        for (int e = 0; e < 4; ++e) local += static_cast<int>(c[e] = hist[4 * tid + e]);
+        const int above = block_excl_suffix(local, scan_scratch);
+        if (above < need && above + local >= need) {
+            int run = above;
 #pragma unroll
-            for (int o = 1; o < 32; o <<= 1) {
-                const unsigned int y = __shfl_down_sync(0xffffffffu, x, o);
-                if (tid + o < 32) x += y;
-            }
-            const unsigned int suffix = x - lsum;
-            if (suffix < static_cast<unsigned int>(need) && x >= static_cast<unsigned int>(need)) {
-                unsigned int run = suffix;
-                for (int e = 7; e >= 0; --e) {
-                    if (run + c[e] >= static_cast<unsigned int>(need)) {
-                        sel_bucket = tid * 8 + e;
-                        sel_above = static_cast<int>(run);
-                        break;
-                    }
-                    run += c[e];
+            for (int e = 3; e >= 0; --e) {
+                if (run + static_cast<int>(c[e]) >= need) {
+                    sel_bucket = 4 * tid + e;
+                    sel_above = run;
+                    break;
                 }
+                run += static_cast<int>(c[e]);
             }
         }
         __syncthreads();
         const int bsel = sel_bucket;
         need -= sel_above;
-        prefix |= static_cast<unsigned long long>(bsel) << shift;
-        mask |= 0xFFull << shift;
+        prefix |= static_cast<unsigned long long>(bsel) << sh;
+        mask |= static_cast<unsigned long long>(dmask) << sh;
         const bool done = static_cast<int>(hist[bsel]) == need;
         __syncthreads();
-        if (done) break;
+        if (done || sh == 0) break;
     }
 
-    // ---- ascending output: each thread owns a contiguous range of j
+    // ---- ascending output: each thread owns a contiguous range of j; keys
+    // above the bucket are kept, keys in it are kept lowest index first
     const int per = (T + STHREADS - 1) / STHREADS;
     const int jb = tid * per, je = min(T, jb + per);
     int n_eq = 0;
-    for (int j = jb; j < je; ++j) n_eq += ((order_key(row[j]) & mask) == prefix) ? 1 : 0;
+    for (int j = jb; j < je; ++j) n_eq += ((key_of(j) & mask) == prefix) ? 1 : 0;
     int tot;
     const int eq_rank = block_excl_scan(n_eq, scan_scratch, &tot);
     int n_sel = 0;
     {
         int r = eq_rank;
         for (int j = jb; j < je; ++j) {
-            const unsigned long long km = order_key(row[j]) & mask;
+            const unsigned long long km = key_of(j) & mask;
             if (km > prefix) ++n_sel;
             else if (km == prefix) n_sel += (r++ < need) ? 1 : 0;
         }
@@ -210,7 +229,7 @@ select_kernel(const double* __restrict__ scores, int T, int k, int h0, int in_sm
     {
         int r = eq_rank;
         for (int j = jb; j < je; ++j) {
-            const unsigned long long km = order_key(row[j]) & mask;
+            const unsigned long long km = key_of(j) & mask;
             bool sel = km > prefix;
             if (km == prefix) sel = (r++ < need);
             if (sel) out[pos++] = j;
