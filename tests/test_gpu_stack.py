@@ -21,6 +21,7 @@ import concurrent.futures as cf
 import math
 import multiprocessing as mp
 import os
+import time
 
 import numpy as np
 import pytest
@@ -72,7 +73,12 @@ def test_small_stack_matches_oracle_with_and_without_lookahead():
         assert err <= REL_TOL, (l, err)
 
 
+def _progress(t0, *what):
+    print(f"[stack test {time.time() - t0:7.1f} s]", *what, flush=True)
+
+
 def test_stack_512_views_all_24_layers_full_size_sampled():
+    t0 = time.time()
     w = workload("stack512")
     L, lin = w.layers, w.linear_layers
     T, t = w.n_tiles, w.tile
@@ -80,6 +86,7 @@ def test_stack_512_views_all_24_layers_full_size_sampled():
     torch.cuda.empty_cache()
     inputs = [synth.make_qkv(w, layer=l, device="cuda") for l in range(L)]
     stack, calib = _stack(w, L, lin)
+    _progress(t0, "inputs and buffers ready")
     # sampled (head, query tiles) per layer; the last tile is always among them
     plan = {}
     for l in range(L):
@@ -104,9 +111,11 @@ def test_stack_512_views_all_24_layers_full_size_sampled():
 
     stack.run(inputs, lookahead=True, on_layer_done=hook)
     sync_ok()
+    _progress(t0, "lookahead pass done")
     first = {l: (got[l]["O"].cpu(), None if got[l]["idx"] is None else got[l]["idx"].cpu()) for l in range(L)}
     stack.run(inputs, lookahead=False, on_layer_done=lambda l, O: sums[l].append(_checksum(O)))
     sync_ok()
+    _progress(t0, "serial pass done")
     for l in range(L):
         assert int(sums[l][0]) == int(sums[l][1]), f"layer {l}: lookahead changed the output"
         if l not in lin:
@@ -141,10 +150,12 @@ def test_stack_512_views_all_24_layers_full_size_sampled():
                     f.paths = paths
                     pending.add(f)
                     futures[(l, h)] = f
+                _progress(t0, f"layer {l}: oracle jobs submitted")
                 inputs[l] = None                       # this layer's inputs are no longer needed
             del inputs
             torch.cuda.empty_cache()
             results = {key: f.result() for key, f in futures.items()}
+            _progress(t0, "oracle jobs done")
     n = oracle.tile_lengths(w.n_tokens, t)
     for l in range(L):
         heads, tiles = plan[l]
