@@ -52,27 +52,21 @@ def measured_peaks():
 
 # ---------------------------------------------------------------- traffic ----
 def recorded_traffic(workload: str):
-    """DRAM bytes per launch of the sparse kernel from the committed ncu summary
-    (profiles/sparse_attn_<workload>_dram.md), or None when there is none or the
-    kernel source changed since it was taken (its sha256 is recorded there)."""
+    """DRAM bytes per launch of the sparse kernel at this workload, from the small
+    record profiles/sparse_attn_<workload>_traffic.json written beside the ncu
+    summary it comes from, or None when there is none or when the kernel source
+    changed since the capture (the record holds attn.cu's sha256)."""
     import hashlib
-    path = os.path.join(ROOT, "profiles", f"sparse_attn_{workload}_dram.md")
+    path = os.path.join(ROOT, "profiles", f"sparse_attn_{workload}_traffic.json")
     src = os.path.join(ROOT, "linear_hybrid_attention_b200", "csrc", "attn.cu")
     if not os.path.exists(path) or not os.path.exists(src):
         return None, "no ncu DRAM capture recorded for this workload"
-    fields = {}
     with open(path) as f:
-        for line in f:
-            if ":" in line and line.startswith("- "):
-                k, v = line[2:].split(":", 1)
-                fields[k.strip()] = v.strip().strip("`")
+        rec = json.load(f)
     sha = hashlib.sha256(open(src, "rb").read()).hexdigest()
-    if fields.get("attn.cu sha256") != sha:
+    if rec.get("attn_cu_sha256") != sha:
         return None, "kernel changed since the recorded ncu DRAM capture"
-    try:
-        return float(fields["dram bytes per launch"]), os.path.relpath(path, ROOT)
-    except (KeyError, ValueError):
-        return None, "ncu DRAM summary unreadable"
+    return float(rec["dram_bytes_per_launch"]), rec.get("summary", os.path.relpath(path, ROOT))
 
 
 # ----------------------------------------------------------------- clocks ----

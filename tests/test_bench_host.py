@@ -23,14 +23,15 @@ def test_selected_flops_counts_every_kept_pair():
     assert bench.selected_flops(idx, 300, 128, 64) == want
 
 
-def _fake_root(tmp_path, attn_src, recorded_sha, nbytes="123456"):
+def _fake_root(tmp_path, attn_src, recorded_sha, nbytes=123456.0):
     csrc = tmp_path / "linear_hybrid_attention_b200" / "csrc"
     csrc.mkdir(parents=True)
     (csrc / "attn.cu").write_bytes(attn_src)
     prof = tmp_path / "profiles"
     prof.mkdir()
-    (prof / "sparse_attn_w_dram.md").write_text(
-        f"# capture\n\n- dram bytes per launch: {nbytes}\n- attn.cu sha256: {recorded_sha}\n")
+    (prof / "sparse_attn_w_traffic.json").write_text(json.dumps(
+        {"dram_bytes_per_launch": nbytes, "attn_cu_sha256": recorded_sha,
+         "summary": "profiles/sparse_attn_w.md"}))
     return str(tmp_path)
 
 
@@ -39,7 +40,7 @@ def test_recorded_traffic_only_for_the_measured_kernel(tmp_path, monkeypatch):
     sha = hashlib.sha256(src).hexdigest()
     monkeypatch.setattr(bench, "ROOT", _fake_root(tmp_path / "a", src, sha))
     value, where = bench.recorded_traffic("w")
-    assert value == 123456.0 and where == os.path.join("profiles", "sparse_attn_w_dram.md")
+    assert value == 123456.0 and where == "profiles/sparse_attn_w.md"
     # the kernel changed after the capture: no traffic figure
     monkeypatch.setattr(bench, "ROOT", _fake_root(tmp_path / "b", src + b" ", sha))
     value, why = bench.recorded_traffic("w")
