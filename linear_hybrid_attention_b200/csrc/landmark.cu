@@ -44,21 +44,23 @@ __device__ __forceinline__ uint16_t f64_to_bf16_rne(double x) {
 //                       copies, once the 16 compute warps have read the stage;
 //   warps 0..15         warp w sums rows [8 w, 8 w + 8) of each tensor, lane l
 //                       columns 2l, 2l+1, in fp64 (exact for bf16 inputs unless
-//                       a tile spans > ~38 binades), into a double-buffered
-//                       partial table; warps 0..5 (192 threads, one output
-//                       each) then add the 16 partials of the item in a fixed
-//                       order and write the means, while the other warps
-//                       already sum the next item.
+//                       a tile spans > ~38 binades), into one of three
+//                       partial tables; warps 0..5 (192 threads, one output
+//                       each) then add the 16 partials of the item as a fixed
+//                       4-level tree and write the means, while the other
+//                       warps already sum the next items.
 // 16 compute warps per SM hide the latency of the fp32 -> fp64 conversions.
 constexpr int LM_STAGES = 3;
+constexpr int NPB = 3;        // partial tables: the compute warps run up to two items ahead of the reduction
 constexpr int LM_WARPS = 16;  // compute warps
+static_assert(LM_WARPS == 16, "the partial reduction is a tree over 16 warps");
 constexpr uint32_t RUN_BYTES = 128 * HD * 2;  // one full tile of one tensor
 
 struct LmSmem {
     uint8_t buf[LM_STAGES][3][RUN_BYTES];
-    double part[2][LM_WARPS][3][HD];
+    double part[NPB][LM_WARPS][3][HD];
     uint64_t full[LM_STAGES], empty[LM_STAGES];
-    uint64_t pfull[2], pempty[2];
+    uint64_t pfull[NPB], pempty[NPB];
     int abort_flag;
 };
 
@@ -83,7 +85,7 @@ landmark_kernel(const uint16_t* __restrict__ Q, const uint16_t* __restrict__ K,
             mbar_init(smem_addr(&sm.full[s]), 1);
             mbar_init(smem_addr(&sm.empty[s]), LM_WARPS);
         }
-        for (int b = 0; b < 2; ++b) {
+        for (int b = 0; b < NPB; ++b) {
             mbar_init(smem_addr(&sm.pfull[b]), LM_WARPS);
             mbar_init(smem_addr(&sm.pempty[b]), 3 * HD);
         }
@@ -128,8 +130,8 @@ landmark_kernel(const uint16_t* __restrict__ Q, const uint16_t* __restrict__ K,
     } else {
         // ============================================ compute warps ====
         for (int it = 0; it < cnt; ++it) {
-            const int s = it % LM_STAGES, pb = it & 1;
-            const uint32_t use = static_cast<uint32_t>(it / LM_STAGES), pu = static_cast<uint32_t>(it >> 1);
+            const int s = it % LM_STAGES, pb = it % NPB;
+            const uint32_t use = static_cast<uint32_t>(it / LM_STAGES), pu = static_cast<uint32_t>(it / NPB);
             int h, j, n;
             item_of(it, h, j, n);
             if (!mbar_wait_warp(smem_addr(&sm.full[s]), use & 1, wc)) break;
@@ -169,7 +171,7 @@ landmark_kernel(const uint16_t* __restrict__ Q, const uint16_t* __restrict__ K,
             fence_proxy_async_smem();  // our reads precede the next bulk write into it
             __syncwarp();
             if (lane == 0) mbar_arrive(smem_addr(&sm.empty[s]));
-            // partial table pb is free once the item two back was reduced
+            // partial table pb is free once the item NPB back was reduced
             if (!mbar_wait_warp(smem_addr(&sm.pempty[pb]), (pu & 1) ^ 1, wc)) break;
 #pragma unroll
             for (int t = 0; t < 3; ++t) {
@@ -179,15 +181,21 @@ landmark_kernel(const uint16_t* __restrict__ Q, const uint16_t* __restrict__ K,
             __syncwarp();
             if (lane == 0) mbar_arrive(smem_addr(&sm.pfull[pb]));
             if (tid < 3 * HD) {
-                // fixed-order reduction of the 16 partials, one output per thread
+                // fixed-order reduction of the 16 partials (a 4-level tree: the
+                // partials and their sums are exact, so any fixed order gives the
+                // same value), one output per thread
                 if (!mbar_wait_warp(smem_addr(&sm.pfull[pb]), pu & 1, wc)) break;
                 const int t = tid / HD, col = tid % HD;
-                double sum = 0.0;
+                double v8[LM_WARPS / 2];
 #pragma unroll
-                for (int wp = 0; wp < LM_WARPS; ++wp) sum += sm.part[pb][wp][t][col];
+                for (int wp = 0; wp < LM_WARPS / 2; ++wp)
+                    v8[wp] = sm.part[pb][2 * wp][t][col] + sm.part[pb][2 * wp + 1][t][col];
+                const double sum = ((v8[0] + v8[1]) + (v8[2] + v8[3])) + ((v8[4] + v8[5]) + (v8[6] + v8[7]));
                 mbar_arrive(smem_addr(&sm.pempty[pb]));
                 if (t >= t0) {
-                    const double mean = sum / static_cast<double>(n);
+                    // n = 128 or 64 is a power of two: the product by 1 / n is the exact quotient
+                    const double mean = n == 128 ? sum * 0.0078125
+                                                 : (n == 64 ? sum * 0.015625 : sum / static_cast<double>(n));
                     const long long o = (static_cast<long long>(h) * T + j) * HD + col;
                     if (t == 0) {
                         Qbar[o] = mean;

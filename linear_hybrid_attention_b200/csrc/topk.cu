@@ -12,7 +12,7 @@
 //    score is one FMA chain over d in index order.  Scores go to the workspace.
 //  * select_kernel: one CTA per (head, query tile); the T scores become
 //    order-preserving 64-bit keys in shared memory, the k-th largest is found
-//    by an 11-bit-digit radix select (2,048-bin shared-memory histogram, early
+//    by a 12-bit-digit radix select (4,096-bin shared-memory histogram, early
 //    exit once the bucket holds exactly the remaining count), and the kept
 //    indices are written in ascending order with two block-wide prefix sums.
 #include <cuda_runtime.h>
@@ -140,14 +140,15 @@ __device__ __forceinline__ int block_excl_suffix(int v, int* scratch) {
 // ----------------------------------------------------------- select ----
 // grid: heads in group x T rows.  The row's scores become order keys in shared
 // memory when they fit (`in_smem`), else they are read from the workspace on
-// every pass.  Radix select of the k-th largest key from the top in 11-bit
-// digits (2,048 bins, one shared-memory atomic per counted key); after each
+// every pass.  Radix select of the k-th largest key from the top in 12-bit
+// digits (4,096 bins, one shared-memory atomic per counted key); after each
 // digit the bucket that holds the k-th key is found with a block-wide suffix
 // sum, and the search stops as soon as that bucket holds exactly the keys
-// still needed (usually after three digits).
-constexpr int DIGIT = 11;
-constexpr int NBINS = 1 << DIGIT;                 // 4 bins per thread
-static_assert(NBINS == 4 * STHREADS, "bins per thread");
+// still needed (usually after two digits: 24 bits of the key).
+constexpr int DIGIT = 12;
+constexpr int NBINS = 1 << DIGIT;
+constexpr int BPT = NBINS / STHREADS;             // bins per thread
+static_assert(BPT * STHREADS == NBINS, "bins per thread");
 
 __global__ void __launch_bounds__(STHREADS)
 select_kernel(const double* __restrict__ scores, int T, int k, int h0, int in_smem,
@@ -174,24 +175,24 @@ select_kernel(const double* __restrict__ scores, int T, int k, int h0, int in_sm
         const int width = shift < 0 ? shift + DIGIT : DIGIT;
         const unsigned int dmask = (1u << width) - 1u;
 #pragma unroll
-        for (int e = 0; e < 4; ++e) hist[4 * tid + e] = 0u;
+        for (int e = 0; e < BPT; ++e) hist[BPT * tid + e] = 0u;
         __syncthreads();
         for (int j = tid; j < T; j += STHREADS) {
             const unsigned long long key = key_of(j);
             if ((key & mask) == prefix) atomicAdd(&hist[static_cast<unsigned int>(key >> sh) & dmask], 1u);
         }
         __syncthreads();
-        unsigned int c[4];
+        unsigned int c[BPT];
         int local = 0;
 #pragma unroll
-        for (int e = 0; e < 4; ++e) local += static_cast<int>(c[e] = hist[4 * tid + e]);
+        for (int e = 0; e < BPT; ++e) local += static_cast<int>(c[e] = hist[BPT * tid + e]);
         const int above = block_excl_suffix(local, scan_scratch);
         if (above < need && above + local >= need) {
             int run = above;
 #pragma unroll
-            for (int e = 3; e >= 0; --e) {
+            for (int e = BPT - 1; e >= 0; --e) {
                 if (run + static_cast<int>(c[e]) >= need) {
-                    sel_bucket = 4 * tid + e;
+                    sel_bucket = BPT * tid + e;
                     sel_above = run;
                     break;
                 }
