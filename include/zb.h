@@ -94,14 +94,27 @@ zb_status zb_landmark_build(const uint16_t* Q, const uint16_t* K, const uint16_t
  * "selected tiles" (Figure 1 (a) caption) without the criterion; this is the
  * mean-pooled reading.  The budget k is the kept share of the key tiles (the
  * y in "xL/yS" of the Table 20 caption is the dropped share).
+ * The selection is that of the fp64 scores, but most scores are never formed
+ * in fp64: each row of Qbar and Kbar becomes three signed 8-bit digit planes of
+ * a 21-bit fixed-point copy, int8 tensor-core products give every score to
+ * within a proven bound, and only the key tiles whose approximate score lies
+ * within that bound of the k-th largest are re-scored in fp64 (one FMA chain
+ * over d in index order) to decide the boundary.
  *   in : Qbar, Kbar fp64 [H][T][d];  0 <= k <= T
- *   ws : scratch for the fp64 score matrix of a group of heads; at least
- *        T*T*8 bytes (one head per pass), up to H*T*T*8 (all heads in one
- *        pass).  zb_tile_score_topk_workspace_bytes() gives a default (4
- *        heads).  Not needed (may be NULL) when k == 0 or k == T.
+ *   ws : scratch for one group of heads: digit planes, exponents and an fp32
+ *        score matrix (T x T rounded up to 128 columns) per head.  Its size
+ *        for one head is zb_tile_score_topk_workspace_bytes() of a one-head
+ *        shape; a larger ws takes that many heads per pass (up to all H).  The
+ *        default size (4 heads) is zb_tile_score_topk_workspace_bytes(s).
+ *        16-byte aligned, owned by the caller, not shared with a call running
+ *        at the same time.  Not needed (may be NULL) when k == 0 or k == T.
  *   out: idx int32 [H][T][k]
+ * Non-finite values in Qbar or Kbar do not stop the call: the rows they reach
+ * are ranked by the fp64 order keys of their scores alone (NaN keys above
+ * +inf or below -inf by sign).
  * Errors: ZB_ERR_NULL, ZB_ERR_SHAPE, ZB_ERR_ALIGN, ZB_ERR_UNSUPPORTED (T > 32768),
- * ZB_ERR_WORKSPACE, ZB_ERR_CUDA.
+ * ZB_ERR_WORKSPACE, ZB_ERR_CUDA; ZB_ERR_TIMEOUT in the device status if a
+ * bounded wait of the score GEMM gave up.
  */
 size_t zb_tile_score_topk_workspace_bytes(zb_shape s);
 zb_status zb_tile_score_topk(const double* Qbar, const double* Kbar, zb_shape s,

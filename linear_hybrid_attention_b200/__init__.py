@@ -35,26 +35,28 @@ __all__ = [
 HEAD_DIM = 64
 
 # kernels each entry point launches (for counting launches in a timed region);
-# zb_tile_score_topk launches 2 per pass over the heads its workspace holds
+# zb_tile_score_topk launches 4 per pass over the heads its workspace holds
 # (topk_launches gives the count of one call)
 LAUNCHES_PER_CALL = {
-    "zb_landmark_build": 1, "zb_tile_score_topk": 2, "zb_tile_sparse_attn": 1, "zb_dense_attn": 1,
+    "zb_landmark_build": 1, "zb_tile_score_topk": 4, "zb_tile_sparse_attn": 1, "zb_dense_attn": 1,
     "zb_linear_state": 2, "zb_linear_apply": 1, "zb_linear_attn": 3, "zb_affine_fit": 3, "zb_gather_tiles": 1,
     "zb_key_mean": 2, "zb_linear_state_centered": 2, "zb_block_mass": 1, "zb_block_mass_top_fraction": 1,
     "zb_block_mass_selected_fraction": 1, "zb_gather_rows": 1, "zb_spatial_order": 0,
 }
 
 
-def topk_launches(heads: int, n_tiles_: int, k: int, ws_bytes: int) -> int:
+def topk_launches(heads: int, n_tokens: int, tile: int, k: int, ws_bytes: int) -> int:
     """Kernels one zb_tile_score_topk call launches: none for k = 0, one fill kernel for
-    k = T, else a score GEMM and a select kernel per pass over as many heads as the
-    workspace holds (T * T doubles per head)."""
+    k = T, else four per pass (digit planes, head summary, int8 score GEMM, select)
+    over as many heads as the workspace holds (one head's share is the default
+    workspace of a one-head shape)."""
+    T = -(-n_tokens // tile)
     if k == 0:
         return 0
-    if k == n_tiles_:
+    if k == T:
         return 1
-    per_pass = min(heads, ws_bytes // (n_tiles_ * n_tiles_ * 8))
-    return 2 * (-(-heads // per_pass))
+    per_pass = min(heads, ws_bytes // topk_workspace_bytes(1, n_tokens, tile))
+    return LAUNCHES_PER_CALL["zb_tile_score_topk"] * (-(-heads // per_pass))
 
 
 class ZbError(RuntimeError):
@@ -540,5 +542,5 @@ class HybridLayer:
         extra = LAUNCHES_PER_CALL["zb_key_mean"] if self.centered else 0
         if self.spatial is not None:
             extra += 4 * LAUNCHES_PER_CALL["zb_gather_rows"]
-        topk = topk_launches(self.heads, self.T, self.k, self.ws_topk.numel())
+        topk = topk_launches(self.heads, self.n_tokens, self.tile, self.k, self.ws_topk.numel())
         return self.LAUNCHES["sparse"] + topk + self.LAUNCHES["calibrate"] + extra + self.LAUNCHES["linear"]

@@ -57,8 +57,16 @@ def test_workspace_sizes(lib):
     lin = lib.zb_linear_attn_workspace_bytes(16, 1024 * 1374, 64)
     assert lin >= n + 16 * 64 * 65 * 4 and lin % 256 == 0
     assert lib.zb_linear_attn_workspace_bytes(16, 1000, 32) == 0
-    assert lib.zb_tile_score_topk_workspace_bytes(_shape(H=16, N=1024 * 1374, t=128)) == 4 * 10992 ** 2 * 8
-    assert lib.zb_tile_score_topk_workspace_bytes(_shape(H=2, N=256, t=64)) == 2 * 16 * 8
+    # selection, per head: digit planes (192 B a row) and exponents of Qbar and Kbar,
+    # the head summary and fp32 score rows padded to 128 columns, each 256-byte aligned
+    assert lib.zb_tile_score_topk_workspace_bytes(_shape(H=16, N=1024 * 1374, t=128)) == 4 * _topk_head(10992)
+    assert lib.zb_tile_score_topk_workspace_bytes(_shape(H=2, N=256, t=64)) == 2 * _topk_head(4)
+
+
+def _topk_head(T):
+    al = lambda x: -(-x // 256) * 256
+    Tp = -(-T // 128) * 128
+    return 2 * al(T * 192) + 2 * al(T * 4) + al(8) + al(T * Tp * 4)
 
 
 def _shape(H=2, N=256, d=64, t=64):
@@ -83,7 +91,7 @@ def test_validation_errors_before_launch(lib):
     assert lib.zb_tile_score_topk(FAKE, FAKE, S, -1, FAKE, FAKE, 1 << 20, None) == 2
     assert lib.zb_tile_score_topk(FAKE, FAKE, S, 2, None, FAKE, 1 << 20, None) == 1
     assert lib.zb_tile_score_topk(FAKE, FAKE, S, 2, FAKE, None, 1 << 20, None) == 5    # no workspace
-    assert lib.zb_tile_score_topk(FAKE, FAKE, S, 2, FAKE, FAKE, 4 * 4 * 8 - 8, None) == 5
+    assert lib.zb_tile_score_topk(FAKE, FAKE, S, 2, FAKE, FAKE, _topk_head(4) - 16, None) == 5
     assert lib.zb_tile_score_topk(FAKE, FAKE, S, 0, None, None, 0, None) == 0  # nothing to do
     # sparse attention
     a = (FAKE, FAKE, FAKE, FAKE, FAKE, FAKE)
@@ -165,13 +173,14 @@ def test_binding_refuses_cpu_tensors():
 
 
 def test_topk_launch_count_follows_the_launcher():
-    # zb_tile_score_topk: nothing for k = 0, one fill kernel for k = T, else a score
-    # GEMM and a select per pass over the heads that the workspace holds
+    # zb_tile_score_topk: nothing for k = 0, one fill kernel for k = T, else digit
+    # planes, head summary, score GEMM and select per pass over the heads the workspace holds
     from linear_hybrid_attention_b200 import topk_launches
-    T = 10992
-    assert topk_launches(16, T, 660, 4 * T * T * 8) == 8
-    assert topk_launches(16, T, 660, 16 * T * T * 8) == 2
-    assert topk_launches(16, T, 660, 5 * T * T * 8 - 1) == 8   # 4 heads per pass
-    assert topk_launches(3, T, 660, 2 * T * T * 8) == 4        # passes of 2 and 1 heads
-    assert topk_launches(16, T, 0, 0) == 0
-    assert topk_launches(16, T, T, 0) == 1
+    N, t = 1024 * 1374, 128
+    T, one = 10992, _topk_head(10992)
+    assert topk_launches(16, N, t, 660, 4 * one) == 16
+    assert topk_launches(16, N, t, 660, 16 * one) == 4
+    assert topk_launches(16, N, t, 660, 5 * one - 1) == 16   # 4 heads per pass
+    assert topk_launches(3, N, t, 660, 2 * one) == 8         # passes of 2 and 1 heads
+    assert topk_launches(16, N, t, 0, 0) == 0
+    assert topk_launches(16, N, t, T, 0) == 1

@@ -109,3 +109,86 @@ def test_gather_tiles():
     assert (o[:, 104:128] == 0).all()
     assert torch.equal(o[:, 128:256], q[:, 0:128])
     assert torch.equal(o[:, 256:384], q[:, 384:512])
+
+
+# ---- the boundary of the selection: near ties, wide bands, exact ties, extreme rows
+def _select_gpu(Qb, Kb, tile, k):
+    import linear_hybrid_attention_b200 as zb
+    H, T, _ = Qb.shape
+    idx = zb.zb_tile_score_topk(torch.from_numpy(Qb).cuda(), torch.from_numpy(Kb).cuda(), T * tile, tile, k)
+    sync_ok()
+    return idx.cpu().numpy().astype(np.int64)
+
+
+def _cluster_case(T, n_cluster, spread, seed):
+    # every query row has a positive first component; the cluster's key rows are one
+    # large vector plus perturbations of relative size `spread`, so their scores lead
+    # every row and only the perturbations order them
+    g = np.random.default_rng(seed)
+    H = 2
+    Qb = g.standard_normal((H, T, 64))
+    Qb[..., 0] = 1.0 + 0.1 * np.abs(Qb[..., 0])
+    Kb = g.standard_normal((H, T, 64))
+    cl = g.choice(T, n_cluster, replace=False)
+    base = np.zeros(64)
+    base[0] = 30.0
+    Kb[:, cl] = base + 30.0 * spread * g.standard_normal((H, n_cluster, 64))
+    return Qb, Kb
+
+
+def test_selection_near_ties_are_decided_in_fp64():
+    # 60 near-equal key tiles (gaps ~1e-10 relative, far inside the int8 bound, far
+    # outside fp64 rounding) with k = 40: the whole decision falls in the band
+    Qb, Kb = _cluster_case(T=300, n_cluster=60, spread=1e-8, seed=5)
+    got = _select_gpu(Qb, Kb, 64, 40)
+    assert np.array_equal(got, oracle.select_tiles(oracle.tile_scores(Qb, Kb), 40))
+
+
+def test_selection_wide_band_radix_path():
+    # 700 near-equal key tiles (more than the 512 a band ranks directly), k = 600
+    Qb, Kb = _cluster_case(T=1000, n_cluster=700, spread=1e-8, seed=6)
+    got = _select_gpu(Qb, Kb, 64, 600)
+    assert np.array_equal(got, oracle.select_tiles(oracle.tile_scores(Qb, Kb), 600))
+
+
+def test_selection_exact_ties_beyond_the_band_cap():
+    # all scores 0 in 2,000 key tiles: ties go to the lowest indices
+    g = np.random.default_rng(7)
+    Qb = np.zeros((1, 2000, 64))
+    Kb = g.standard_normal((1, 2000, 64))
+    got = _select_gpu(Qb, Kb, 64, 5)
+    assert (got == np.arange(5)).all()
+
+
+def test_selection_rows_with_a_large_dynamic_range():
+    # one component 1e6 times the others in every query and key row, plus rows of
+    # very different magnitudes: the fixed-point copies lose the small components,
+    # the band widens, the selection stays that of the fp64 scores
+    g = np.random.default_rng(8)
+    H, T, k = 2, 400, 37
+    Qb = g.standard_normal((H, T, 64))
+    Kb = g.standard_normal((H, T, 64))
+    Qb[..., 3] *= 1e6
+    Kb[..., 3] *= 1e6
+    Kb *= np.exp2(g.integers(-60, 20, size=(H, T, 1)))
+    Qb[:, ::7] *= 1e-200
+    got = _select_gpu(Qb, Kb, 64, k)
+    assert np.array_equal(got, oracle.select_tiles(oracle.tile_scores(Qb, Kb), k))
+
+
+def test_selection_non_finite_rows_give_valid_sets():
+    # a NaN in one query row and an inf in one key row of head 1: the call succeeds
+    # and every row is a strictly ascending set of k indices in range; head 0 (finite)
+    # matches the oracle
+    g = np.random.default_rng(9)
+    H, T, k = 2, 200, 11
+    Qb = g.standard_normal((H, T, 64))
+    Kb = g.standard_normal((H, T, 64))
+    Qb[0, 17, 5] = np.nan
+    Kb[1, 40, 2] = np.inf
+    got = _select_gpu(Qb, Kb, 64, k)
+    assert ((got >= 0) & (got < T)).all()
+    assert (np.diff(got, axis=-1) > 0).all()
+    ref = oracle.select_tiles(oracle.tile_scores(Qb[:1], Kb[:1]), k)
+    rows = np.arange(T) != 17
+    assert np.array_equal(got[0, rows], ref[0, rows])
