@@ -106,12 +106,14 @@ digits_kernel(const double* __restrict__ Qbar, const double* __restrict__ Kbar, 
 
 // One CTA per head: e_ref = the largest key-row exponent (0 if none), and
 // whether a key row holds a non-finite value.
-__global__ void __launch_bounds__(256) head_info_kernel(const int* __restrict__ ke, int T, int2* __restrict__ hinfo) {
-    __shared__ int smax[8], sbad[8];
+constexpr int HI_THREADS = 1024;
+__global__ void __launch_bounds__(HI_THREADS) head_info_kernel(const int* __restrict__ ke, int T, int2* __restrict__ hinfo) {
+    __shared__ int smax[HI_THREADS / 32], sbad[HI_THREADS / 32];
     const int hl = blockIdx.x;
+    const int* e_h = ke + static_cast<long long>(hl) * T;
     int emax = -(1 << 30), bad = 0;
-    for (int j = threadIdx.x; j < T; j += blockDim.x) {
-        const int e = ke[static_cast<long long>(hl) * T + j];
+    for (int j = threadIdx.x; j < T; j += HI_THREADS) {
+        const int e = e_h[j];
         if (e == EXP_NONFINITE) bad = 1;
         else if (e != EXP_ZERO) emax = max(emax, e);
     }
@@ -123,7 +125,7 @@ __global__ void __launch_bounds__(256) head_info_kernel(const int* __restrict__ 
     if ((threadIdx.x & 31) == 0) { smax[threadIdx.x >> 5] = emax; sbad[threadIdx.x >> 5] = bad; }
     __syncthreads();
     if (threadIdx.x == 0) {
-        for (int w = 1; w < 8; ++w) { emax = max(emax, smax[w]); bad |= sbad[w]; }
+        for (int w = 1; w < HI_THREADS / 32; ++w) { emax = max(emax, smax[w]); bad |= sbad[w]; }
         hinfo[hl] = make_int2(emax == -(1 << 30) ? 0 : emax, bad);
     }
 }
@@ -448,7 +450,8 @@ select_kernel(const float* __restrict__ scores, const double* __restrict__ Qbar,
     __shared__ int band_j[BAND_CAP];
     __shared__ unsigned long long band_key[BAND_CAP];
     __shared__ double qrow[HD];
-    __shared__ int wcnt[SWARPS], woff[SWARPS], scratch[SWARPS];
+    __shared__ unsigned int kept_words[MAX_T / 32];
+    __shared__ int wcnt[SWARPS], scratch[SWARPS];
     __shared__ float red_mn[SWARPS], red_mx[SWARPS];
     __shared__ int nband, sel_bucket, sel_above;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -510,7 +513,8 @@ select_kernel(const float* __restrict__ scores, const double* __restrict__ Qbar,
         hi_f = __double2float_ru(U + slack + 2.0 * E_BOUND);
     }
 
-    // ---- classify: kept (> hi), band, dropped (< lo); warp w owns [w seg, (w+1) seg)
+    // ---- classify: kept (> hi), band, dropped (< lo).  Warp w owns the 32-aligned
+    // range [w seg, (w+1) seg) and records the kept set as ballot words.
     const int seg = ((T + SWARPS - 1) / SWARPS + 31) & ~31;
     const int wb = warp * seg, we = min(T, wb + seg);
     int kept = 0;
@@ -522,7 +526,9 @@ select_kernel(const float* __restrict__ scores, const double* __restrict__ Qbar,
             is_kept = v > hi_f;
             is_band = exact || (v >= lo_f && v <= hi_f);
         }
-        kept += __popc(__ballot_sync(0xffffffffu, is_kept));
+        const unsigned int word = __ballot_sync(0xffffffffu, is_kept);
+        if (lane == 0) kept_words[j0 >> 5] = word;
+        kept += __popc(word);
         if (is_band) {
             const int slot = atomicAdd(&nband, 1);
             if (slot < BAND_CAP) band_j[slot] = j;
@@ -537,8 +543,16 @@ select_kernel(const float* __restrict__ scores, const double* __restrict__ Qbar,
     const int nb = nband;
 
     if (nb <= BAND_CAP) {
-        // ---- narrow band: fp64 scores, rank by (score desc, index asc)
-        for (int t = tid; t < nb; t += STHREADS) band_key[t] = order_key(score64(qrow, kh + static_cast<long long>(band_j[t]) * HD));
+        // ---- narrow band: fp64 scores (one warp per tile: lane l takes d = 2l, 2l + 1,
+        // then a butterfly sum that leaves the same value in every lane), ranked by
+        // (score desc, index asc); the band's top `need` join the kept words
+        for (int t = warp; t < nb; t += SWARPS) {
+            const double2 kv = __ldg(reinterpret_cast<const double2*>(kh + static_cast<long long>(band_j[t]) * HD) + lane);
+            double acc = fma(qrow[2 * lane], kv.x, qrow[2 * lane + 1] * kv.y);
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+            if (lane == 0) band_key[t] = order_key(acc);
+        }
         __syncthreads();
         for (int t = tid; t < nb; t += STHREADS) {
             const unsigned long long kt = band_key[t];
@@ -548,9 +562,7 @@ select_kernel(const float* __restrict__ scores, const double* __restrict__ Qbar,
                 const unsigned long long ku = band_key[u];
                 rank += (ku > kt || (ku == kt && band_j[u] < jt)) ? 1 : 0;
             }
-            const bool sel = rank < need;
-            xs[jt] = sel ? INFINITY : -INFINITY;
-            if (sel) atomicAdd(&wcnt[jt / seg], 1);
+            if (rank < need) atomicOr(&kept_words[jt >> 5], 1u << (jt & 31));
         }
         __syncthreads();
     } else {
@@ -587,7 +599,8 @@ select_kernel(const float* __restrict__ scores, const double* __restrict__ Qbar,
             __syncthreads();
             if (done || sh == 0) break;
         }
-        // marks in ascending j per thread range: above the prefix kept, equal ones lowest index first
+        // kept band tiles, in ascending j per thread range: above the prefix all, equal
+        // ones lowest index first
         const int per = (T + STHREADS - 1) / STHREADS;
         const int rb = min(T, tid * per), re = min(T, rb + per);
         int n_eq = 0;
@@ -598,39 +611,28 @@ select_kernel(const float* __restrict__ scores, const double* __restrict__ Qbar,
         for (int j = rb; j < re; ++j) {
             if (!in_band(j)) continue;
             const unsigned long long km = key_of(j) & mask;
-            const bool sel = km > prefix || (km == prefix && r++ < rem);
-            xs[j] = sel ? INFINITY : -INFINITY;
+            if (km > prefix || (km == prefix && r++ < rem)) atomicOr(&kept_words[j >> 5], 1u << (j & 31));
         }
-        __syncthreads();
-        int cnt = 0;
-        for (int j0 = wb; j0 < we; j0 += 32) {
-            const int j = j0 + lane;
-            bool sel = false;
-            if (j < we) { const float v = xs[j]; sel = v > hi_f || v == INFINITY; }
-            cnt += __popc(__ballot_sync(0xffffffffu, sel));
-        }
-        if (lane == 0) wcnt[warp] = cnt;
         __syncthreads();
     }
 
-    // ---- ascending output
-    if (tid == 0) {
-        int run = 0;
-        for (int w = 0; w < SWARPS; ++w) { woff[w] = run; run += wcnt[w]; }
-    }
-    __syncthreads();
+    // ---- ascending output from the kept words: thread t takes words [t wpt, (t+1) wpt)
+    const int nwords = (T + 31) >> 5;
+    const int wpt = (nwords + STHREADS - 1) / STHREADS;
+    const int w0 = min(nwords, tid * wpt), w1 = min(nwords, w0 + wpt);
+    int cnt = 0;
+    for (int w = w0; w < w1; ++w) cnt += __popc(kept_words[w]);
+    int total;
+    int pos = block_excl_scan(cnt, scratch, &total);
     int32_t* out = idx + (h * T + i) * static_cast<long long>(k);
-    int pos = woff[warp];
-    for (int j0 = wb; j0 < we; j0 += 32) {
-        const int j = j0 + lane;
-        bool sel = false;
-        if (j < we) { const float v = xs[j]; sel = v > hi_f || v == INFINITY; }
-        const unsigned int m = __ballot_sync(0xffffffffu, sel);
-        if (sel) {
-            const int p = pos + __popc(m & ((1u << lane) - 1u));
-            if (p < k) out[p] = j;
+    for (int w = w0; w < w1; ++w) {
+        unsigned int bits = kept_words[w];
+        while (bits) {
+            const int b = __ffs(bits) - 1;
+            bits &= bits - 1u;
+            if (pos < k) out[pos] = 32 * w + b;
+            ++pos;
         }
-        pos += __popc(m);
     }
 }
 
@@ -718,7 +720,7 @@ extern "C" zb_status zb_tile_score_topk(const double* Qbar, const double* Kbar, 
         const long long drows = 2ll * hn * T;
         topk::digits_kernel<<<static_cast<unsigned>((drows + 7) / 8), 256, 0, st>>>(Qbar, Kbar, T, h0, hn, qd, kd,
                                                                                     qe, ke);
-        topk::head_info_kernel<<<hn, 256, 0, st>>>(ke, static_cast<int>(T), hinfo);
+        topk::head_info_kernel<<<hn, topk::HI_THREADS, 0, st>>>(ke, static_cast<int>(T), hinfo);
         const long long tiles = hn * Tb * Tb;
         const int grid = static_cast<int>(tiles < dev.sm_count ? tiles : dev.sm_count);
         topk::score_i8_kernel<<<grid, topk::GTHREADS, topk::GEMM_SMEM, st>>>(
