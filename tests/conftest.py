@@ -27,3 +27,21 @@ def pytest_collection_modifyitems(config, items):
     for item in items:
         if "gpu" in item.keywords:
             item.add_marker(skip)
+
+
+def pytest_sessionfinish(session, exitstatus):
+    # ZB_PARITY_REPORT=<path>: write every float parity check of the session (per-head
+    # error against its bar, and the per-element figure with a floor of 1e-3 max|ref|)
+    path = os.environ.get("ZB_PARITY_REPORT")
+    if not path:
+        return
+    try:
+        from tests.gpu_helpers import REPORT
+    except Exception:  # pragma: no cover
+        return
+    import json
+    os.makedirs(os.path.dirname(os.path.abspath(path)), exist_ok=True)
+    with open(path, "w") as f:
+        json.dump({"checks": REPORT,
+                   "max_per_head": max((r["per_head"] for r in REPORT), default=None),
+                   "max_per_element": max((r["per_element"] for r in REPORT), default=None)}, f, indent=1)

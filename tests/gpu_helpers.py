@@ -25,6 +25,36 @@ def rel_err_per_head(got, ref):
     return max(errs)
 
 
+# the per-element figure reported beside it: |gpu - oracle| / max(|oracle|, floor),
+# floor = ELEM_FLOOR * max |oracle| of the head
+ELEM_FLOOR = 1e-3
+
+# (test, label, per-head error, per-element error) of every check_close in this session
+REPORT = []
+
+
+def elem_err_per_head(got, ref):
+    got = np.asarray(got, dtype=np.float64)
+    ref = np.asarray(ref, dtype=np.float64)
+    errs = []
+    for h in range(ref.shape[0]):
+        a = np.abs(ref[h])
+        den = np.maximum(a, ELEM_FLOOR * a.max()) if a.max() > 0 else np.ones_like(a)
+        errs.append((np.abs(got[h] - ref[h]) / den).max())
+    return max(errs)
+
+
+def check_close(got, ref, tol=REL_TOL, label=""):
+    """Assert the per-head error bar; record it with the per-element figure."""
+    import os
+    head = rel_err_per_head(got, ref)
+    elem = elem_err_per_head(got, ref)
+    REPORT.append({"test": os.environ.get("PYTEST_CURRENT_TEST", "").split(" ")[0], "label": label,
+                   "per_head": float(head), "per_element": float(elem), "tol": tol})
+    assert head <= tol, (label, head, elem)
+    return head, elem
+
+
 def bf16_round_f64(x):
     """Nearest bf16 value (ties to even) of fp64 values, returned as fp64.
 

@@ -7,7 +7,7 @@ import torch
 
 import oracle
 import synth
-from tests.gpu_helpers import REL_TOL, host, rel_err_per_head, sync_ok, workload
+from tests.gpu_helpers import REL_TOL, host, check_close, sync_ok, workload
 
 pytestmark = pytest.mark.gpu
 
@@ -50,8 +50,7 @@ def test_sparse_attention_matches_oracle(name, over, k):
     ref_idx = _oracle_idx(w, Q64, K64, k)
     assert np.array_equal(idx.cpu().numpy(), ref_idx)
     ref = oracle.sparse_attention(Q64, K64, V64, w.tile, ref_idx, 1 / math.sqrt(64))
-    err = rel_err_per_head(host(O), ref)
-    assert err <= REL_TOL, err
+    check_close(host(O), ref)
 
 
 def test_sparse_attention_rescales_o_when_the_row_max_grows():
@@ -79,8 +78,7 @@ def test_sparse_attention_rescales_o_when_the_row_max_grows():
                       for i, j1 in enumerate(ref_idx[h, :, -1][:23])] for h in range(2)])
     assert ((last - first) * lg > 8).mean() > 0.2
     ref = oracle.sparse_attention(Q64, K64, V64, w.tile, ref_idx, s)
-    err = rel_err_per_head(host(O), ref)
-    assert err <= REL_TOL, err
+    check_close(host(O), ref)
 
 
 def test_sparse_lse_matches_oracle_logsumexp():
@@ -110,7 +108,7 @@ def test_keep_all_tiles_equals_dense():
     Q, K, V = synth.make_qkv(w, device="cuda")
     O, idx = _sparse_gpu(w, Q, K, V, k=w.n_tiles)
     ref = oracle.dense_attention(host(Q), host(K), host(V), 1 / math.sqrt(64))
-    assert rel_err_per_head(host(O), ref) <= REL_TOL
+    check_close(host(O), ref)
 
 
 def test_tile_constant_keys_make_landmarks_exact():
@@ -123,7 +121,7 @@ def test_tile_constant_keys_make_landmarks_exact():
     for k in (0, 3, 11):
         O, _ = _sparse_gpu(w, Q, K, V, k=k)
         ref = oracle.dense_attention(host(Q), host(K), host(V), 1 / math.sqrt(64))
-        assert rel_err_per_head(host(O), ref) <= REL_TOL, k
+        check_close(host(O), ref, label=str(k))
 
 
 @pytest.mark.parametrize("k,use_lm", [(0, True), (4, False), (1, True)])
@@ -134,7 +132,7 @@ def test_sparse_variants(k, use_lm):
     Q64, K64, V64 = host(Q), host(K), host(V)
     ref_idx = _oracle_idx(w, Q64, K64, k)
     ref = oracle.sparse_attention(Q64, K64, V64, w.tile, ref_idx, 1 / math.sqrt(64), use_landmarks=use_lm)
-    assert rel_err_per_head(host(O), ref) <= REL_TOL
+    check_close(host(O), ref)
 
 
 def test_sparse_full_views32_sampled():
@@ -150,7 +148,7 @@ def test_sparse_full_views32_sampled():
     ref = oracle.sparse_attention(Q64, K64, V64, w.tile, ref_idx, 1 / math.sqrt(64), query_tiles=tiles)
     got = np.concatenate([host(O)[:, j * w.tile: j * w.tile + w.tile] for j in tiles[:-1]]
                          + [np.pad(host(O)[:, (w.n_tiles - 1) * w.tile:], ((0, 0), (0, 64), (0, 0)))], axis=1)
-    assert rel_err_per_head(got, ref) <= REL_TOL
+    check_close(got, ref)
     # every output row is a convex combination of value rows
     Vh = V.float()
     assert (O.float() <= Vh.amax(1, keepdim=True) + 1e-2).all()
@@ -183,4 +181,4 @@ def test_dense_matches_oracle(nq, nk):
     O = zb.zb_dense_attn(Q, K, V)
     sync_ok()
     ref = oracle.dense_attention(host(Q), host(K), host(V), 1 / 8)
-    assert rel_err_per_head(host(O), ref) <= REL_TOL
+    check_close(host(O), ref)

@@ -11,7 +11,7 @@ import torch
 
 import oracle
 import synth
-from tests.gpu_helpers import REL_TOL, host, rel_err_per_head, sync_ok, workload
+from tests.gpu_helpers import REL_TOL, host, check_close, sync_ok, workload
 
 pytestmark = pytest.mark.gpu
 
@@ -50,8 +50,7 @@ def test_spatial_sparse_stage_two_views_matches_oracle():
     Q64, K64, V64 = host(Q), host(K), host(V)
     ref, ref_idx = oracle.spatial_sparse_attention(Q64, K64, V64, w.tile, order, 1 / math.sqrt(64), w.k)
     assert np.array_equal(layer.idx.cpu().numpy(), ref_idx)
-    err = rel_err_per_head(host(O), ref)
-    assert err <= REL_TOL, err
+    check_close(host(O), ref)
     # the spatial order really changes the result against the plain tiling
     plain = zb.HybridLayer(w.heads, w.n_tokens, w.tile, w.k, [0]).sparse(Q, K, V)
     sync_ok()
@@ -90,6 +89,5 @@ def test_spatial_sparse_stage_32_views_full_size_sampled():
             rows_new = np.arange(i * w.tile, i * w.tile + n[i])
             want = ref[m * w.tile: m * w.tile + n[i]]
             part = got[order[rows_new]]          # original positions of the tile's tokens
-            err = np.abs(part - want).max() / np.abs(want).max()
-            assert err <= REL_TOL, (h, i, err)
+            check_close(part[None], want[None], label=f"head {h} tile {i}")
     del inv

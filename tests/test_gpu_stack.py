@@ -35,7 +35,7 @@ if ROOT not in sys.path:
 import oracle  # noqa: E402
 import synth  # noqa: E402
 from tests import stack_oracle_jobs as jobs  # noqa: E402
-from tests.gpu_helpers import REL_TOL, host, rel_err_per_head, sync_ok, workload  # noqa: E402
+from tests.gpu_helpers import REL_TOL, host, check_close, sync_ok, workload  # noqa: E402
 
 pytestmark = pytest.mark.gpu
 
@@ -74,8 +74,7 @@ def test_small_stack_matches_oracle_with_and_without_lookahead():
             idx = oracle.select_tiles(oracle.tile_scores(oracle.landmark_means(Q64, w.tile),
                                                          oracle.landmark_means(K64, w.tile)), w.k)
             ref = oracle.sparse_attention(Q64, K64, V64, w.tile, idx, s)
-        err = rel_err_per_head(host(outs[True][l]), ref)
-        assert err <= REL_TOL, (l, err)
+        check_close(host(outs[True][l]), ref)
 
 
 def _progress(t0, *what):
@@ -92,6 +91,12 @@ def test_stack_512_views_all_24_layers_full_size_sampled():
                        timeout=1200)
     assert r.returncode == 0, (r.stdout[-3000:], r.stderr[-3000:])
     assert "stack check passed" in r.stdout, r.stdout[-3000:]
+    import json
+    from tests.gpu_helpers import REPORT
+    for line in r.stdout.splitlines():
+        if line.startswith("stack parity "):
+            for rec in json.loads(line[len("stack parity "):]):
+                REPORT.append(dict(rec, test=rec["test"] or "tests/test_gpu_stack.py::_stack_512_full_size_check"))
 
 
 def _stack_512_full_size_check():
@@ -187,12 +192,15 @@ def _stack_512_full_size_check():
             for m, i in enumerate(tiles):
                 want = ref[m * t: m * t + n[i]] if l not in lin else ref[off: off + n[i]]
                 part = gotO[off: off + n[i]]
-                err = np.abs(part - want).max() / np.abs(want).max()
-                assert err <= REL_TOL, (l, h, i, err)
+                check_close(part[None], want[None], label=f"layer {l} head {h} tile {i}")
                 off += n[i]
 
 
 if __name__ == "__main__":
     torch.cuda.set_device(0)
     _stack_512_full_size_check()
+    import json
+    from tests.gpu_helpers import REPORT
+    # the parent test folds these into the session's parity report
+    print("stack parity " + json.dumps(REPORT), flush=True)
     print("stack check passed", flush=True)
