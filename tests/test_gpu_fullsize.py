@@ -109,3 +109,23 @@ def test_linear_stage_512_views_layer1_full_size_sampled():
     want = oracle.linear_attention(q64[:, srows], k64, v64, A, b)[0]
     got = host(o_l[h, srows])
     check_close(got[None], want[None], label=f"head {h}")
+
+
+def test_selection_1024_views_every_row_of_one_head():
+    """Every one of the 10,992 query tiles of head 5 at 1,024 views, in the bench's
+    launch configuration: the selected sets equal the oracle's."""
+    import linear_hybrid_attention_b200 as zb
+    w = workload("views1024")
+    Q, K, V = synth.make_qkv(w, device="cuda")
+    h = 5
+    lm = zb.zb_landmark_build(Q[h:h + 1].contiguous(), K[h:h + 1].contiguous(), V[h:h + 1].contiguous(), w.tile)
+    idx = zb.zb_tile_score_topk(lm.Qbar, lm.Kbar, w.n_tokens, w.tile, w.k)
+    sync_ok()
+    got = idx.cpu().numpy()[0]
+    del lm, idx
+    Qb = oracle.landmark_means(host(Q[h:h + 1]), w.tile)
+    Kb = oracle.landmark_means(host(K[h:h + 1]), w.tile)
+    del Q, K, V
+    ref = oracle.select_tiles(oracle.tile_scores(Qb, Kb), w.k)[0]
+    bad = np.flatnonzero((got != ref).any(-1))
+    assert bad.size == 0, (bad.size, bad[:5])
