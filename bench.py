@@ -225,6 +225,12 @@ def oracle_sample(w, Q, K, V, calib_tiles, sample_tiles=4, calib_rows=16, head=0
 
 
 # ------------------------------------------------------------------- main ----
+def landmark_flops(heads: int, n_tokens: int, n_tiles_: int, k: int, d: int) -> float:
+    """4 * d per (query row, landmark): every row attends to the T - k landmarks of its
+    omitted tiles (logit q . Kbar_j and the product with Vbar_j)."""
+    return float(4.0 * d * heads * n_tokens * (n_tiles_ - k))
+
+
 def selected_flops(idx_cpu: np.ndarray, n_tokens: int, tile: int, d: int) -> float:
     """4 * d * sum over (h, i, j in sel) n_i * n_j: the algorithmic FLOPs of QK^T and PV."""
     T = idx_cpu.shape[1]
@@ -616,6 +622,12 @@ def main():
                 "peak_kind": f"bf16 sustained ({peaks['source']}); kernel runs inside a long step",
                 "frac_of_burst": sparse_tf / peaks["bf16_tflops"],
                 "algorithmic": f"{flops:.4e} FLOP per launch = 4*d*sum n_i*n_j over kept (query tile, key tile) pairs"}
+    lm_flops = landmark_flops(w.heads, w.n_tokens, w.n_tiles, w.k, w.head_dim)
+    roofline["incl_landmarks"] = {
+        "achieved": (flops + lm_flops) / kt["sparse_attn"] / 1e12,
+        "frac": (flops + lm_flops) / kt["sparse_attn"] / 1e12 / peaks["bf16_tflops_sustained"],
+        "algorithmic": f"{flops + lm_flops:.4e} FLOP per launch: the kept pairs plus 4*d per (query row, landmark) "
+                       f"over the T - k landmarks of every row ({lm_flops:.3e})"}
     kernel_rooflines = {
         "zb_landmark_build": {"bound": "hbm", "achieved": lm_bytes / kt["landmark"] / 1e9, "peak": hbm,
                               "unit": "GB/s", "frac": lm_bytes / kt["landmark"] / 1e9 / hbm, "ms": kt["landmark"] * 1e3},

@@ -23,6 +23,13 @@ def test_selected_flops_counts_every_kept_pair():
     assert bench.selected_flops(idx, 300, 128, 64) == want
 
 
+def test_landmark_flops_count_every_row_and_omitted_tile():
+    # 2 heads, 300 tokens in 3 tiles, k = 2: every row sees 1 landmark
+    assert bench.landmark_flops(2, 300, 3, 2, 64) == 4 * 64 * 2 * 300 * 1
+    # the 1,024-view stage: 5.95e13 landmark FLOPs beside 4.87e14 selected
+    assert abs(bench.landmark_flops(16, 1_406_976, 10_992, 660, 64) - 5.95e13) / 5.95e13 < 1e-3
+
+
 def _fake_root(tmp_path, attn_src, recorded_sha, nbytes=123456.0):
     csrc = tmp_path / "linear_hybrid_attention_b200" / "csrc"
     csrc.mkdir(parents=True)
