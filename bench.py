@@ -498,6 +498,7 @@ def main():
     ap.add_argument("--no-block-mass", action="store_true", help="skip the block-mass diagnostic")
     ap.add_argument("--no-stack", action="store_true", help="skip the 24-layer 512-view stack")
     ap.add_argument("--no-spatial", action="store_true", help="skip the spatial-tiles measurement")
+    ap.add_argument("--no-keep20", action="store_true", help="skip the k = ceil(0.2 T) sparse-kernel point")
     ap.add_argument("--profile", action="store_true", help="short run for profilers: no JSON extras")
     args = ap.parse_args()
 
@@ -677,6 +678,40 @@ def main():
                      "note": "zb_dense_attn on head 0 at full length, scaled by the head count"}
         del Od
 
+    # ------------------------------------------ the pages' keep-20% point ----
+    # The same inputs with k = ceil(0.2 T) (the "0.8S" sparsity of Table 20's
+    # allocations): selection, then the tile-sparse kernel timed on its own
+    # (one warm-up launch, two timed), against the same sustained peak.
+    keep20 = None
+    if not args.no_keep20 and w.name == "views1024":
+        k20 = -(-w.n_tiles // 5)
+        idx20 = torch.empty((w.heads, w.n_tiles, k20), dtype=torch.int32, device=dev)
+        zb.zb_tile_score_topk(layer.lm.Qbar, layer.lm.Kbar, w.n_tokens, w.tile, k20, out=idx20, ws=layer.ws_topk)
+        n_t = torch.full((w.n_tiles,), float(w.tile), dtype=torch.float64, device=dev)
+        n_t[-1] = w.n_tokens - (w.n_tiles - 1) * w.tile
+        fl20 = sum(float(4.0 * w.head_dim * (n_t[idx20[h].long()].sum(-1) * n_t).sum().item())
+                   for h in range(w.heads))
+        lm20 = landmark_flops(w.heads, w.n_tokens, w.n_tiles, k20, w.head_dim)
+        run20 = lambda: zb.zb_tile_sparse_attn(Q, K, V, layer.lm.Kbar_bf16, layer.lm.Vbar_bf16, idx20, k20, w.tile,
+                                               True, layer.scale, out=layer.O_sparse, ws=layer.ws_attn)
+        run20()
+        torch.cuda.synchronize()
+        e20 = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
+        e20[0].record(stream)
+        run20()
+        e20[1].record(stream)
+        run20()
+        e20[2].record(stream)
+        torch.cuda.synchronize()
+        zb.zb_last_device_status()
+        t20 = statistics.mean([e20[0].elapsed_time(e20[1]), e20[1].elapsed_time(e20[2])]) / 1e3
+        keep20 = {"k": k20, "ms": t20 * 1e3, "tflops": fl20 / t20 / 1e12,
+                  "frac": fl20 / t20 / 1e12 / peaks["bf16_tflops_sustained"],
+                  "frac_incl_landmarks": (fl20 + lm20) / t20 / 1e12 / peaks["bf16_tflops_sustained"],
+                  "note": "zb_tile_sparse_attn alone on the 1,024-view inputs with the k = ceil(0.2 T) selection; "
+                          "frac on selected-tile FLOPs against the sustained bf16 peak"}
+        del idx20
+
     # -------------------------------------------- linear-centered variant ----
     # Outside the timed step: the centred linear stage (keys shifted by their
     # per-head mean) on the same inputs, its two new kernels against HBM, and
@@ -824,7 +859,7 @@ def main():
                 "roofline": roofline, "kernel_roofline": kernel_rooflines, "stage_ms": stage_ms,
                 "kernel_ms": {n: v * 1e3 for n, v in kt.items()}, "clocks": clk, "cpu_baseline": cpu,
                 "hybrid_0.7L_mtokens_s": hybrid_07, "dense_reference": dense_ref, "linear_centered": centered,
-                "block_mass": block_mass, "stack512": stack, "spatial_tiles": spatial,
+                "block_mass": block_mass, "stack512": stack, "spatial_tiles": spatial, "keep20": keep20,
                 "value_definition": "value = 2 N / t_step with every call of the hot path in the step, the "
                                     "calibration (dense attention on 4,096 rows) and the affine fit included",
                 "value_fit_offline": value_fit_offline,
