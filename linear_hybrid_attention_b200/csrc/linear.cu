@@ -689,14 +689,21 @@ linear_apply_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                 const float inv = 1.f / __uint_as_float(den);
                 const float* bb = sm.bvec[nb & 1];
                 uint8_t* orow = sm.ost[ob] + row * 128;
+                const uint64_t inv2 = f2_pack(inv, inv);
+                const uint2* bb2 = reinterpret_cast<const uint2*>(bb);
 #pragma unroll
                 for (int c = 0; c < 8; ++c) {
-                    float o[8];
+                    uint32_t pk[4];
 #pragma unroll
-                    for (int e = 0; e < 8; ++e) o[e] = fmaf(__uint_as_float(r[c * 8 + e]), inv, bb[c * 8 + e]);
-                    *reinterpret_cast<uint4*>(orow + ((c ^ (row & 7)) << 4)) =
-                        make_uint4(pack_bf16x2(o[0], o[1]), pack_bf16x2(o[2], o[3]), pack_bf16x2(o[4], o[5]),
-                                   pack_bf16x2(o[6], o[7]));
+                    for (int e = 0; e < 4; ++e) {
+                        const uint2 bv = bb2[c * 4 + e];
+                        const uint64_t o2 = f2_fma(f2_pack(__uint_as_float(r[c * 8 + 2 * e]), __uint_as_float(r[c * 8 + 2 * e + 1])),
+                                                   inv2, f2_pack(__uint_as_float(bv.x), __uint_as_float(bv.y)));
+                        float o0, o1;
+                        f2_unpack(o2, o0, o1);
+                        pk[e] = pack_bf16x2(o0, o1);
+                    }
+                    *reinterpret_cast<uint4*>(orow + ((c ^ (row & 7)) << 4)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
                 }
             }
             fence_proxy_async_smem();  // the TMA store reads the tile through the async proxy
