@@ -552,7 +552,7 @@ def main():
         zb.zb_linear_state(k, v, L.S, L.z, L.ws_lin)
         mark(4)
         zb.zb_gather_tiles(q, w.tile, L.calib, out=L.Qc)
-        zb.zb_dense_attn(L.Qc, k, v, L.scale, out=L.Yc, out_fp32=True)
+        zb.zb_dense_attn_split(L.Qc, k, v, L.calib_splits, L.scale, out=L.Yc, out_fp32=True, ws=L.ws_dense)
         mark(5)
         zb.zb_linear_apply(L.Qc, L.S, L.z, None, None, out=L.Xc, out_fp32=True)
         zb.zb_affine_fit(L.Xc, L.Yc, L.A, L.b, L.ws_fit)

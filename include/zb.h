@@ -168,6 +168,34 @@ zb_status zb_dense_attn(const uint16_t* Q, int64_t n_q, const uint16_t* K,
                         float* lse, void* stream);
 
 /*
+ * Dense softmax attention as zb_dense_attn, with the keys split into `splits`
+ * equal parts so that a small query set (the affine fit's calibration rows:
+ * "Zebra3D: Efficient Hybrid Foundation Models For Scalable 3D
+ * Reconstruction", Abstract, closed-form fit against the dense layer) fills
+ * the GPU.  The dense kernel runs over heads * splits virtual heads (virtual
+ * head h * splits + p sees keys [p n_kv / splits, (p + 1) n_kv / splits) of
+ * head h: the same [H][n_kv][d] memory viewed as [H * splits][n_kv / splits][d])
+ * into fp32 partial outputs with their log-sum-exp, and a merge kernel forms
+ *   O = sum_p e^(lse_p - M) O_p / sum_p e^(lse_p - M),  M = max_p lse_p,
+ *   lse = M + ln sum_p e^(lse_p - M)  (natural log),
+ * the softmax over all n_kv keys.  splits == 1 is zb_dense_attn itself.
+ *   in : Q bf16 [H][n_q][d];  K, V bf16 [H][n_kv][d];  1 <= splits <= 16,
+ *        n_kv a multiple of splits
+ *   ws : zb_dense_attn_split_workspace_bytes() bytes (0 for splits == 1):
+ *        query replicas, partial outputs and their lse; 16-byte aligned,
+ *        owned by the caller, not shared with a call running at the same time
+ *   out: O [H][n_q][d], bf16 (out_fp32 == 0) or fp32;  lse fp32 [H][n_q]
+ *        (may be NULL)
+ * Errors: ZB_ERR_NULL, ZB_ERR_SHAPE (also n_kv not a multiple of splits),
+ * ZB_ERR_ALIGN, ZB_ERR_UNSUPPORTED, ZB_ERR_WORKSPACE, ZB_ERR_CUDA.
+ */
+size_t zb_dense_attn_split_workspace_bytes(int64_t n_q, int32_t heads, int32_t head_dim, int32_t splits);
+zb_status zb_dense_attn_split(const uint16_t* Q, int64_t n_q, const uint16_t* K, const uint16_t* V,
+                              int64_t n_kv, int32_t heads, int32_t head_dim, float scale, int32_t splits,
+                              void* O, int32_t out_fp32, float* lse, void* ws, size_t ws_bytes,
+                              void* stream);
+
+/*
  * Linear-attention state (Abstract: linear attention for tolerant stages):
  *   S[h] = sum_r phi(k_r)^T v_r  (d x d),  z[h] = sum_r phi(k_r)  (d),
  * phi(x) = elu(x) + 1, non-causal over all N tokens.  phi(k) is rounded to

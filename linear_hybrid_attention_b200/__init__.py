@@ -26,7 +26,7 @@ from . import _lib
 
 __all__ = [
     "ZbError", "Landmarks", "zb_abi_version", "zb_landmark_build", "zb_tile_score_topk",
-    "zb_tile_sparse_attn", "zb_dense_attn", "zb_linear_state", "zb_linear_apply", "zb_linear_attn",
+    "zb_tile_sparse_attn", "zb_dense_attn", "zb_dense_attn_split", "dense_splits", "zb_linear_state", "zb_linear_apply", "zb_linear_attn",
     "zb_affine_fit", "zb_gather_tiles", "zb_last_device_status", "HybridLayer",
     "LAUNCHES_PER_CALL", "zb_key_mean", "zb_linear_state_centered", "zb_block_mass",
     "zb_block_mass_top_fraction", "zb_block_mass_selected_fraction", "zb_spatial_order", "zb_gather_rows",
@@ -39,6 +39,7 @@ HEAD_DIM = 64
 # (topk_launches gives the count of one call)
 LAUNCHES_PER_CALL = {
     "zb_landmark_build": 1, "zb_tile_score_topk": 4, "zb_tile_sparse_attn": 1, "zb_dense_attn": 1,
+    "zb_dense_attn_split": 2,
     "zb_linear_state": 2, "zb_linear_apply": 1, "zb_linear_attn": 3, "zb_affine_fit": 3, "zb_gather_tiles": 1,
     "zb_key_mean": 2, "zb_linear_state_centered": 2, "zb_block_mass": 1, "zb_block_mass_top_fraction": 1,
     "zb_block_mass_selected_fraction": 1, "zb_gather_rows": 1, "zb_spatial_order": 0,
@@ -215,6 +216,53 @@ def zb_dense_attn(Q, K, V, scale: Optional[float] = None, out: Optional[torch.Te
     st = _lib_handle().zb_dense_attn(_ptr(Q), Nq, _ptr(K), _ptr(V), Nk, H, d, float(scale), _ptr(O),
                                      1 if out_fp32 else 0, _ptr(lse), _stream())
     _check(st, "zb_dense_attn")
+    return (O, lse) if lse is not None else O
+
+
+def dense_splits(heads: int, n_q: int, n_kv: int, sms: int, slots_per_sm: int = 2, max_splits: int = 8) -> int:
+    """Key splits for zb_dense_attn_split: among the counts that divide n_kv, the one
+    whose work items (heads x query tiles x splits, each 1/splits of a row sweep) fill
+    the GPU's sms * slots_per_sm attention pipelines in the fewest sweep lengths (ties
+    to fewer splits); no split unless that saves at least 5% (each item also loads
+    its queries and writes an epilogue, and the parts are merged)."""
+    items = heads * -(-n_q // 128)
+    slots = max(1, sms * slots_per_sm)
+    unsplit = -(-items // slots)
+    best, best_cost = 1, unsplit
+    for s in range(2, max_splits + 1):
+        if n_kv % s:
+            continue
+        cost = -(-items * s // slots) / s
+        if cost < best_cost - 1e-9:
+            best, best_cost = s, cost
+    return best if best_cost <= 0.95 * unsplit else 1
+
+
+def dense_split_workspace_bytes(n_q: int, heads: int, splits: int, head_dim: int = HEAD_DIM) -> int:
+    return int(_lib_handle().zb_dense_attn_split_workspace_bytes(n_q, heads, head_dim, splits))
+
+
+def zb_dense_attn_split(Q, K, V, splits: int, scale: Optional[float] = None, out: Optional[torch.Tensor] = None,
+                        lse: Optional[torch.Tensor] = None, want_lse: bool = False, out_fp32: bool = False,
+                        ws: Optional[torch.Tensor] = None):
+    """Dense softmax attention with the keys split in `splits` equal parts and merged
+    (same result as zb_dense_attn; fills the GPU for small query sets)."""
+    for t, n in ((Q, "Q"), (K, "K"), (V, "V")):
+        _need(t, torch.bfloat16, n, 3)
+    H, Nq, d = Q.shape
+    Nk = K.shape[1]
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    O = _out((H, Nq, d), torch.float32 if out_fp32 else torch.bfloat16, Q.device, out, "O")
+    if want_lse or lse is not None:
+        lse = _out((H, Nq), torch.float32, Q.device, lse, "lse")
+    need = dense_split_workspace_bytes(Nq, H, splits, d)
+    if ws is None and need > 0:
+        ws = torch.empty(need, dtype=torch.uint8, device=Q.device)
+    st = _lib_handle().zb_dense_attn_split(_ptr(Q), Nq, _ptr(K), _ptr(V), Nk, H, d, float(scale), int(splits), _ptr(O),
+                                           1 if out_fp32 else 0, _ptr(lse), _ptr(ws),
+                                           0 if ws is None else ws.numel() * ws.element_size(), _stream())
+    _check(st, "zb_dense_attn_split")
     return (O, lse) if lse is not None else O
 
 
@@ -471,6 +519,12 @@ class HybridLayer:
         self.b = torch.empty(H, d, dtype=torch.float32, device=dev)
         self.ws_fit = torch.empty(max(affine_fit_workspace_bytes(H, max(R, d + 1), d), 16), dtype=torch.uint8,
                                   device=dev)
+        # the calibration's dense pass splits the keys so that its H x R / 128 work
+        # items fill the GPU
+        sms = torch.cuda.get_device_properties(dev).multi_processor_count if dev.type == "cuda" else 148
+        self.calib_splits = dense_splits(H, R, N, sms)
+        self.ws_dense = torch.empty(max(dense_split_workspace_bytes(R, H, self.calib_splits, d), 16),
+                                    dtype=torch.uint8, device=dev)
         # spatial tiles: (views, grid, specials, win_rows, win_cols); the sparse stage
         # runs on the tokens gathered into zb_spatial_order's order
         self.spatial = None
@@ -488,8 +542,7 @@ class HybridLayer:
     LAUNCHES = {
         "sparse": LAUNCHES_PER_CALL["zb_landmark_build"] + LAUNCHES_PER_CALL["zb_tile_sparse_attn"],
         "calibrate": LAUNCHES_PER_CALL["zb_linear_state"] + LAUNCHES_PER_CALL["zb_gather_tiles"]
-        + LAUNCHES_PER_CALL["zb_dense_attn"] + LAUNCHES_PER_CALL["zb_linear_apply"]
-        + LAUNCHES_PER_CALL["zb_affine_fit"],
+        + LAUNCHES_PER_CALL["zb_linear_apply"] + LAUNCHES_PER_CALL["zb_affine_fit"],  # + the dense pass
         "linear": LAUNCHES_PER_CALL["zb_linear_apply"],
     }
 
@@ -520,7 +573,8 @@ class HybridLayer:
     def calibrate(self, Q, K, V):
         self._state(K, V)
         zb_gather_tiles(Q, self.tile, self.calib, out=self.Qc)
-        zb_dense_attn(self.Qc, K, V, self.scale, out=self.Yc, out_fp32=True)
+        zb_dense_attn_split(self.Qc, K, V, self.calib_splits, self.scale, out=self.Yc, out_fp32=True,
+                            ws=self.ws_dense)
         zb_linear_apply(self.Qc, self.S, self.z, None, None, out=self.Xc, out_fp32=True)
         zb_affine_fit(self.Xc, self.Yc, self.A, self.b, self.ws_fit)
         return self.A, self.b
@@ -543,4 +597,10 @@ class HybridLayer:
         if self.spatial is not None:
             extra += 4 * LAUNCHES_PER_CALL["zb_gather_rows"]
         topk = topk_launches(self.heads, self.n_tokens, self.tile, self.k, self.ws_topk.numel())
-        return self.LAUNCHES["sparse"] + topk + self.LAUNCHES["calibrate"] + extra + self.LAUNCHES["linear"]
+        return (self.LAUNCHES["sparse"] + topk + self.LAUNCHES["calibrate"] + self.dense_launches + extra
+                + self.LAUNCHES["linear"])
+
+    @property
+    def dense_launches(self) -> int:
+        """Kernels of the calibration's dense pass (the dense kernel, and the merge when split)."""
+        return LAUNCHES_PER_CALL["zb_dense_attn_split" if self.calib_splits > 1 else "zb_dense_attn"]

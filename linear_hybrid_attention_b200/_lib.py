@@ -31,6 +31,9 @@ PROTOTYPES = {
     "zb_tile_sparse_attn": (c_i32, [c_vp, c_vp, c_vp, c_vp, c_vp, c_vp, c_i32, c_i32, c_f32, ZbShape,
                                     c_vp, c_vp, c_vp, c_sz, c_vp]),
     "zb_dense_attn": (c_i32, [c_vp, c_i64, c_vp, c_vp, c_i64, c_i32, c_i32, c_f32, c_vp, c_i32, c_vp, c_vp]),
+    "zb_dense_attn_split_workspace_bytes": (c_sz, [c_i64, c_i32, c_i32, c_i32]),
+    "zb_dense_attn_split": (c_i32, [c_vp, c_i64, c_vp, c_vp, c_i64, c_i32, c_i32, c_f32, c_i32, c_vp, c_i32, c_vp,
+                                    c_vp, c_sz, c_vp]),
     "zb_linear_state_workspace_bytes": (c_sz, [c_i32, c_i64, c_i32]),
     "zb_linear_state": (c_i32, [c_vp, c_vp, c_i32, c_i64, c_i32, c_vp, c_vp, c_vp, c_sz, c_vp]),
     "zb_linear_state_static_scratch_bytes": (c_sz, []),

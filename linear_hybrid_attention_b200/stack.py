@@ -26,7 +26,7 @@ from typing import Callable, Optional, Sequence
 
 import torch
 
-from . import (HybridLayer, zb_affine_fit, zb_dense_attn, zb_gather_tiles, zb_landmark_build,
+from . import (HybridLayer, zb_affine_fit, zb_dense_attn_split, zb_gather_tiles, zb_landmark_build,
                zb_linear_apply, zb_tile_score_topk, zb_tile_sparse_attn)
 
 
@@ -65,7 +65,7 @@ class HybridStack:
     def _back(self, layer: int, buf: HybridLayer, Q, K, V) -> torch.Tensor:
         """The rest of the layer; returns its output buffer."""
         if self.is_linear(layer):
-            zb_dense_attn(buf.Qc, K, V, buf.scale, out=buf.Yc, out_fp32=True)
+            zb_dense_attn_split(buf.Qc, K, V, buf.calib_splits, buf.scale, out=buf.Yc, out_fp32=True, ws=buf.ws_dense)
             zb_linear_apply(buf.Qc, buf.S, buf.z, None, None, out=buf.Xc, out_fp32=True)
             zb_affine_fit(buf.Xc, buf.Yc, buf.A, buf.b, buf.ws_fit)
             return zb_linear_apply(Q, buf.S, buf.z, buf.A, buf.b, out=buf.O_linear)
@@ -77,10 +77,11 @@ class HybridStack:
         n = 0
         for l in range(self.n_layers):
             b = self.bufs[l & 1]
+            calib = b.LAUNCHES["calibrate"] + b.dense_launches
             if self.is_linear(l):
-                n += b.LAUNCHES["calibrate"] + b.LAUNCHES["linear"]
+                n += calib + b.LAUNCHES["linear"]
             else:
-                n += b.launches_per_step - b.LAUNCHES["calibrate"] - b.LAUNCHES["linear"]
+                n += b.launches_per_step - calib - b.LAUNCHES["linear"]
         return n
 
     # ---------------------------------------------------------------- run ----

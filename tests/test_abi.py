@@ -184,3 +184,37 @@ def test_topk_launch_count_follows_the_launcher():
     assert topk_launches(3, N, t, 660, 2 * one) == 8         # passes of 2 and 1 heads
     assert topk_launches(16, N, t, 0, 0) == 0
     assert topk_launches(16, N, t, T, 0) == 1
+
+
+def test_dense_split_validation_and_workspace(lib):
+    # workspace: query replicas (bf16), partial outputs (fp32) and their lse, 256-byte aligned
+    al = lambda x: -(-x // 256) * 256
+    rows = 4096 * 16 * 4
+    assert lib.zb_dense_attn_split_workspace_bytes(4096, 16, 64, 4) == al(rows * 128) + al(rows * 256) + al(rows * 4)
+    assert lib.zb_dense_attn_split_workspace_bytes(4096, 16, 64, 1) == 0
+    assert lib.zb_dense_attn_split_workspace_bytes(4096, 16, 64, 17) == 0
+    assert lib.zb_dense_attn_split_workspace_bytes(4096, 16, 32, 4) == 0
+    call = lambda nq, nk, H, d, s, O, ws, wsb: lib.zb_dense_attn_split(FAKE, nq, FAKE, FAKE, nk, H, d, 0.125, s, O,
+                                                                       1, None, ws, wsb, None)
+    assert call(100, 1001, 2, 64, 4, FAKE, FAKE, 1 << 30) == 2     # keys not a multiple of the splits
+    assert call(100, 1000, 2, 64, 0, FAKE, FAKE, 1 << 30) == 2     # no split
+    assert call(100, 1000, 2, 64, 17, FAKE, FAKE, 1 << 30) == 2    # too many
+    assert call(100, 1000, 2, 32, 4, FAKE, FAKE, 1 << 30) == 4     # head_dim
+    assert call(100, 1000, 2, 64, 4, None, FAKE, 1 << 30) == 1     # no output
+    assert call(100, 1000, 2, 64, 4, FAKE + 8, FAKE, 1 << 30) == 3 # misaligned output
+    need = lib.zb_dense_attn_split_workspace_bytes(100, 2, 64, 4)
+    assert call(100, 1000, 2, 64, 4, FAKE, FAKE, need - 1) == 5    # workspace too small
+    assert call(100, 1000, 2, 64, 4, FAKE, None, need) == 5        # no workspace
+
+
+def test_dense_splits_fill_the_pipelines():
+    from linear_hybrid_attention_b200 import dense_splits
+    # calibration at 1,024 views: 16 heads x 32 query tiles on 148 SMs x 2 pipelines;
+    # 512 items need 2 sweeps, 4 splits 7 quarter sweeps (1.75)
+    assert dense_splits(16, 4096, 1_406_976, 148) == 4
+    # enough items already: no split
+    assert dense_splits(16, 128 * 300, 1_406_976, 148) == 1
+    # only counts dividing the key count
+    assert dense_splits(16, 4096, 1_406_977, 148) == 1
+    # one head, one query tile: as many splits as allowed that divide the keys
+    assert dense_splits(1, 128, 8 * 1000, 148) == 8

@@ -182,3 +182,36 @@ def test_dense_matches_oracle(nq, nk):
     sync_ok()
     ref = oracle.dense_attention(host(Q), host(K), host(V), 1 / 8)
     check_close(host(O), ref)
+
+
+@pytest.mark.parametrize("nq,nk,splits", [(300, 1000, 4), (4096, 6000, 3), (1, 77, 7), (257, 4096, 2), (128, 640, 5)])
+def test_dense_split_matches_oracle(nq, nk, splits):
+    """Keys split in equal parts and merged by log-sum-exp: the dense softmax over
+    all keys, in fp32 and bf16 outputs, with the merged log-sum-exp."""
+    zb = _zb()
+    g = torch.Generator(device="cuda").manual_seed(3 * nq + nk + splits)
+    H = 3
+    Q = torch.randn(H, nq, 64, generator=g, device="cuda").to(torch.bfloat16)
+    K = torch.randn(H, nk, 64, generator=g, device="cuda").to(torch.bfloat16)
+    V = torch.randn(H, nk, 64, generator=g, device="cuda").to(torch.bfloat16)
+    O32, lse = zb.zb_dense_attn_split(Q, K, V, splits, want_lse=True, out_fp32=True)
+    O16 = zb.zb_dense_attn_split(Q, K, V, splits)
+    sync_ok()
+    q, k, v = host(Q), host(K), host(V)
+    ref = oracle.dense_attention(q, k, v, 1 / 8)
+    check_close(O32.cpu().numpy(), ref, label=f"fp32 splits {splits}")
+    check_close(host(O16), ref, label=f"bf16 splits {splits}")
+    logits = np.einsum("hqd,hkd->hqk", q, k) / 8
+    m = logits.max(-1)
+    ref_lse = m + np.log(np.exp(logits - m[..., None]).sum(-1))
+    assert np.abs(lse.cpu().numpy() - ref_lse).max() <= 1e-2 * max(1.0, np.abs(ref_lse).max())
+
+
+def test_dense_split_of_one_is_the_dense_call():
+    zb = _zb()
+    w = workload("tiny")
+    Q, K, V = synth.make_qkv(w, device="cuda")
+    a = zb.zb_dense_attn(Q, K, V, out_fp32=True)
+    b = zb.zb_dense_attn_split(Q, K, V, 1, out_fp32=True)
+    sync_ok()
+    assert torch.equal(a, b)
