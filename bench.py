@@ -163,6 +163,36 @@ def read_stream_gbs(device, gib: int = 4, reps: int = 5) -> float:
     return nbytes / min(times) / 1e9
 
 
+def hbm_isolated(fns: dict, device, local_rank: int, seconds: float = 0.5) -> dict:
+    """Each HBM kernel alone: launched back to back for about `seconds` (L2 flushed
+    before every launch), CUDA events around each launch, nvidia-smi clocks sampled
+    over the whole loop.  Returns the median ms of each and the clock record."""
+    flush = L2Flush(device)
+    for fn in fns.values():
+        fn()
+    torch.cuda.synchronize()
+    clocks = ClockSampler(local_rank)
+    clocks.start()
+    out = {}
+    for name, fn in fns.items():
+        evs = []
+        t0 = time.time()
+        while time.time() - t0 < seconds:
+            for _ in range(20):
+                flush()
+                a = torch.cuda.Event(enable_timing=True)
+                b = torch.cuda.Event(enable_timing=True)
+                a.record()
+                fn()
+                b.record()
+                evs.append((a, b))
+            torch.cuda.synchronize()
+        out[name] = statistics.median(a.elapsed_time(b) for a, b in evs)
+    clk = clocks.stop()
+    del flush
+    return {"ms": out, "clocks": clk}
+
+
 # --------------------------------------------------------------- CPU oracle ----
 def oracle_sample(w, Q, K, V, calib_tiles, sample_tiles=4, calib_rows=16, head=0):
     """Time the fp64 oracle on a bounded sample of one head and extrapolate.
@@ -835,6 +865,23 @@ def main():
             kr["frac_of_spec"] = kr["achieved"] / SPEC_HBM_GBS
     hbm_peaks = {"copy_gbs (MEASURED_PEAKS.json, the roofline peak)": hbm, "read_stream_gbs (measured here)": read_gbs,
                  "spec_gbs": SPEC_HBM_GBS}
+    # the same kernels alone, at the clock they then run at: the in-step figures
+    # above run at the clock the long tile-sparse kernel leaves under the power cap
+    iso = hbm_isolated({
+        "zb_landmark_build": lambda: zb.zb_landmark_build(Q, K, V, w.tile, out=layer.lm),
+        "zb_linear_state": lambda: zb.zb_linear_state(K, V, layer.S, layer.z, layer.ws_lin),
+        "zb_linear_apply": lambda: zb.zb_linear_apply(Q, layer.S, layer.z, layer.A, layer.b, out=layer.O_linear),
+    }, dev, local_rank)
+    iso_bytes = {"zb_landmark_build": lm_bytes, "zb_linear_state": lin_state_bytes, "zb_linear_apply": lin_apply_bytes}
+    for n, ms in iso["ms"].items():
+        kernel_rooflines[n]["alone"] = {"ms": ms, "frac": iso_bytes[n] / (ms / 1e3) / 1e9 / hbm}
+    t_iso = iso["ms"]["zb_linear_state"] + iso["ms"]["zb_linear_apply"]
+    kernel_rooflines["zb_linear_attn (state + apply)"]["alone"] = {
+        "ms": t_iso, "frac": (lin_state_bytes + lin_apply_bytes) / (t_iso / 1e3) / 1e9 / hbm}
+    hbm_clocks = {"in_step": clk, "alone": iso["clocks"],
+                  "note": "frac is measured inside the timed step (clocks: the step's samples, mostly during the "
+                          "tile-sparse kernel); alone = each kernel launched back to back for 0.5 s with L2 "
+                          "flushed before every launch (clocks sampled over that loop)"}
 
     # the step without calibration: the affine fit done once, offline, and the
     # fitted (A, b) reused -- the linear stage is then its two passes
@@ -865,7 +912,7 @@ def main():
                 "value_fit_offline": value_fit_offline,
                 "value_fit_offline_definition": "2 N / (landmarks + selection + tile-sparse attention + linear "
                                                 "state + fitted linear output): the fit done once, offline",
-                "hbm_peaks": hbm_peaks, "peaks": peaks}
+                "hbm_peaks": hbm_peaks, "hbm_kernel_clocks": hbm_clocks, "peaks": peaks}
         print(json.dumps(line), flush=True)
     if world > 1:
         torch.distributed.destroy_process_group()
