@@ -408,20 +408,22 @@ __global__ void key_mean_reduce_kernel(const double* __restrict__ partial, int c
 //   warp 0       TMA producer of the Q tiles (ring of AP_STAGES);
 //   warp 1       MMA issuer: D[128 x 80] = phi(Q) B^T into one of D_BUFS TMEM
 //                accumulators (80 of 128 columns each);
-//   warps 2..7   phi in place on each Q tile in shared memory; warps 4..7
-//                also build the B operand / bias of each new head;
-//   warps 8..11  epilogue: one thread per row, O = D[:64] / D[64] + b', each
-//                thread writing its whole 128-byte bf16 row.
+//   warps 2..5   phi in place on each Q tile in shared memory, and the B
+//                operand / bias of each new head;
+//   warps 6..13  epilogue, two warps per TMEM lane quarter (warp w reads lanes
+//                32 (w % 4).., columns 32 ((w - 6) / 4)..): O = D / D[64] + b'
+//                for half a row per thread, into a swizzled staging tile.
 // The roles only meet at mbarriers, so loads, phi, MMA and stores of
 // successive tiles overlap.
 constexpr int AP_STAGES = 6;
-constexpr int AP_THREADS = 384;
+constexpr int AP_THREADS = 448;
 constexpr int D_BUFS = 4;
 constexpr int BN_ROWS = 80;  // 64 columns of S A, one of z, 15 of zeros
 constexpr uint32_t B_BYTES = BN_ROWS * 128;
 constexpr int PHI_BAR = 1;   // named barrier of the operand builders (warps 4..7, 128 threads)
-constexpr int PHI_THREADS = 192;  // warps 2..7 apply phi
-constexpr int EPI_BAR = 2;        // named barrier of the epilogue warps (128 threads)
+constexpr int PHI_THREADS = 128;  // warps 2..5 apply phi
+constexpr int EPI_BAR = 2;        // named barrier of the epilogue warps (256 threads)
+constexpr int EPI_THREADS = 256;
 
 struct ApplySmem {
     uint8_t q[AP_STAGES][TILE_BYTES];
@@ -464,12 +466,12 @@ linear_apply_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
         }
         for (int d = 0; d < D_BUFS; ++d) {
             mbar_init(smem_addr(&sm.mma_done[d]), 1);
-            mbar_init(smem_addr(&sm.d_free[d]), 128);
+            mbar_init(smem_addr(&sm.d_free[d]), EPI_THREADS);
         }
         for (int i = 0; i < 2; ++i) {
             mbar_init(smem_addr(&sm.b_free[i]), 1);
             mbar_init(smem_addr(&sm.bvec_ready[i]), 128);
-            mbar_init(smem_addr(&sm.bvec_free[i]), 128);
+            mbar_init(smem_addr(&sm.bvec_free[i]), EPI_THREADS);
         }
         mbar_init(smem_addr(&sm.drain), 1);
         fence_mbar_init();
@@ -542,13 +544,13 @@ linear_apply_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
             mbar_wait(smem_addr(&sm.drain), 0, w2);
         }
         __syncwarp();
-    } else if (warp >= 2 && warp < 8) {
+    } else if (warp >= 2 && warp < 6) {
         // ======================================= phi and per-head operands ====
         // Every thread runs every iteration (after an abort it skips the waits
         // and the work but keeps the builders' named barriers matched).
-        const int t = tid - 128;          // builder index (warps 4..7)
-        const int tp = tid - 64;          // phi index (warps 2..7)
-        const bool builder = warp >= 4;
+        const int t = tid - 64;           // builder index (warps 2..5)
+        const int tp = tid - 64;          // phi index (warps 2..5)
+        const bool builder = true;
         int h_prev = -1, nb = -1;
         bool ok = true;
         for (int it = 0; it < cnt; ++it) {
@@ -647,7 +649,7 @@ linear_apply_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
             fence_proxy_async_smem();  // the MMA reads phi(Q) and B through the async proxy
             mbar_arrive(smem_addr(&sm.phi_done[s]));
         }
-    } else if (warp >= 8) {
+    } else if (warp >= 6) {
         // ================================================== epilogue ====
         // Each thread writes its row into a 128-byte-swizzled staging tile (no
         // bank conflicts); one thread then stores the tile with TMA (rows past
@@ -655,7 +657,8 @@ linear_apply_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
         // abort it skips the waits and the work but keeps the named barriers
         // matched).
         const int row = (warp & 3) * 32 + lane;
-        const int et = tid - 256;
+        const int hf = (warp - 6) >> 2;  // column half of the row
+        const int et = tid - 192;
         const uint32_t lane_addr = static_cast<uint32_t>((warp & 3) * 32) << 16;
         int h_prev = -1, nb = -1;
         bool ok = true;
@@ -672,17 +675,15 @@ linear_apply_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
             const uint32_t du = static_cast<uint32_t>(it / D_BUFS);
             // the store from this staging buffer two tiles ago has read it
             if (et == 0) bulk_wait_group_read<1>();
-            named_bar_sync(EPI_BAR, 128);
+            named_bar_sync(EPI_BAR, EPI_THREADS);
             if (ok && !mbar_wait(smem_addr(&sm.mma_done[d]), du & 1, wc)) ok = false;
             if (ok) {
                 tc_fence_after();
-                uint32_t r[64], den;
+                uint32_t r[32], den;
                 const uint32_t ta = tmem + lane_addr + d * 128;
-                tmem_ld32(ta, sub32(r, 0));
-                tmem_ld32(ta + 32, sub32(r, 32));
+                tmem_ld32(ta + 32 * hf, r);
                 asm volatile("tcgen05.ld.sync.aligned.32x32b.x1.b32 {%0}, [%1];" : "=r"(den) : "r"(ta + 64));
-                tmem_wait_ld_dep(sub32(r, 0));
-                tmem_wait_ld_dep(sub32(r, 32));
+                tmem_wait_ld_dep(r);
                 asm volatile("tcgen05.wait::ld.sync.aligned;" : "+r"(den)::"memory");
                 tc_fence_before();
                 mbar_arrive(smem_addr(&sm.d_free[d]));
@@ -692,12 +693,13 @@ linear_apply_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                 const uint64_t inv2 = f2_pack(inv, inv);
                 const uint2* bb2 = reinterpret_cast<const uint2*>(bb);
 #pragma unroll
-                for (int c = 0; c < 8; ++c) {
+                for (int cc = 0; cc < 4; ++cc) {
+                    const int c = 4 * hf + cc;
                     uint32_t pk[4];
 #pragma unroll
                     for (int e = 0; e < 4; ++e) {
                         const uint2 bv = bb2[c * 4 + e];
-                        const uint64_t o2 = f2_fma(f2_pack(__uint_as_float(r[c * 8 + 2 * e]), __uint_as_float(r[c * 8 + 2 * e + 1])),
+                        const uint64_t o2 = f2_fma(f2_pack(__uint_as_float(r[cc * 8 + 2 * e]), __uint_as_float(r[cc * 8 + 2 * e + 1])),
                                                    inv2, f2_pack(__uint_as_float(bv.x), __uint_as_float(bv.y)));
                         float o0, o1;
                         f2_unpack(o2, o0, o1);
@@ -707,7 +709,7 @@ linear_apply_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                 }
             }
             fence_proxy_async_smem();  // the TMA store reads the tile through the async proxy
-            named_bar_sync(EPI_BAR, 128);
+            named_bar_sync(EPI_BAR, EPI_THREADS);
             if (et == 0 && ok) {
                 tma_store_3d(&tm_o, smem_addr(sm.ost[ob]), 0, t * TILE, h);
                 bulk_commit_group();
