@@ -350,7 +350,7 @@ score_i8_kernel(const int8_t* __restrict__ qd, const int8_t* __restrict__ kd, co
 }
 
 // ------------------------------------------------------------ select ----
-constexpr int STHREADS = 512;
+constexpr int STHREADS = 256;
 constexpr int SWARPS = STHREADS / 32;
 constexpr int NBINS = 4096;
 constexpr int BPT = NBINS / STHREADS;  // bins per thread in the bucket search
@@ -441,7 +441,7 @@ ZB_DEVINL int lin_bin(float v, float a, float c) {
 }
 
 // grid: heads in group x T query rows.
-__global__ void __launch_bounds__(STHREADS, 2)
+__global__ void __launch_bounds__(STHREADS, 3)
 select_kernel(const float* __restrict__ scores, const double* __restrict__ Qbar, const double* __restrict__ Kbar,
               const int* __restrict__ qe, const int2* __restrict__ hinfo, int T, int Tp, int k, int h0,
               int32_t* __restrict__ idx) {
