@@ -471,7 +471,7 @@ select_kernel(const float* __restrict__ scores, const double* __restrict__ Qbar,
             if (4 * q + u < T) { mn = fminf(mn, w[u]); mx = fmaxf(mx, w[u]); }
     }
     if (tid < HD) qrow[tid] = Qbar[(h * T + i) * HD + tid];
-    const bool exact = hinfo[hl].y != 0 || qe[static_cast<long long>(hl) * T + i] == EXP_NONFINITE;
+    bool exact = hinfo[hl].y != 0 || qe[static_cast<long long>(hl) * T + i] == EXP_NONFINITE;
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) {
         mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, o));
@@ -517,30 +517,46 @@ select_kernel(const float* __restrict__ scores, const double* __restrict__ Qbar,
     // range [w seg, (w+1) seg) and records the kept set as ballot words.
     const int seg = ((T + SWARPS - 1) / SWARPS + 31) & ~31;
     const int wb = warp * seg, we = min(T, wb + seg);
-    int kept = 0;
-    for (int j0 = wb; j0 < we; j0 += 32) {
-        const int j = j0 + lane;
-        bool is_kept = false, is_band = false;
-        if (j < we) {
-            const float v = xs[j];
-            is_kept = v > hi_f;
-            is_band = exact || (v >= lo_f && v <= hi_f);
+    auto classify = [&]() -> int {  // the kept words and the band list; returns #kept
+        int kept = 0;
+        for (int j0 = wb; j0 < we; j0 += 32) {
+            const int j = j0 + lane;
+            bool is_kept = false, is_band = false;
+            if (j < we) {
+                const float v = xs[j];
+                is_kept = v > hi_f;
+                is_band = exact || (v >= lo_f && v <= hi_f);
+            }
+            const unsigned int word = __ballot_sync(0xffffffffu, is_kept);
+            if (lane == 0) kept_words[j0 >> 5] = word;
+            kept += __popc(word);
+            if (is_band) {
+                const int slot = atomicAdd(&nband, 1);
+                if (slot < BAND_CAP) band_j[slot] = j;
+            }
         }
-        const unsigned int word = __ballot_sync(0xffffffffu, is_kept);
-        if (lane == 0) kept_words[j0 >> 5] = word;
-        kept += __popc(word);
-        if (is_band) {
-            const int slot = atomicAdd(&nband, 1);
-            if (slot < BAND_CAP) band_j[slot] = j;
-        }
-    }
-    if (lane == 0) wcnt[warp] = kept;
-    __syncthreads();
-    int kept_all = 0;
+        if (lane == 0) wcnt[warp] = kept;
+        __syncthreads();
+        int kept_all = 0;
 #pragma unroll
-    for (int w = 0; w < SWARPS; ++w) kept_all += wcnt[w];
-    const int need = k - kept_all;  // >= 1: fewer than k approximate scores exceed the bracket
-    const int nb = nband;
+        for (int w = 0; w < SWARPS; ++w) kept_all += wcnt[w];
+        return kept_all;
+    };
+    int kept_all = classify();
+    int nb = nband;
+    // The bracket guarantees 1 <= k - #kept <= #band.  Should that ever fail for a row,
+    // the row is classified again with every tile in the band: the exact fp64 path.
+    if (!(k - kept_all >= 1 && k - kept_all <= nb)) {
+        __syncthreads();  // every thread has read nband and wcnt
+        if (tid == 0) nband = 0;
+        __syncthreads();
+        exact = true;
+        lo_f = -INFINITY;
+        hi_f = INFINITY;
+        kept_all = classify();
+        nb = nband;
+    }
+    const int need = k - kept_all;
 
     if (nb <= BAND_CAP) {
         // ---- narrow band: fp64 scores (one warp per tile: lane l takes d = 2l, 2l + 1,
