@@ -193,6 +193,19 @@ def hbm_isolated(fns: dict, device, local_rank: int, seconds: float = 0.5) -> di
     return {"ms": out, "clocks": clk}
 
 
+def cpu_model() -> str:
+    """The host CPU's model name (from /proc/cpuinfo), for the CPU baseline's record."""
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.lower().startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    import platform
+    return platform.processor() or "unknown"
+
+
 # --------------------------------------------------------------- CPU oracle ----
 def oracle_sample(w, Q, K, V, calib_tiles, sample_tiles=4, calib_rows=16, head=0):
     """Time the fp64 oracle on a bounded sample of one head and extrapolate.
@@ -287,7 +300,8 @@ def run_reference(args, w):
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": t * 1e3, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
             "config": config_dict(w),
-            "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle", "sample": desc},
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "cpu_model": cpu_model(), "kind": "oracle",
+                             "sample": desc},
             "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
     return 0
@@ -632,7 +646,7 @@ def main():
     for ev in events:
         for i, n in enumerate(names):
             per[n].append(ev[i].elapsed_time(ev[i + 1]) / 1e3)
-    kt = {n: statistics.mean(v) for n, v in per.items()}
+    kt = {n: statistics.median(v) for n, v in per.items()}  # median over the timed steps
 
     peaks = measured_peaks()
     idx_cpu = layer.idx.cpu().numpy()
@@ -850,7 +864,8 @@ def main():
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu:
         t_cpu, desc, cores = oracle_sample(w, Q, K, V, calib)
-        cpu = {"value": tokens_per_step / t_cpu / 1e6, "unit": UNIT, "cores": cores, "kind": "oracle",
+        cpu = {"value": tokens_per_step / t_cpu / 1e6, "unit": UNIT, "cores": cores, "cpu_model": cpu_model(),
+               "kind": "oracle",
                "sample": desc}
 
     # read-only HBM stream rate (a second denominator for the HBM-bound kernels)
