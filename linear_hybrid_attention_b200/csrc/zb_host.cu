@@ -103,7 +103,7 @@ zb_status make_map_bf16_3d(CUtensorMap* map, const void* base, int inner, long l
 
 using namespace zb;
 
-extern "C" int32_t zb_abi_version(void) { return 100; }
+extern "C" int32_t zb_abi_version(void) { return 101; }
 
 extern "C" const char* zb_status_string(int32_t status) {
     switch (status) {

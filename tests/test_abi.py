@@ -41,7 +41,7 @@ def test_every_declared_symbol_is_exported(lib):
 
 
 def test_version_and_status_strings(lib):
-    assert lib.zb_abi_version() == 100
+    assert lib.zb_abi_version() == 101  # 1.1: zb_dense_attn_split, the int8 selection's workspace
     for code, name in [(0, "ZB_OK"), (2, "ZB_ERR_SHAPE"), (7, "ZB_ERR_TIMEOUT"), (9, "ZB_ERR_INDEX")]:
         assert lib.zb_status_string(code).decode().startswith(name)
     assert b"unknown" in lib.zb_status_string(1234)
