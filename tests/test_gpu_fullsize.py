@@ -138,3 +138,24 @@ def test_selection_1024_views_every_row_of_one_head():
     ref = oracle.select_tiles(oracle.tile_scores(Qb, Kb), w.k)[0]
     bad = np.flatnonzero((got != ref).any(-1))
     assert bad.size == 0, (bad.size, bad[:5])
+
+
+def test_selection_1024_views_keep20_every_row_of_one_head():
+    """The pages' keep-20% budget (k = 2,199 of 10,992) on head 11 at 1,024 views: every
+    query tile's selected set equals the oracle's."""
+    import linear_hybrid_attention_b200 as zb
+    w = workload("views1024")
+    k20 = -(-w.n_tiles // 5)
+    Q, K, V = synth.make_qkv(w, device="cuda")
+    h = 11
+    lm = zb.zb_landmark_build(Q[h:h + 1].contiguous(), K[h:h + 1].contiguous(), V[h:h + 1].contiguous(), w.tile)
+    idx = zb.zb_tile_score_topk(lm.Qbar, lm.Kbar, w.n_tokens, w.tile, k20)
+    sync_ok()
+    got = idx.cpu().numpy()[0]
+    del lm, idx
+    Qb = oracle.landmark_means(host(Q[h:h + 1]), w.tile)
+    Kb = oracle.landmark_means(host(K[h:h + 1]), w.tile)
+    del Q, K, V
+    ref = oracle.select_tiles(oracle.tile_scores(Qb, Kb), k20)[0]
+    bad = np.flatnonzero((got != ref).any(-1))
+    assert bad.size == 0, (bad.size, bad[:5])

@@ -192,3 +192,17 @@ def test_selection_non_finite_rows_give_valid_sets():
     ref = oracle.select_tiles(oracle.tile_scores(Qb[:1], Kb[:1]), k)
     rows = np.arange(T) != 17
     assert np.array_equal(got[0, rows], ref[0, rows])
+
+
+@pytest.mark.parametrize("seed", [101, 202, 303, 404, 505, 606, 707, 808])
+def test_selection_every_row_of_the_32_view_stage_many_seeds(seed):
+    # 16 heads x 344 query tiles per seed, every row against the oracle
+    import linear_hybrid_attention_b200 as zb
+    w = workload("views32")
+    Q, K, V = synth.make_qkv(w, device="cuda", seed=seed)
+    lm = zb.zb_landmark_build(Q, K, V, w.tile)
+    idx = zb.zb_tile_score_topk(lm.Qbar, lm.Kbar, w.n_tokens, w.tile, w.k)
+    sync_ok()
+    ref = oracle.select_tiles(oracle.tile_scores(oracle.landmark_means(host(Q), w.tile),
+                                                 oracle.landmark_means(host(K), w.tile)), w.k)
+    assert np.array_equal(idx.cpu().numpy().astype(np.int64), ref)
