@@ -23,16 +23,16 @@
 //    of both rows < 64 (2^22) = 2^28; dropped digit products <= 64 * 127^2 *
 //    (2^7 + 2^7 + 1) < 2^28; fp32 rounding of the combination <= 2^10.1 times a
 //    scale <= 2^14; the fp64 dot product's own error <= 64 u 2^48 < 4.
-//  * select_kernel (one CTA per query row): a 4,096-bin linear histogram of
-//    s~ over [min, max] brackets the k-th largest s~ between L and U; key
-//    tiles with s~ > U + 2E are certainly kept, those with s~ < L - 2E
-//    certainly dropped.  The few in the band between are re-scored with one
-//    fp64 FMA chain over d in index order and ranked by (score, index); the
+//  * select_kernel (one CTA of 256 threads per query row, four per SM): a
+//    2,048-bin linear histogram of s~ over [min, max] brackets the k-th largest
+//    s~ between L and U; key tiles with s~ > U + 2E are certainly kept, those
+//    with s~ < L - 2E certainly dropped.  The few in the band between are
+//    re-scored in fp64 (one warp per tile) and ranked by (score, index); the
 //    band's top (k - #kept) join the kept set, which is written ascending.
 //    With tau the k-th largest s~ (L <= tau <= U): a tile ranked above a kept
 //    one has s~ > U, and at most k - 1 tiles do; each of the >= k tiles with
 //    s~ >= tau ranks above a dropped one.  So the result is the fp64
-//    selection whatever the band holds.  Rows whose band exceeds 512
+//    selection whatever the band holds.  Rows whose band exceeds 128
 //    entries (ties, constant rows) resolve it with a radix select over the
 //    fp64 keys, re-scoring band tiles in every pass; rows of heads with a
 //    non-finite value treat every tile as band.
@@ -352,10 +352,11 @@ score_i8_kernel(const int8_t* __restrict__ qd, const int8_t* __restrict__ kd, co
 // ------------------------------------------------------------ select ----
 constexpr int STHREADS = 256;
 constexpr int SWARPS = STHREADS / 32;
-constexpr int NBINS = 4096;
+constexpr int NBINS = 2048;
 constexpr int BPT = NBINS / STHREADS;  // bins per thread in the bucket search
-constexpr int BAND_CAP = 512;
-constexpr int DIGIT = 12;              // radix digit of the fp64 keys in a wide band
+constexpr int BAND_CAP = 128;
+constexpr int DIGIT = 11;              // radix digit of the fp64 keys in a wide band
+static_assert((1 << DIGIT) <= NBINS, "a radix digit's buckets must fit the histogram");
 static_assert(BPT * STHREADS == NBINS, "bins per thread");
 
 // Block-wide exclusive prefix sum of one int per thread.
@@ -441,16 +442,15 @@ ZB_DEVINL int lin_bin(float v, float a, float c) {
 }
 
 // grid: heads in group x T query rows.
-__global__ void __launch_bounds__(STHREADS, 3)
+__global__ void __launch_bounds__(STHREADS, 4)
 select_kernel(const float* __restrict__ scores, const double* __restrict__ Qbar, const double* __restrict__ Kbar,
               const int* __restrict__ qe, const int2* __restrict__ hinfo, int T, int Tp, int k, int h0,
               int32_t* __restrict__ idx) {
-    extern __shared__ __align__(16) float xs[];  // the row's approximate scores, then the band's marks
+    extern __shared__ __align__(16) float xs[];  // the row's approximate scores; then the kept words
     __shared__ unsigned int hist[NBINS];
     __shared__ int band_j[BAND_CAP];
     __shared__ unsigned long long band_key[BAND_CAP];
     __shared__ double qrow[HD];
-    __shared__ unsigned int kept_words[MAX_T / 32];
     __shared__ int wcnt[SWARPS], scratch[SWARPS];
     __shared__ float red_mn[SWARPS], red_mx[SWARPS];
     __shared__ int nband, sel_bucket, sel_above;
@@ -460,6 +460,7 @@ select_kernel(const float* __restrict__ scores, const double* __restrict__ Qbar,
     const float* grow = scores + (static_cast<long long>(hl) * T + i) * Tp;
     const double* kh = Kbar + h * T * HD;
     const int T4 = (T + 3) >> 2;
+    unsigned int* kept_words = reinterpret_cast<unsigned int*>(xs + 4 * T4);
 
     float mn = INFINITY, mx = -INFINITY;
     for (int q = tid; q < T4; q += STHREADS) {
@@ -716,7 +717,7 @@ extern "C" zb_status zb_tile_score_topk(const double* Qbar, const double* Kbar, 
     if ((e = current_device(&dev)) != ZB_OK) return e;
     int per_pass = static_cast<int>(ws_bytes / one < static_cast<size_t>(s.heads) ? ws_bytes / one : s.heads);
     const int Tp = static_cast<int>((T + topk::GTILE - 1) / topk::GTILE) * topk::GTILE;
-    const size_t ssmem = static_cast<size_t>((T + 3) / 4) * 16;
+    const size_t ssmem = static_cast<size_t>((T + 3) / 4) * 16 + static_cast<size_t>((T + 31) / 32) * 4;
     if (cudaFuncSetAttribute(topk::score_i8_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              static_cast<int>(topk::GEMM_SMEM)) != cudaSuccess ||
         cudaFuncSetAttribute(topk::select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
