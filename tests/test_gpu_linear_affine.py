@@ -33,7 +33,7 @@ def test_linear_state_matches_oracle(heads, n):
     np.testing.assert_allclose(z.cpu().numpy(), z_ref, rtol=5e-3)
 
 
-@pytest.mark.parametrize("heads,n,affine", [(2, 256, False), (3, 5000, True), (16, 43968, True)])
+@pytest.mark.parametrize("heads,n,affine", [(2, 256, False), (3, 5000, True), (2, 1000, True), (16, 43968, True)])
 def test_linear_attention_matches_oracle(heads, n, affine):
     zb = _zb()
     w = workload("linear256", heads=heads, n_tokens=n)
