@@ -420,7 +420,7 @@ constexpr int AP_THREADS = 448;
 constexpr int D_BUFS = 4;
 constexpr int BN_ROWS = 80;  // 64 columns of S A, one of z, 15 of zeros
 constexpr uint32_t B_BYTES = BN_ROWS * 128;
-constexpr int PHI_BAR = 1;   // named barrier of the operand builders (warps 4..7, 128 threads)
+constexpr int PHI_BAR = 1;   // named barrier of the operand builders (warps 2..5, 128 threads)
 constexpr int PHI_THREADS = 128;  // warps 2..5 apply phi
 constexpr int EPI_BAR = 2;        // named barrier of the epilogue warps (256 threads)
 constexpr int EPI_THREADS = 256;
@@ -548,14 +548,11 @@ linear_apply_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
         // ======================================= phi and per-head operands ====
         // Every thread runs every iteration (after an abort it skips the waits
         // and the work but keeps the builders' named barriers matched).
-        const int t = tid - 64;           // builder index (warps 2..5)
-        const int tp = tid - 64;          // phi index (warps 2..5)
-        const bool builder = true;
+        const int t = tid - 64;           // builder and phi index (warps 2..5)
         int h_prev = -1, nb = -1;
         bool ok = true;
         for (int it = 0; it < cnt; ++it) {
             const int h = head_of(it);
-            if (h != h_prev && !builder) h_prev = h;
             if (h != h_prev) {
                 ++nb;
                 h_prev = h;
@@ -634,12 +631,12 @@ linear_apply_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                 uint4 v[PER];
 #pragma unroll
                 for (int u = 0; u < PER; ++u) {
-                    const int c = tp + u * PHI_THREADS;
+                    const int c = t + u * PHI_THREADS;
                     if (c < TILE * 8) v[u] = *reinterpret_cast<const uint4*>(qt + c * 16);
                 }
 #pragma unroll
                 for (int u = 0; u < PER; ++u) {
-                    const int c = tp + u * PHI_THREADS;
+                    const int c = t + u * PHI_THREADS;
                     if (c < TILE * 8) {
                         *reinterpret_cast<uint4*>(qt + c * 16) = make_uint4(phi_bf16x2(v[u].x), phi_bf16x2(v[u].y),
                                                                             phi_bf16x2(v[u].z), phi_bf16x2(v[u].w));
