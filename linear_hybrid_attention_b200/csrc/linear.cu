@@ -156,13 +156,16 @@ __device__ __forceinline__ void linear_state_body(const CUtensorMap& tm_k, const
     float z0[8], z1[8];
 #pragma unroll
     for (int e = 0; e < 8; ++e) z0[e] = z1[e] = 0.f;
-    // the shifts of this thread's 8 features in both heads
-    float mu[2][8];
+    // the shifts of this thread's 8 features in both heads, as fp32 pairs
+    uint64_t mu2[2][4];
 #pragma unroll
-    for (int e = 0; e < 8; ++e) {
-        mu[0][e] = CENTERED ? __ldg(key_shift + h0 * HD + cg * 8 + e) : 0.f;
-        mu[1][e] = CENTERED ? __ldg(key_shift + h1 * HD + cg * 8 + e) : 0.f;
+    for (int e = 0; e < 4; ++e) {
+        mu2[0][e] = CENTERED ? f2_pack(__ldg(key_shift + h0 * HD + cg * 8 + 2 * e), __ldg(key_shift + h0 * HD + cg * 8 + 2 * e + 1))
+                             : f2_pack(0.f, 0.f);
+        mu2[1][e] = CENTERED ? f2_pack(__ldg(key_shift + h1 * HD + cg * 8 + 2 * e), __ldg(key_shift + h1 * HD + cg * 8 + 2 * e + 1))
+                             : f2_pack(0.f, 0.f);
     }
+    const uint64_t log2e2 = f2_pack(1.4426950408889634f, 1.4426950408889634f);
     bool ok = true;
     int consumed = 0;  // loads whose full barrier was waited on
 
@@ -181,19 +184,22 @@ __device__ __forceinline__ void linear_state_body(const CUtensorMap& tm_k, const
                 for (int m = 0; m < TILE / (ST_THREADS / 8); ++m) {
                     const int r = rbase + (ST_THREADS / 8) * m;
                     uint4* p = reinterpret_cast<uint4*>(kt + r * 128 + ((cg ^ (r & 7)) << 4));
-                    uint4 v = *p;
+                    const uint4 v = *p;
                     uint32_t w[4] = {v.x, v.y, v.z, v.w};
                     const bool valid = row0 + r < n;
 #pragma unroll
                     for (int e = 0; e < 4; ++e) {
-                        float xa = bf16_lo(w[e]), xb = bf16_hi(w[e]);
-                        if constexpr (CENTERED) {
-                            xa -= mu[hh][2 * e];
-                            xb -= mu[hh][2 * e + 1];
-                        }
-                        const float a = valid ? phi(xa) : 0.f;
-                        const float b = valid ? phi(xb) : 0.f;
-                        w[e] = pack_bf16x2(a, b);
+                        uint64_t x2 = f2_pack(bf16_lo(w[e]), bf16_hi(w[e]));
+                        if constexpr (CENTERED) x2 = f2_sub(x2, mu2[hh][e]);
+                        float xa, xb;
+                        f2_unpack(x2, xa, xb);
+                        // phi(x) = max(x, 0) + 2^(min(x, 0) log2 e), where x - max(x, 0)
+                        // is min(x, 0) exactly
+                        const uint64_t pos = f2_pack(fmaxf(xa, 0.f), fmaxf(xb, 0.f));
+                        float na, nb, a, b;
+                        f2_unpack(f2_mul(f2_sub(x2, pos), log2e2), na, nb);
+                        f2_unpack(f2_add(pos, f2_pack(ex2(na), ex2(nb))), a, b);
+                        w[e] = valid ? pack_bf16x2(a, b) : 0u;
                         // z sums the bf16-rounded features that the MMA uses
                         if (hh == 0) { z0[2 * e] += bf16_lo(w[e]); z0[2 * e + 1] += bf16_hi(w[e]); }
                         else { z1[2 * e] += bf16_lo(w[e]); z1[2 * e + 1] += bf16_hi(w[e]); }
