@@ -582,6 +582,10 @@ def main():
 
     def run_step(L, q, k, v, ev=None):
         """One pass of the hot path on (q, k, v) with the buffers of HybridLayer L."""
+        run_sparse_stage(L, q, k, v, ev)
+        run_linear_stage(L, q, k, v, ev)
+
+    def run_sparse_stage(L, q, k, v, ev=None):
         def mark(i):
             if ev is not None:
                 ev[i].record(stream)
@@ -593,6 +597,11 @@ def main():
         zb.zb_tile_sparse_attn(q, k, v, L.lm.Kbar_bf16, L.lm.Vbar_bf16, L.idx, w.k, w.tile, True,
                                L.scale, out=L.O_sparse, ws=L.ws_attn)
         mark(3)
+
+    def run_linear_stage(L, q, k, v, ev=None):
+        def mark(i):
+            if ev is not None:
+                ev[i].record(stream)
         zb.zb_linear_state(k, v, L.S, L.z, L.ws_lin)
         mark(4)
         zb.zb_gather_tiles(q, w.tile, L.calib, out=L.Qc)
@@ -813,6 +822,7 @@ def main():
 
         def pipelined(n):
             in_ready = [torch.cuda.Event() for _ in range(n)]
+            lin_done = [torch.cuda.Event() for _ in range(n)]
             done = [torch.cuda.Event() for _ in range(n)]
             out_done = [torch.cuda.Event() for _ in range(n)]
             cin.wait_stream(stream)
@@ -832,12 +842,18 @@ def main():
                 stream.wait_event(in_ready[s_])
                 if s_ >= 2:
                     stream.wait_event(out_done[s_ - 2])        # layers[b]'s outputs are out
-                run_step(layers[b_], *din[b_])
+                # the linear stage first, so that its output moves out while the
+                # sparse stage computes and only the sparse output is left to drain
+                run_linear_stage(layers[b_], *din[b_])
+                lin_done[s_].record(stream)
+                cout.wait_event(lin_done[s_])
+                with torch.cuda.stream(cout):
+                    outs[1].copy_(layers[b_].O_linear, non_blocking=True)
+                run_sparse_stage(layers[b_], *din[b_])
                 done[s_].record(stream)
                 cout.wait_event(done[s_])
                 with torch.cuda.stream(cout):
                     outs[0].copy_(layers[b_].O_sparse, non_blocking=True)
-                    outs[1].copy_(layers[b_].O_linear, non_blocking=True)
                     out_done[s_].record(cout)
             stream.wait_event(out_done[n - 1])
 
@@ -856,7 +872,8 @@ def main():
                "d2h_bytes_per_step": 2 * tensor_bytes, "steps": e2e_steps,
                "api": "HybridLayer C-ABI calls; every step's Q, K, V copied in from pinned host memory and both "
                       "outputs copied back inside the timed region, pipelined: the next step's inputs and the "
-                      "previous step's outputs move on two copy streams while a step computes",
+                      "previous step's outputs move on two copy streams while a step computes (each step runs "
+                      "its linear stage first, whose output then moves out during the sparse stage)",
                "serial_value": serial_tput / 1e6,
                "serial_note": "the same with every copy on the compute stream, no overlap"}
         del pin, outs, layer2, layers, din
