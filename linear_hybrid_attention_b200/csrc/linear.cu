@@ -665,6 +665,7 @@ linear_apply_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
         const uint32_t lane_addr = static_cast<uint32_t>((warp & 3) * 32) << 16;
         int h_prev = -1, nb = -1;
         bool ok = true;
+        uint64_t bv2[16];  // this thread's 32 bias values (columns 32 hf ..), as fp32 pairs
         for (int it = 0; it < cnt; ++it) {
             const long long item = first + it;
             const int h = static_cast<int>(item / Tn), t = static_cast<int>(item % Tn);
@@ -673,6 +674,14 @@ linear_apply_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                 ++nb;
                 h_prev = h;
                 if (ok && !mbar_wait(smem_addr(&sm.bvec_ready[nb & 1]), (nb >> 1) & 1, wc)) ok = false;
+                if (ok) {
+                    const uint2* bsrc = reinterpret_cast<const uint2*>(sm.bvec[nb & 1]) + 16 * hf;
+#pragma unroll
+                    for (int q = 0; q < 16; ++q) {
+                        const uint2 v = bsrc[q];
+                        bv2[q] = f2_pack(__uint_as_float(v.x), __uint_as_float(v.y));
+                    }
+                }
             }
             const int d = it % D_BUFS, ob = it & 1;
             const uint32_t du = static_cast<uint32_t>(it / D_BUFS);
@@ -691,19 +700,16 @@ linear_apply_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                 tc_fence_before();
                 mbar_arrive(smem_addr(&sm.d_free[d]));
                 const float inv = 1.f / __uint_as_float(den);
-                const float* bb = sm.bvec[nb & 1];
                 uint8_t* orow = sm.ost[ob] + row * 128;
                 const uint64_t inv2 = f2_pack(inv, inv);
-                const uint2* bb2 = reinterpret_cast<const uint2*>(bb);
 #pragma unroll
                 for (int cc = 0; cc < 4; ++cc) {
                     const int c = 4 * hf + cc;
                     uint32_t pk[4];
 #pragma unroll
                     for (int e = 0; e < 4; ++e) {
-                        const uint2 bv = bb2[c * 4 + e];
                         const uint64_t o2 = f2_fma(f2_pack(__uint_as_float(r[cc * 8 + 2 * e]), __uint_as_float(r[cc * 8 + 2 * e + 1])),
-                                                   inv2, f2_pack(__uint_as_float(bv.x), __uint_as_float(bv.y)));
+                                                   inv2, bv2[cc * 4 + e]);
                         float o0, o1;
                         f2_unpack(o2, o0, o1);
                         pk[e] = pack_bf16x2(o0, o1);
