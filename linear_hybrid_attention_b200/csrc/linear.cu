@@ -13,7 +13,8 @@
 // Both passes stream HBM once and put the d x d products on tcgen05:
 //  * state: one CTA per (head pair, token chunk).  A 128-token step loads K
 //    and V of two heads by TMA, applies phi to K in place (shared memory, same
-//    swizzled layout) while summing z, and issues
+//    swizzled layout; fp32 arithmetic on packed pairs, rounded to bf16) while
+//    summing z, and issues
 //        D[128 x 128] += [phi(K_h0)^T ; phi(K_h1)^T] . [V_h0 | V_h1]
 //    (both operands MN-major); the diagonal 64 x 64 blocks are S_h0, S_h1.
 //    Per-CTA partials are added in a fixed order by a second kernel.
