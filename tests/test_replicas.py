@@ -72,24 +72,25 @@ def _head_worker(rank, world, port, heads, q):
     dist.destroy_process_group()
 
 
-@pytest.mark.parametrize("heads", [16, 5])
-def test_head_partition_gathers_the_per_head_results_in_order(heads):
+@pytest.mark.parametrize("heads,world", [(16, 2), (5, 2), (16, 3)])
+def test_head_partition_gathers_the_per_head_results_in_order(heads, world):
     ctx = mp.get_context("spawn")
     q = ctx.Queue()
     port = _free_port()
-    procs = [ctx.Process(target=_head_worker, args=(r, 2, port, heads, q)) for r in range(2)]
+    procs = [ctx.Process(target=_head_worker, args=(r, world, port, heads, q)) for r in range(world)]
     for p in procs:
         p.start()
-    res = sorted((q.get(timeout=120) for _ in range(2)), key=lambda t: t[0])
+    res = sorted((q.get(timeout=120) for _ in range(world)), key=lambda t: t[0])
     for p in procs:
         p.join(120)
         assert p.exitcode == 0
     g = torch.Generator().manual_seed(9)
     full_in = torch.randn(heads, 40, 8, generator=g)
     want = full_in * 2.0 + torch.arange(heads, dtype=torch.float32)[:, None, None]
-    (r0, a0, b0, o0), (r1, a1, b1, o1) = res
-    assert (a0, b1) == (0, heads) and b0 == a1                 # the blocks tile the heads
-    assert torch.equal(o0, want) and torch.equal(o1, want)
+    assert res[0][1] == 0 and res[-1][2] == heads                     # the blocks tile the heads
+    assert all(res[r][2] == res[r + 1][1] for r in range(world - 1))
+    for _, _, _, out in res:
+        assert torch.equal(out, want)
 
 
 def test_head_range_balanced():
