@@ -584,6 +584,33 @@ class HybridLayer:
             self._state(K, V)
         return zb_linear_apply(Q, self.S, self.z, self.A, self.b, out=self.O_linear)
 
+    def save_fit(self, path) -> None:
+        """Write the fitted (A, b) of this layer's linear stage to an ``.npz`` file.
+
+        (A, b) is the only state a stage keeps between inputs: a fit made once
+        offline on calibration rows serves every later input of the layer.
+        """
+        import numpy as np
+        np.savez(path, A=self.A.detach().cpu().numpy(), b=self.b.detach().cpu().numpy(),
+                 heads=self.heads, head_dim=self.d, centered=self.centered)
+
+    def load_fit(self, path) -> None:
+        """Read (A, b) written by ``save_fit`` into this layer; ``linear(Q, K, V,
+        refresh_state=True)`` then runs the linear stage with it, no calibration."""
+        import numpy as np
+        with np.load(path) as f:
+            A, b = f["A"], f["b"]
+            heads, head_dim, centered = int(f["heads"]), int(f["head_dim"]), bool(f["centered"])
+        if (heads, head_dim) != (self.heads, self.d) or A.shape != tuple(self.A.shape) or \
+                b.shape != tuple(self.b.shape) or A.dtype != np.float32 or b.dtype != np.float32:
+            raise ValueError(f"fit in {path} is for {heads} heads x d = {head_dim} with A {A.shape} "
+                             f"{A.dtype}, b {b.shape}; this layer has {self.heads} heads x d = {self.d}")
+        if centered != self.centered:
+            raise ValueError(f"fit in {path} was made for centered={centered}, this layer has "
+                             f"centered={self.centered}")
+        self.A.copy_(torch.from_numpy(A))
+        self.b.copy_(torch.from_numpy(b))
+
     def step(self, Q, K, V):
         """One pass of the whole hot path: both stage types on the same input."""
         o_s = self.sparse(Q, K, V)
