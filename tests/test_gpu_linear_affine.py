@@ -267,3 +267,23 @@ def test_fitted_linear_stage_full_256_views_sampled():
         srows, want = ref[slot]
         got = host(o_l[h:h + 1, srows])[0]
         check_close(got[None], want[None], label=f"head {h}")
+
+
+def test_saved_fit_reproduces_the_linear_stage_on_new_inputs(tmp_path):
+    """A fit saved by one layer and loaded by another gives the same linear output on a new
+    input, bit for bit, with no calibration in the second layer."""
+    zb = _zb()
+    w = workload("linear256", heads=2, n_tokens=5000)
+    Q, K, V = synth.make_qkv(w, device="cuda")
+    calib = synth.calibration_tiles(w.n_tiles, 4)
+    first = zb.HybridLayer(w.heads, w.n_tokens, w.tile, 1, calib)
+    first.calibrate(Q, K, V)
+    path = tmp_path / "fit.npz"
+    first.save_fit(path)
+    Q2, K2, V2 = synth.make_qkv(w, layer=1, device="cuda")   # another input of the same shape
+    want = first.linear(Q2, K2, V2, refresh_state=True).clone()
+    second = zb.HybridLayer(w.heads, w.n_tokens, w.tile, 1, calib)
+    second.load_fit(path)
+    got = second.linear(Q2, K2, V2, refresh_state=True)
+    sync_ok()
+    assert torch.equal(got, want)
