@@ -331,7 +331,7 @@ def block_mass(Q, K, scale: float, block: int) -> np.ndarray:
     p_rc, p = softmax over all keys of scale * q_r . k_c.  Blocks are runs of
     ``block`` tokens in sequence order, the last one ragged (the tiling of
     ``tile_lengths``).  The pages measure this with 64 x 64 token blocks on a
-    dense pass to judge how concentrated attention is ([ABS]'s page, Figure 2
+    dense pass to show how concentrated attention is ([ABS]'s page, Figure 2
     (b) and Figure 8: mass kept by the heaviest 20% of 64 x 64 blocks).
     """
     Q, K = _f64(Q), _f64(K)
