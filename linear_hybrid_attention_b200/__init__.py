@@ -597,7 +597,11 @@ class HybridLayer:
     def load_fit(self, path) -> None:
         """Read (A, b) written by ``save_fit`` into this layer; ``linear(Q, K, V,
         refresh_state=True)`` then runs the linear stage with it, no calibration."""
+        import os
         import numpy as np
+        path = os.fspath(path)
+        if not os.path.exists(path) and os.path.exists(path + ".npz"):
+            path += ".npz"  # numpy's savez adds the suffix when the name has none
         with np.load(path) as f:
             A, b = f["A"], f["b"]
             heads, head_dim, centered = int(f["heads"]), int(f["head_dim"]), bool(f["centered"])

@@ -42,3 +42,13 @@ def test_load_rejects_a_fit_of_the_other_variant(tmp_path):
     _layer(centered=True).save_fit(path)
     with pytest.raises(ValueError):
         _layer().load_fit(path)
+
+
+def test_a_name_without_the_suffix_works_both_ways(tmp_path):
+    a = _layer()
+    a.A.fill_(0.5)
+    a.b.fill_(-1.0)
+    a.save_fit(tmp_path / "fit")          # numpy writes fit.npz
+    b = _layer()
+    b.load_fit(tmp_path / "fit")
+    assert torch.equal(a.A, b.A) and torch.equal(a.b, b.b)
