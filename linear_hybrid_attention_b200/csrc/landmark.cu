@@ -102,8 +102,23 @@ landmark_kernel(const uint16_t* __restrict__ Q, const uint16_t* __restrict__ K,
                 }
                 const int lo_min = (mn >> 7) & 0xFF, lo_max = (mx >> 7) & 0xFF;
                 const int hi_min = (mn >> 23) & 0xFF, hi_max = (mx >> 23) & 0xFF;
-                acc[2 * e] += quad_sum_lo(x[0][e], x[1][e], x[2][e], x[3][e], lo_min > 0 && lo_max - lo_min <= 14);
-                acc[2 * e + 1] += quad_sum_hi(x[0][e], x[1][e], x[2][e], x[3][e], hi_min > 0 && hi_max - hi_min <= 14);
+                const bool lo_ok = lo_min > 0 && lo_max - lo_min <= 14;
+                const bool hi_ok = hi_min > 0 && hi_max - hi_min <= 14;
+                if (lo_ok && hi_ok) {
+                    // both columns exact in fp32: one packed fp32x2 chain (the same
+                    // additions in the same order as quad_sum_lo / quad_sum_hi)
+                    const uint64_t ab = f2_add(f2_pack(bf16_lo(x[0][e]), bf16_hi(x[0][e])),
+                                               f2_pack(bf16_lo(x[1][e]), bf16_hi(x[1][e])));
+                    const uint64_t cd = f2_add(f2_pack(bf16_lo(x[2][e]), bf16_hi(x[2][e])),
+                                               f2_pack(bf16_lo(x[3][e]), bf16_hi(x[3][e])));
+                    float slo, shi;
+                    f2_unpack(f2_add(ab, cd), slo, shi);
+                    acc[2 * e] += static_cast<double>(slo);
+                    acc[2 * e + 1] += static_cast<double>(shi);
+                } else {
+                    acc[2 * e] += quad_sum_lo(x[0][e], x[1][e], x[2][e], x[3][e], lo_ok);
+                    acc[2 * e + 1] += quad_sum_hi(x[0][e], x[1][e], x[2][e], x[3][e], hi_ok);
+                }
             }
         }
     }
